@@ -1,0 +1,84 @@
+"""Naive chunkwise form of the KDA recurrence, fp64 NumPy -- TEST INFRASTRUCTURE ONLY.
+
+A second witness for the oracle.  It restates the token recurrence of "Kimi K3:
+Architecture, Training, and Million-Token Agentic RL" (sections 3.1-3.2) as
+whole-chunk matrix products, the form that section 3.3 says chunked prefill
+uses (tokens inside a chunk become matrix operations, the state crosses only
+chunk boundaries: (X_[c], S_in[c]) -> (Y_[c], S_out[c]), S_in[c+1] = S_out[c]).
+The note defers the derivation to a companion note that is not available, so
+it is derived here from the recurrence itself:
+
+Inside one chunk of tokens r = 1..C with incoming state S0, let
+G_r = g_1 + ... + g_r (per key channel; inclusive, because alpha_r decays the
+state before token r edits it).  Unrolling the edit-order step gives
+
+  S_r      = Diag(e^{G_r}) S0 + sum_{s<=r} Diag(e^{G_r - G_s}) k_s d_s^T
+  d_r      = beta_r (v_r - Sbar_r^T k_r)
+           = beta_r (v_r - S0^T (k_r e^{G_r})
+                      - sum_{s<r} <k_r e^{G_r}, k_s e^{-G_s}> d_s)
+
+so with Kt = K*e^{G}, Kh = K*e^{-G}, Qt = Q*e^{G} (row r scaled by e^{G_r}):
+
+  (I + A) D = Diag(beta) (V - Kt S0),   A = strictly_lower(Diag(beta) Kt Kh^T)
+  D        = U - W S0,  U = T Diag(beta) V,  W = T Diag(beta) Kt,  T = (I + A)^-1
+  O        = Qt S0 + lower_incl_diag(Qt Kh^T) D          (read after write)
+  S_out    = Diag(e^{G_C}) S0 + (K * e^{G_C - G})^T D
+
+Library primitives used: matrix products and ``np.linalg.inv``.  In fp64 the
+e^{-G} factors stay finite for chunks up to about 140 tokens (G >= -5 per token).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+G_MIN = -5.0
+
+
+def _gate(z: np.ndarray, A: np.ndarray) -> np.ndarray:
+    """g = g_min * sigmoid(exp(A) * z), section 3.3 gate equation (one head)."""
+    return G_MIN / (1.0 + np.exp(-(np.exp(A) * z)))
+
+
+def chunk_step(q, k, v, g, beta, S0):
+    """One chunk for one head: q, k, g [C,dk]; v [C,dv]; beta [C]; S0 [dk,dv].
+
+    Returns ``(O [C,dv], S_out [dk,dv])``.
+    """
+    C = q.shape[0]
+    G = np.cumsum(g, axis=0)
+    Kt, Kh, Qt = k * np.exp(G), k * np.exp(-G), q * np.exp(G)
+    A = np.tril(beta[:, None] * (Kt @ Kh.T), -1)
+    Tinv = np.linalg.inv(np.eye(C) + A)
+    W = Tinv @ (beta[:, None] * Kt)
+    U = Tinv @ (beta[:, None] * v)
+    D = U - W @ S0
+    O = Qt @ S0 + np.tril(Qt @ Kh.T) @ D
+    S_out = np.exp(G[-1])[:, None] * S0 + (k * np.exp(G[-1] - G)).T @ D
+    return O, S_out
+
+
+def prefill(q, k, v, z, A, beta, cu_seqlens, initial_state=None, chunk: int = 16):
+    """Chunkwise prefill with chunks aligned to each sequence start.
+
+    Same shapes and result as ``oracle.prefill``; every argument is a float64
+    (or int for cu_seqlens) NumPy array.
+    """
+    q, k, v, z, A, beta = (np.asarray(t, dtype=np.float64) for t in (q, k, v, z, A, beta))
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    n = cu.shape[0] - 1
+    o = np.zeros((T, H, dv))
+    sf = np.zeros((n, H, dk, dv))
+    for i in range(n):
+        for h in range(H):
+            S = (np.zeros((dk, dv)) if initial_state is None
+                 else np.asarray(initial_state[i, h], dtype=np.float64).copy())
+            for c0 in range(int(cu[i]), int(cu[i + 1]), chunk):
+                c1 = min(c0 + chunk, int(cu[i + 1]))
+                g = _gate(z[c0:c1, h], A[h])
+                O, S = chunk_step(q[c0:c1, h], k[c0:c1, h], v[c0:c1, h], g,
+                                  beta[c0:c1, h], S)
+                o[c0:c1, h] = O
+            sf[i, h] = S
+    return o, sf
