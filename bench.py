@@ -1,0 +1,374 @@
+"""Benchmark of the KDA mixer on B200: chunked prefill (headline) and decode step.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one kda_prefill call over the 32K-token, 96-head workload
+(B=1, H=96, T=32768, dk=dv=128, bf16 q/k/v/z, fp32 A/beta/state), inputs
+resident in HBM.  Each rank runs its own independent problem (weak scaling, no
+collective on the data path).  Rank 0 prints one JSON line with tokens/s,
+TFLOP/s, the dominant kernel's roofline, the decode-step GB/s (B=256 cached
+states, H=96, in place), an end-to-end figure through the C ABI with pinned
+host buffers, SM clocks sampled during the timed region, and the CPU oracle
+timed on a bounded sample of the same workload.
+
+--impl reference times the CPU oracle itself as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "KDA prefill tokens/s + TFLOP/s (H=96,d=128,T=32K); decode-step GB/s vs HBM peak"
+BYTES_PER_TOKEN_HEAD = 1284        # q,k,v,z bf16 (4*256) + beta fp32 (4) + o bf16 (256)
+FLOPS_PER_TOKEN_HEAD = 108544      # 6*dk*dv + 16*(3*dk + 2*dv) at dk = dv = 128
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi during a region."""
+    QUERY = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.bus = None
+        try:
+            p = torch.cuda.get_device_properties(device)
+            self.bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        except Exception:
+            self.bus = None
+
+    def start(self):
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        rows = [r.split(",") for r in self.out.read().strip().splitlines() if r.strip()]
+        os.unlink(self.out.name)
+        mine = [r for r in rows if len(r) >= 10 and self.bus
+                and r[1].strip().upper().endswith(self.bus[-12:].upper())]
+        if not mine and len({r[0] for r in rows if len(r) >= 10}) == 1:
+            mine = [r for r in rows if len(r) >= 10]
+        if not mine:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[2]) for r in mine if r[2].strip().replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in mine if r[3].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in mine for i in range(4)
+                          if r[6 + i].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(mine)}
+
+
+def _source_sha(name: str) -> str:
+    path = os.path.join(ROOT, "linear_attention_serving_prefill_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _traffic(kernel_file: str, units: int):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current source of the kernel; else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel_file)
+    if not rec or rec.get("source_sha") != _source_sha(kernel_file):
+        return None
+    return rec["dram_bytes_per_unit"] * units
+
+
+def cpu_oracle_sample(inp, target_s: float, max_heads: int = 96):
+    """Times the fp64 CPU oracle on a bounded sample of the prefill workload:
+    the first L tokens of the first h heads, L chosen from a short calibration
+    so the timed run takes about target_s seconds.  Returns a dict."""
+    from oracle import oracle
+    cores = oracle.max_threads()
+    h = min(max_heads, inp["q"].shape[1], max(1, cores))
+
+    def sample(L):
+        sl = slice(0, L)
+        args = [inp[key][sl, :h].cpu() for key in ("q", "k", "v", "z")]
+        return args + [inp["A"][:h].cpu(), inp["beta"][sl, :h].cpu(),
+                       torch.tensor([0, L], dtype=torch.int32)]
+
+    cal = sample(128)
+    t0 = time.perf_counter()
+    oracle.prefill(*cal)
+    rate = h * 128 / (time.perf_counter() - t0)          # token-heads / s
+    L = int(max(128, min(inp["q"].shape[0], rate * target_s / h)))
+    args = sample(L)
+    t0 = time.perf_counter()
+    oracle.prefill(*args)
+    dt = time.perf_counter() - t0
+    th_per_s = h * L / dt
+    return {"token_heads_per_s": th_per_s, "tokens_per_s": th_per_s / inp["q"].shape[1],
+            "cores": min(h, cores), "seconds": dt,
+            "sample": f"first {L} tokens x {h} heads of the 32K workload ({h * L} token-heads, "
+                      f"fp64 token-by-token oracle, OpenMP over heads); tokens/s = "
+                      f"token-heads/s / 96 heads"}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle, timed as it stands on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from linear_attention_serving_prefill_b200.workloads import CONFIGS, config_inputs
+    cfg = CONFIGS["prefill_32k"]
+    # Inputs: the same distributions; generate only the rows the sample touches.
+    from linear_attention_serving_prefill_b200.workloads import prefill_inputs
+    per_step = max(2.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    inp = prefill_inputs([2048], cfg.H, cfg.dk, cfg.dv, cfg.dtype, seed=cfg.seed)
+    res = None
+    for _ in range(args.warmup):
+        cpu_oracle_sample(inp, per_step)
+    vals = []
+    for _ in range(args.steps):
+        res = cpu_oracle_sample(inp, per_step)
+        vals.append(res["tokens_per_s"])
+    value = statistics.median(vals) if vals else 0.0
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * res["seconds"] if res else None, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "global_batch": 1, "seq_len": 32768,
+                   "parallelism": "host cores (OpenMP over heads)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": res["cores"] if res else 0,
+                         "kind": "oracle", "sample": res["sample"] if res else ""},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--algo", default="auto", choices=["auto", "cuda_core", "tensor_core"])
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from linear_attention_serving_prefill_b200 import binding as K
+    from linear_attention_serving_prefill_b200.workloads import (CONFIGS, config_inputs,
+                                                                 decode_inputs)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    cfg = CONFIGS["prefill_32k"]
+    from dataclasses import replace
+    inp = config_inputs(replace(cfg, seed=cfg.seed + 1000 * rank), device=dev)
+    T, H, dk, dv = inp["q"].shape[0], cfg.H, cfg.dk, cfg.dv
+    stream = torch.cuda.current_stream()
+    o = torch.empty(T, H, dv, dtype=torch.bfloat16, device=dev)
+    S = torch.empty(1, H, dk, dv, dtype=torch.float32, device=dev)
+    ws_bytes = K.kda_prefill_workspace_size(T, 1, H, dk, dv, torch.bfloat16, args.algo)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+
+    def step():
+        K.kda_prefill(inp["q"], inp["k"], inp["v"], inp["z"], inp["A"], inp["beta"],
+                      inp["cu_seqlens"], inp["cu_seqlens_host"], None, final_state=S, o=o,
+                      workspace=ws, algo=args.algo, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    evs[0].record(stream)
+    for i in range(args.steps):
+        step()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier()
+    torch.cuda.synchronize()
+    per_launch = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
+    total_ms = evs[0].elapsed_time(evs[-1])
+    total_ms = max_over_ranks(total_ms)
+    ms_per_step = total_ms / args.steps
+    tokens = T * world
+    value = tokens / (ms_per_step / 1e3)
+    th = T * H
+    tflops = th * FLOPS_PER_TOKEN_HEAD * world / (ms_per_step / 1e3) / 1e12
+
+    hbm_peak, tc_peak, peak_src = _peaks()
+    # The step is one kernel launch on the CUDA-core path: its event pair is the launch.
+    launch_ms = statistics.mean(per_launch)
+    alg_bytes = th * BYTES_PER_TOKEN_HEAD
+    achieved = alg_bytes / (launch_ms / 1e3) / 1e9
+    kernel_file = "kda_prefill_cuda_core.cu"
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": _traffic(kernel_file, th),
+                "kernel": "prefill_cuda_core_kernel", "peak_source": peak_src,
+                "algorithmic_bytes_per_launch": alg_bytes,
+                "tensor_frac": (th * FLOPS_PER_TOKEN_HEAD / (launch_ms / 1e3) / 1e12) / tc_peak}
+    launches = args.steps
+
+    # Decode step: B=256 cached states, H=96, updated in place; GB/s of state traffic.
+    dcfg = CONFIGS["decode_256"]
+    d = decode_inputs(dcfg.B, dcfg.H, dcfg.dk, dcfg.dv, dcfg.dtype, seed=dcfg.seed + 1000 * rank,
+                      nsets=dcfg.nsets, device=dev)
+    od = torch.empty(dcfg.B, dcfg.H, dcfg.dv, dtype=torch.bfloat16, device=dev)
+
+    def dstep(i):
+        j = i % dcfg.nsets
+        K.kda_decode_step(d["q"][j], d["k"][j], d["v"][j], d["z"][j], d["A"], d["beta"][j],
+                          d["state"], None, o=od, stream=stream)
+
+    for i in range(args.warmup):
+        dstep(i)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.decode_steps):
+        dstep(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dms = max_over_ranks(e0.elapsed_time(e1)) / args.decode_steps
+    state_bytes = 2 * dcfg.B * dcfg.H * dcfg.dk * dcfg.dv * 4
+    dgbs = state_bytes / (dms / 1e3) / 1e9
+    decode = {"config": dcfg.name, "ms_per_step": dms, "state_gbs": dgbs,
+              "frac_of_hbm": dgbs / hbm_peak, "steps": args.decode_steps,
+              "state_bytes_per_step": state_bytes, "gpu_launches": args.decode_steps}
+    del d, od
+
+    # End to end through the C ABI: pinned host inputs -> device, prefill, result -> host.
+    host = {key: inp[key].cpu().pin_memory() for key in ("q", "k", "v", "z", "beta", "A")}
+    host_cu = inp["cu_seqlens_host"].pin_memory()
+    dbuf = {key: torch.empty_like(inp[key]) for key in host}
+    cu_dev = torch.empty_like(inp["cu_seqlens"])
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    S_host = torch.empty(S.shape, dtype=S.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values()) + host_cu.numel() * 4
+    d2h = o_host.numel() * o_host.element_size() + S_host.numel() * 4
+
+    def e2e_step():
+        for key in host:
+            dbuf[key].copy_(host[key], non_blocking=True)
+        cu_dev.copy_(host_cu, non_blocking=True)
+        K.kda_prefill(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["z"], dbuf["A"], dbuf["beta"], cu_dev,
+                      inp["cu_seqlens_host"], None, final_state=S, o=o, workspace=ws,
+                      algo=args.algo, stream=stream)
+        o_host.copy_(o, non_blocking=True)
+        S_host.copy_(S, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ems = max_over_ranks(e0.elapsed_time(e1)) / args.e2e_steps
+    e2e = {"value": tokens / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r = cpu_oracle_sample(inp, args.cpu_seconds)
+        cpu = {"value": r["tokens_per_s"], "unit": "tokens/s", "cores": r["cores"],
+               "kind": "oracle", "sample": r["sample"], "seconds": r["seconds"]}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": cfg.name, "global_batch": world, "seq_len": T, "heads": H,
+                       "dk": dk, "dv": dv, "parallelism": f"dp{world} (one independent problem per GPU)",
+                       "algo": args.algo,
+                       "l2": "inputs larger than L2 (q,k,v,z = 3.2 GB per step), no flush"},
+            "tflops": tflops,
+            "roofline": roofline,
+            "decode": decode,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+            "gpu": torch.cuda.get_device_name(dev),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,159 @@
+/*
+ * kda.h -- C ABI of libkda_b200.so, the B200 (sm_100a) Kimi Delta Attention mixer.
+ *
+ * What the library computes, per head h with a dk x dv fp32 state S
+ * ("Kimi K3: Architecture, Training, and Million-Token Agentic RL", brenchcc
+ * research note):
+ *   - recurrence, section 3.1 equation:
+ *       S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *       o_t = S_t^T q_t            (the read follows the write; no 1/sqrt(dk))
+ *     Diag(alpha_t) scales the ROWS of S, one row per key channel.
+ *   - lower-bounded gate, section 3.3 equation (restated in "Kimi K3 Under the
+ *     Hood", section "Sequence mixing: three KDA layers per global MLA layer"):
+ *       g[t,h,c] = -5 * sigmoid(exp(A[h,c]) * z[t,h,c]),  alpha = exp(g)
+ *   - chunked prefill, section 3.3 chunk I/O equation: tokens inside a chunk
+ *     become matrix products, the state crosses only chunk boundaries,
+ *     S_in[c+1] = S_out[c]; decode follows the recurrence one token at a time
+ *     (section 3.2, (x_t, S_{t-1}) -> (y_t, S_t)).
+ *   - prefix-cache resume ("Kimi K3 Under the Hood", section "Serving two
+ *     incompatible cache types"; brenchcc note section 9): a request copies a
+ *     cached state into its running state and resumes prefill from it -- here
+ *     the optional initial_state / final_state of kda_prefill.
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are dense, row-major, contiguous, on the current CUDA device
+ *     unless stated "host".  T = total packed tokens, N = sequences, H = heads.
+ *       q, k, z : [T, H, dk]   storage dtype `dt`
+ *       v, o    : [T, H, dv]   storage dtype `dt`
+ *       beta    : [T, H]       fp32, expected in [0, 1]
+ *       A       : [H, dk]      fp32 (gate log-scale, one per head and key channel)
+ *       states  : [N or P, H, dk, dv] fp32, dv contiguous (row = key channel)
+ *   - dk, dv in {32, 64, 128}.  Device pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Every call is asynchronous on that stream: it validates arguments on the
+ *     host, enqueues kernels and returns; it never synchronises.
+ *   - Ownership: the caller owns every buffer (inputs, outputs, states and the
+ *     prefill workspace).  The library allocates no device memory, keeps no
+ *     per-call state and may be called from several host threads.
+ *   - Errors: argument checks run before anything is enqueued, and a failing
+ *     check returns its code with nothing launched.  A launch failure returns
+ *     KDA_ERR_CUDA.  NaN / Inf in the data are not detected; they propagate as
+ *     the mathematics says.
+ */
+#ifndef KDA_B200_H
+#define KDA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KDA_ABI_VERSION 1
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, bad cu_seqlens */
+    KDA_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement (e.g. dk=96) */
+    KDA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than kda_prefill_workspace_size */
+    KDA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+    KDA_ERR_TIMEOUT = 5        /* a bounded on-device wait gave up (see kda_device_status) */
+} kda_status;
+
+typedef enum {
+    KDA_DTYPE_BF16 = 0,        /* q, k, v, z, o stored as bfloat16 */
+    KDA_DTYPE_F32 = 1          /* q, k, v, z, o stored as fp32 */
+} kda_dtype;
+
+typedef enum {
+    KDA_ALGO_AUTO = 0,         /* tensor-core path for bf16, CUDA-core fp32 path for fp32 */
+    KDA_ALGO_CUDA_CORE = 1,    /* chunked prefill in fp32 FMA on CUDA cores (check mode) */
+    KDA_ALGO_TENSOR_CORE = 2   /* chunked prefill on tcgen05 tensor cores (bf16 only) */
+} kda_algo;
+
+/* Version of this ABI (KDA_ABI_VERSION of the build). */
+int32_t kda_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *kda_status_string(kda_status s);
+
+/*
+ * Bytes of device workspace kda_prefill needs for these sizes and algorithm.
+ * The value depends only on the arguments (an upper bound over every
+ * cu_seqlens with this total_tokens and num_seqs), so one buffer can be
+ * reused across calls of the same shape.  Returns 0 for invalid arguments.
+ */
+size_t kda_prefill_workspace_size(int32_t total_tokens, int32_t num_seqs, int32_t H,
+                                  int32_t dk, int32_t dv, kda_dtype dt, kda_algo algo);
+
+/*
+ * Chunked prefill over packed variable-length sequences ("Kimi K3:
+ * Architecture, Training, and Million-Token Agentic RL", section 3.3).
+ *
+ * For each sequence n (tokens cu_seqlens[n] .. cu_seqlens[n+1]-1) and head h,
+ * starts from initial_state[n,h] (zeros if initial_state is NULL), writes
+ * o[t,h,:] = S_t^T q_t for every token, and, if final_state is non-NULL, the
+ * state after the sequence's last token into final_state[n,h].  A sequence of
+ * length 0 passes its initial state through.  final_state may equal
+ * initial_state (in-place resume); no other buffers may overlap.
+ *
+ *   cu_seqlens_dev  [N+1] int32, device: 0 = cu[0] <= cu[1] <= ... <= cu[N] = T.
+ *   cu_seqlens_host [N+1] int32, HOST copy of the same offsets, or NULL.  When
+ *                   given it is validated (KDA_ERR_INVALID_ARG if malformed) and
+ *                   used to schedule long sequences first; the device copy is
+ *                   not read on the host.
+ *   workspace       device buffer of at least
+ *                   kda_prefill_workspace_size(T, N, H, dk, dv, dt, algo) bytes
+ *                   (may be NULL when that size is 0); contents are scratch.
+ *   algo            KDA_ALGO_AUTO, or a forced path; KDA_ALGO_TENSOR_CORE with
+ *                   dt = KDA_DTYPE_F32 returns KDA_ERR_UNSUPPORTED.
+ * kda_prefill is kda_prefill_ex with algo = KDA_ALGO_AUTO.
+ */
+kda_status kda_prefill(const void *q, const void *k, const void *v, const void *z,
+                       const float *A, const float *beta,
+                       const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                       int32_t num_seqs, int32_t total_tokens, int32_t H, int32_t dk,
+                       int32_t dv, kda_dtype dt, const float *initial_state,
+                       float *final_state, void *o, void *workspace,
+                       size_t workspace_bytes, void *stream);
+
+kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const void *z,
+                          const float *A, const float *beta,
+                          const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                          int32_t num_seqs, int32_t total_tokens, int32_t H, int32_t dk,
+                          int32_t dv, kda_dtype dt, const float *initial_state,
+                          float *final_state, void *o, void *workspace,
+                          size_t workspace_bytes, kda_algo algo, void *stream);
+
+/*
+ * One recurrent decode step for B sequences, one new token each ("Kimi K3:
+ * Architecture, Training, and Million-Token Agentic RL", section 3.2 edit
+ * order: Sbar = Diag(alpha) S; vhat = Sbar^T k; S = Sbar + beta k (v - vhat)^T;
+ * o = S^T q).
+ *
+ *   q, k, z [B, H, dk], v [B, H, dv], o [B, H, dv] in dtype dt; beta [B, H] fp32.
+ *   state   [P, H, dk, dv] fp32 pool, updated IN PLACE: row slots[b] (or b when
+ *           slots is NULL) holds sequence b's state.  Duplicate slot values are
+ *           a data race (not detected); slot values must lie in [0, P).
+ *   pool_size P >= B when slots is NULL; slots is a device array of B int32.
+ */
+kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *z,
+                           const float *A, const float *beta, int32_t B, int32_t H,
+                           int32_t dk, int32_t dv, kda_dtype dt, float *state,
+                           int32_t pool_size, const int32_t *slots, void *o,
+                           void *stream);
+
+/*
+ * Reads and clears the library's device status word for the current device
+ * (synchronises `stream` first).  Kernels that wait on an on-chip barrier
+ * with an iteration limit record KDA_ERR_TIMEOUT there instead of hanging;
+ * *status_out receives KDA_OK or the first recorded code.
+ */
+kda_status kda_device_status(void *stream, int32_t *status_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_B200_H */

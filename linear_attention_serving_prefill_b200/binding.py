@@ -1,0 +1,154 @@
+"""Thin ctypes binding of libkda_b200.so (argument marshalling only).
+
+Every function here checks tensor placement and dtype, passes raw device
+pointers and sizes to the C ABI declared in ``include/kda.h``, and raises
+``KdaError`` on a non-zero status.  All arithmetic runs in the CUDA library;
+there is no fallback: if the library is missing the import of this module
+fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libkda_b200.so")
+
+KDA_DTYPE = {torch.bfloat16: 0, torch.float32: 1}
+KDA_ALGO = {"auto": 0, "cuda_core": 1, "tensor_core": 2}
+STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
+                3: "KDA_ERR_WORKSPACE", 4: "KDA_ERR_CUDA", 5: "KDA_ERR_TIMEOUT"}
+
+# Every exported symbol of include/kda.h, with its ctypes signature.
+_P, _I32, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+SIGNATURES = {
+    "kda_abi_version": ([], _I32),
+    "kda_status_string": ([_I32], ctypes.c_char_p),
+    "kda_prefill_workspace_size": ([_I32, _I32, _I32, _I32, _I32, _I32, _I32], _SZ),
+    "kda_prefill": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _P], _I32),
+    "kda_prefill_ex": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _I32, _P], _I32),
+    "kda_decode_step": ([_P] * 6 + [_I32] * 5 + [_P, _I32, _P, _P, _P], _I32),
+    "kda_device_status": ([_P, _P], _I32),
+}
+
+
+class KdaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(code, code)} "
+                         f"({_lib.kda_status_string(code).decode()})")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"KDA CUDA library not built: {_LIB_PATH} is missing "
+                          "(run python -m linear_attention_serving_prefill_b200.build)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    for name, (args, res) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.argtypes, fn.restype = args, res
+    return lib
+
+
+_lib = _load()
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def kda_status_string(code: int) -> str:
+    return _lib.kda_status_string(code).decode()
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise KdaError(code, where)
+
+
+def _dev(t: Optional[torch.Tensor], name: str, dtype=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def kda_prefill_workspace_size(total_tokens: int, num_seqs: int, H: int, dk: int, dv: int,
+                               dtype=torch.bfloat16, algo: str = "auto") -> int:
+    return int(_lib.kda_prefill_workspace_size(total_tokens, num_seqs, H, dk, dv,
+                                               KDA_DTYPE[dtype], KDA_ALGO[algo]))
+
+
+def kda_prefill(q, k, v, z, A, beta, cu_seqlens, cu_seqlens_host=None, initial_state=None,
+                output_final_state: bool = True, final_state=None, o=None, workspace=None,
+                algo: str = "auto", stream=None):
+    """Chunked KDA prefill over packed sequences; returns ``(o, final_state)``.
+
+    q, k, z [T,H,dk], v [T,H,dv] (bf16 or fp32, one dtype); A [H,dk] fp32;
+    beta [T,H] fp32; cu_seqlens [N+1] int32 on the device; cu_seqlens_host an
+    optional CPU copy; initial_state [N,H,dk,dv] fp32 or None.  ``final_state``
+    may be passed (e.g. ``initial_state`` itself, for in-place resume);
+    otherwise it is allocated when ``output_final_state``.
+    """
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = cu_seqlens.shape[0] - 1
+    dt = q.dtype
+    if dt not in KDA_DTYPE:
+        raise ValueError(f"unsupported dtype {dt}")
+    if o is None:
+        o = torch.empty(T, H, dv, dtype=dt, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+    need = kda_prefill_workspace_size(T, N, H, dk, dv, dt, algo)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    host = None
+    if cu_seqlens_host is not None:
+        ch = cu_seqlens_host.to(torch.int32).contiguous()
+        host = ctypes.c_void_p(ch.data_ptr())
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    code = _lib.kda_prefill_ex(
+        _dev(q, "q", dt), _dev(k, "k", dt), _dev(v, "v", dt), _dev(z, "z", dt),
+        _dev(A, "A", torch.float32), _dev(beta, "beta", torch.float32),
+        _dev(cu_seqlens, "cu_seqlens", torch.int32), host, N, T, H, dk, dv, KDA_DTYPE[dt],
+        _dev(initial_state, "initial_state", torch.float32),
+        _dev(final_state, "final_state", torch.float32), _dev(o, "o", dt),
+        _dev(workspace, "workspace"), ws_bytes, KDA_ALGO[algo], _stream_ptr(stream))
+    _check(code, "kda_prefill")
+    return o, final_state
+
+
+def kda_decode_step(q, k, v, z, A, beta, state, slots=None, o=None, stream=None):
+    """One decode step; ``state`` [P,H,dk,dv] fp32 is updated in place; returns o."""
+    B, H, dk = q.shape
+    dv = v.shape[2]
+    dt = q.dtype
+    if o is None:
+        o = torch.empty(B, H, dv, dtype=dt, device=q.device)
+    code = _lib.kda_decode_step(
+        _dev(q, "q", dt), _dev(k, "k", dt), _dev(v, "v", dt), _dev(z, "z", dt),
+        _dev(A, "A", torch.float32), _dev(beta, "beta", torch.float32), B, H, dk, dv,
+        KDA_DTYPE[dt], _dev(state, "state", torch.float32), state.shape[0],
+        _dev(slots, "slots", torch.int32), _dev(o, "o", dt), _stream_ptr(stream))
+    _check(code, "kda_decode_step")
+    return o
+
+
+def kda_device_status(stream=None) -> int:
+    out = ctypes.c_int32(0)
+    _check(_lib.kda_device_status(_stream_ptr(stream), ctypes.byref(out)), "kda_device_status")
+    return int(out.value)

@@ -1,0 +1,172 @@
+// C-ABI layer of libkda_b200: argument validation, workspace sizing and
+// dispatch to the kernels.  Nothing here allocates device memory; every call is
+// asynchronous on the caller's stream.
+#include <mutex>
+#include <stdint.h>
+#include <string.h>
+
+#include "kda.h"
+#include "kda_internal.h"
+
+// Device status word: kernels with bounded on-chip waits record a timeout here
+// instead of hanging.  One instance per device that loads the library.
+__device__ int32_t g_kda_device_status = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_status_mu;
+int32_t *g_status_ptr[kMaxDevices] = {nullptr};
+
+bool head_dim_ok(int32_t d) { return d == 32 || d == 64 || d == 128; }
+bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
+
+kda_status status_word(int32_t **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_status_mu);
+    if (!g_status_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_kda_device_status) != cudaSuccess) return KDA_ERR_CUDA;
+        g_status_ptr[dev] = (int32_t *)p;
+    }
+    *out = g_status_ptr[dev];
+    return KDA_OK;
+}
+
+// Validation shared by kda_prefill_workspace_size and kda_prefill_ex.
+kda_status check_prefill_sizes(int32_t total_tokens, int32_t num_seqs, int32_t H, int32_t dk,
+                               int32_t dv, kda_dtype dt, kda_algo algo)
+{
+    if (total_tokens < 0 || num_seqs < 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+    if (dt != KDA_DTYPE_BF16 && dt != KDA_DTYPE_F32) return KDA_ERR_INVALID_ARG;
+    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_CUDA_CORE && algo != KDA_ALGO_TENSOR_CORE)
+        return KDA_ERR_INVALID_ARG;
+    if (dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (algo == KDA_ALGO_TENSOR_CORE) return KDA_ERR_UNSUPPORTED;  // not in this build yet
+    return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" int32_t kda_abi_version(void) { return KDA_ABI_VERSION; }
+
+extern "C" const char *kda_status_string(kda_status s)
+{
+    switch (s) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: unsupported configuration";
+    case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing or too small";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA runtime error";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: an on-device wait gave up";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+extern "C" size_t kda_prefill_workspace_size(int32_t total_tokens, int32_t num_seqs, int32_t H,
+                                             int32_t dk, int32_t dv, kda_dtype dt, kda_algo algo)
+{
+    if (check_prefill_sizes(total_tokens, num_seqs, H, dk, dv, dt, algo) != KDA_OK) return 0;
+    return 0;  // the CUDA-core path keeps everything on chip
+}
+
+extern "C" kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const void *z,
+                                     const float *A, const float *beta,
+                                     const int32_t *cu_seqlens_dev,
+                                     const int32_t *cu_seqlens_host, int32_t num_seqs,
+                                     int32_t total_tokens, int32_t H, int32_t dk, int32_t dv,
+                                     kda_dtype dt, const float *initial_state,
+                                     float *final_state, void *o, void *workspace,
+                                     size_t workspace_bytes, kda_algo algo, void *stream)
+{
+    kda_status st = check_prefill_sizes(total_tokens, num_seqs, H, dk, dv, dt, algo);
+    if (st != KDA_OK) return st;
+    if (num_seqs > 0 && !cu_seqlens_dev) return KDA_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!q || !k || !v || !z || !A || !beta || !o)) return KDA_ERR_INVALID_ARG;
+    for (const void *p : {q, k, v, z, (const void *)o, (const void *)initial_state,
+                          (const void *)final_state})
+        if (p && !aligned(p, 16)) return KDA_ERR_INVALID_ARG;
+    if ((A && !aligned(A, 4)) || (beta && !aligned(beta, 4)) ||
+        (cu_seqlens_dev && !aligned(cu_seqlens_dev, 4)))
+        return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens_host) {
+        if (cu_seqlens_host[0] != 0 || cu_seqlens_host[num_seqs] != total_tokens)
+            return KDA_ERR_INVALID_ARG;
+        for (int32_t i = 0; i < num_seqs; ++i)
+            if (cu_seqlens_host[i + 1] < cu_seqlens_host[i]) return KDA_ERR_INVALID_ARG;
+    }
+    const size_t need = kda_prefill_workspace_size(total_tokens, num_seqs, H, dk, dv, dt, algo);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
+    if (num_seqs == 0) return KDA_OK;
+
+    int32_t *status = nullptr;
+    if ((st = status_word(&status)) != KDA_OK) return st;
+
+    kda::PrefillArgs a;
+    a.q = q; a.k = k; a.v = v; a.z = z; a.A = A; a.beta = beta;
+    a.cu_seqlens = cu_seqlens_dev; a.seq_order = nullptr;
+    a.num_seqs = num_seqs; a.total_tokens = total_tokens; a.H = H; a.dk = dk; a.dv = dv;
+    a.bf16 = (dt == KDA_DTYPE_BF16);
+    a.initial_state = initial_state; a.final_state = final_state; a.o = o;
+    a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.status = status;
+
+    cudaError_t err = kda::launch_prefill_cuda_core(a, (cudaStream_t)stream);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+extern "C" kda_status kda_prefill(const void *q, const void *k, const void *v, const void *z,
+                                  const float *A, const float *beta,
+                                  const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                                  int32_t num_seqs, int32_t total_tokens, int32_t H, int32_t dk,
+                                  int32_t dv, kda_dtype dt, const float *initial_state,
+                                  float *final_state, void *o, void *workspace,
+                                  size_t workspace_bytes, void *stream)
+{
+    return kda_prefill_ex(q, k, v, z, A, beta, cu_seqlens_dev, cu_seqlens_host, num_seqs,
+                          total_tokens, H, dk, dv, dt, initial_state, final_state, o, workspace,
+                          workspace_bytes, KDA_ALGO_AUTO, stream);
+}
+
+extern "C" kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *z,
+                                      const float *A, const float *beta, int32_t B, int32_t H,
+                                      int32_t dk, int32_t dv, kda_dtype dt, float *state,
+                                      int32_t pool_size, const int32_t *slots, void *o,
+                                      void *stream)
+{
+    if (B < 0 || H <= 0 || pool_size < 0) return KDA_ERR_INVALID_ARG;
+    if (dt != KDA_DTYPE_BF16 && dt != KDA_DTYPE_F32) return KDA_ERR_INVALID_ARG;
+    if (dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (B == 0) return KDA_OK;
+    if (!q || !k || !v || !z || !A || !beta || !state || !o) return KDA_ERR_INVALID_ARG;
+    if (!slots && pool_size < B) return KDA_ERR_INVALID_ARG;
+    for (const void *p : {q, k, v, z, (const void *)o, (const void *)state})
+        if (!aligned(p, 16)) return KDA_ERR_INVALID_ARG;
+    if (!aligned(A, 4) || !aligned(beta, 4) || (slots && !aligned(slots, 4)))
+        return KDA_ERR_INVALID_ARG;
+
+    kda::DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.z = z; a.A = A; a.beta = beta;
+    a.B = B; a.H = H; a.dk = dk; a.dv = dv; a.bf16 = (dt == KDA_DTYPE_BF16);
+    a.state = state; a.slots = slots; a.o = o;
+    cudaError_t err = kda::launch_decode_step(a, (cudaStream_t)stream);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+extern "C" kda_status kda_device_status(void *stream, int32_t *status_out)
+{
+    if (!status_out) return KDA_ERR_INVALID_ARG;
+    int32_t *word = nullptr;
+    kda_status st = status_word(&word);
+    if (st != KDA_OK) return st;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return KDA_ERR_CUDA;
+    int32_t v = 0, zero = 0;
+    if (cudaMemcpy(&v, word, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return KDA_ERR_CUDA;
+    if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    *status_out = v;
+    return KDA_OK;
+}

@@ -1,0 +1,42 @@
+// Internal launch interface between the C-ABI layer (kda_api.cu) and the kernel
+// translation units.  Every launcher enqueues on `stream` and returns the
+// cudaGetLastError() of its launch.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kda {
+
+struct PrefillArgs {
+    const void *q, *k, *v, *z;
+    const float *A, *beta;
+    const int32_t *cu_seqlens;      // device [N+1]
+    const int32_t *seq_order;       // device [N] launch order (longest first) or nullptr
+    int32_t num_seqs, total_tokens, H, dk, dv;
+    bool bf16;                      // storage dtype of q, k, v, z, o
+    const float *initial_state;     // [N,H,dk,dv] or nullptr
+    float *final_state;             // [N,H,dk,dv] or nullptr
+    void *o;
+    void *workspace;
+    size_t workspace_bytes;
+    int32_t *status;                // device status word
+};
+
+struct DecodeArgs {
+    const void *q, *k, *v, *z;
+    const float *A, *beta;
+    int32_t B, H, dk, dv;
+    bool bf16;
+    float *state;
+    const int32_t *slots;
+    void *o;
+};
+
+// Fused chunked prefill on CUDA cores, all arithmetic in fp32 (16-token chunks).
+cudaError_t launch_prefill_cuda_core(const PrefillArgs &a, cudaStream_t stream);
+
+// Single-token decode step (HBM-bound, one CTA per (sequence, head)).
+cudaError_t launch_decode_step(const DecodeArgs &a, cudaStream_t stream);
+
+}  // namespace kda

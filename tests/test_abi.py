@@ -1,0 +1,151 @@
+"""C-ABI checks that need no GPU: symbols, status strings, host-side validation.
+
+Every call here either fails validation on the host (so nothing is launched and
+no pointer is dereferenced) or, for a valid call, runs only where no GPU exists
+(it must then return KDA_ERR_CUDA rather than crash).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from linear_attention_serving_prefill_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE, CUDA = 0, 1, 2, 3, 4
+BF16, F32 = 0, 1
+AUTO, CORE, TC = 0, 1, 2
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert names, "no declarations parsed"
+    lib = ctypes.CDLL(B.library_path())
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/kda.h but not exported"
+    assert set(names) == set(B.SIGNATURES), "binding signatures out of sync with the header"
+
+
+def test_abi_version_and_status_strings():
+    assert B._lib.kda_abi_version() == 1
+    for code in range(6):
+        s = B.kda_status_string(code)
+        assert s.startswith(B.STATUS_NAMES[code])
+    assert B.kda_status_string(99) == "KDA_ERR_UNKNOWN"
+
+
+def _fake(addr=0x10000):
+    return ctypes.c_void_p(addr)
+
+
+def _prefill(**kw):
+    a = dict(q=_fake(), k=_fake(), v=_fake(), z=_fake(), A=_fake(), beta=_fake(),
+             cu=_fake(), cu_host=None, N=2, T=10, H=4, dk=128, dv=128, dt=BF16, s0=None,
+             sf=None, o=_fake(), ws=None, ws_bytes=0, algo=AUTO, stream=None)
+    a.update(kw)
+    return B._lib.kda_prefill_ex(a["q"], a["k"], a["v"], a["z"], a["A"], a["beta"], a["cu"],
+                                 a["cu_host"], a["N"], a["T"], a["H"], a["dk"], a["dv"], a["dt"],
+                                 a["s0"], a["sf"], a["o"], a["ws"], a["ws_bytes"], a["algo"],
+                                 a["stream"])
+
+
+def _host_cu(vals):
+    arr = (ctypes.c_int32 * len(vals))(*vals)
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+def test_prefill_rejects_bad_sizes():
+    assert _prefill(dk=96) == UNSUPPORTED
+    assert _prefill(dv=48) == UNSUPPORTED
+    assert _prefill(dk=0) == INVALID
+    assert _prefill(H=0) == INVALID
+    assert _prefill(N=-1) == INVALID
+    assert _prefill(T=-5) == INVALID
+    assert _prefill(dt=7) == INVALID
+    assert _prefill(algo=9) == INVALID
+    assert _prefill(algo=TC, dt=F32) == UNSUPPORTED
+
+
+def test_prefill_rejects_null_and_misaligned_pointers():
+    for name in ("q", "k", "v", "z", "A", "beta", "o", "cu"):
+        assert _prefill(**{name: None}) == INVALID, name
+    for name in ("q", "k", "v", "z", "o"):
+        assert _prefill(**{name: _fake(0x10008)}) == INVALID, name
+    assert _prefill(s0=_fake(0x10004)) == INVALID
+    assert _prefill(sf=_fake(0x10002)) == INVALID
+    assert _prefill(A=_fake(0x10002)) == INVALID
+
+
+def test_prefill_rejects_malformed_cu_seqlens_host():
+    for vals in ([1, 5, 10], [0, 5, 9], [0, 6, 5], [0, 11, 10]):
+        p, keep = _host_cu(vals)
+        assert _prefill(cu_host=p) == INVALID, vals
+
+
+def test_prefill_workspace_checks():
+    need = B._lib.kda_prefill_workspace_size(10, 2, 4, 128, 128, BF16, AUTO)
+    if need == 0:
+        pytest.skip("this configuration needs no workspace")
+    assert _prefill(ws=None, ws_bytes=0) == WORKSPACE
+    assert _prefill(ws=_fake(), ws_bytes=need - 1) == WORKSPACE
+
+
+def test_workspace_size_rejects_invalid_and_is_shape_only():
+    assert B._lib.kda_prefill_workspace_size(10, 2, 4, 96, 128, BF16, AUTO) == 0
+    assert B._lib.kda_prefill_workspace_size(-1, 2, 4, 128, 128, BF16, AUTO) == 0
+    a = B._lib.kda_prefill_workspace_size(1000, 3, 8, 128, 128, BF16, AUTO)
+    b = B._lib.kda_prefill_workspace_size(1000, 3, 8, 128, 128, BF16, AUTO)
+    assert a == b
+
+
+def test_empty_batch_is_a_no_op():
+    # N = 0, T = 0: nothing to launch, no pointer needed, no CUDA call made.
+    assert _prefill(N=0, T=0, q=None, k=None, v=None, z=None, A=None, beta=None, o=None,
+                    cu=None) == OK
+    assert B._lib.kda_decode_step(None, None, None, None, None, None, 0, 4, 128, 128, BF16,
+                                  None, 0, None, None, None) == OK
+
+
+def _decode(**kw):
+    a = dict(q=_fake(), k=_fake(), v=_fake(), z=_fake(), A=_fake(), beta=_fake(), Bn=4, H=2,
+             dk=128, dv=128, dt=BF16, state=_fake(), P=4, slots=None, o=_fake(), stream=None)
+    a.update(kw)
+    return B._lib.kda_decode_step(a["q"], a["k"], a["v"], a["z"], a["A"], a["beta"], a["Bn"],
+                                  a["H"], a["dk"], a["dv"], a["dt"], a["state"], a["P"],
+                                  a["slots"], a["o"], a["stream"])
+
+
+def test_decode_rejects_bad_arguments():
+    assert _decode(dk=100) == UNSUPPORTED
+    assert _decode(H=0) == INVALID
+    assert _decode(Bn=-1) == INVALID
+    assert _decode(P=3) == INVALID          # pool smaller than the batch without slots
+    assert _decode(state=None) == INVALID
+    assert _decode(q=_fake(0x10004)) == INVALID
+    assert _decode(slots=_fake(0x10002)) == INVALID
+    assert _decode(dt=3) == INVALID
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_valid_call_without_gpu_reports_cuda_error():
+    p, keep = _host_cu([0, 4, 10])
+    assert _prefill(cu_host=p) == CUDA
+    out = ctypes.c_int32(0)
+    assert B._lib.kda_device_status(None, ctypes.byref(out)) == CUDA
+
+
+def test_binding_rejects_cpu_tensors():
+    x = torch.zeros(4, 2, 32, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        B.kda_decode_step(x, x, x, x, torch.zeros(2, 32), torch.zeros(4, 2),
+                          torch.zeros(4, 2, 32, 32))

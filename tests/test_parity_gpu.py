@@ -1,0 +1,241 @@
+"""GPU parity: the CUDA library against the fp64 CPU oracle (B200 only).
+
+Metric: max|err| / max|ref| per output tensor (o and final state separately);
+bar 2e-2 for bf16 inputs with fp32 state, 1e-4 for fp32 inputs.  Every call
+goes through the C ABI (ctypes binding).  Full-size workloads are compared on
+sampled (sequence, head) pairs, each computed whole by the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_serving_prefill_b200 import binding as K
+from linear_attention_serving_prefill_b200.workloads import (CONFIGS, config_inputs,
+                                                             decode_inputs, prefill_inputs)
+from oracle import oracle
+from tests.kda_testutil import (TOL_BF16, TOL_F32, gpu_subset, oracle_subset, relerr, to_np)
+
+pytestmark = pytest.mark.gpu
+
+PREFILL_ALGOS = ["cuda_core"]
+
+
+def _cuda(inp):
+    out = {}
+    for key, val in inp.items():
+        out[key] = val.cuda() if isinstance(val, torch.Tensor) and key != "cu_seqlens_host" else val
+    return out
+
+
+def _run(inp, algo="auto", **kw):
+    return K.kda_prefill(inp["q"], inp["k"], inp["v"], inp["z"], inp["A"], inp["beta"],
+                         inp["cu_seqlens"], inp["cu_seqlens_host"],
+                         initial_state=inp["initial_state"], algo=algo, **kw)
+
+
+def _check_all(inp, o, S, tol):
+    n = len(inp["lengths"])
+    ref_o, ref_S, tok = oracle_subset(inp, list(range(n)), list(range(inp["q"].shape[1])))
+    got_o, got_S = gpu_subset(o, S, tok, list(range(n)), list(range(inp["q"].shape[1])))
+    eo, es = relerr(got_o, ref_o) if got_o.size else 0.0, relerr(got_S, ref_S)
+    assert eo <= tol and es <= tol, (eo, es)
+    return eo, es
+
+
+def test_tiny_f32_config():
+    inp = _cuda(config_inputs(CONFIGS["tiny_f32"]))
+    o, S = _run(inp)
+    torch.cuda.synchronize()
+    _check_all(inp, o, S, TOL_F32)
+
+
+@pytest.mark.parametrize("algo", PREFILL_ALGOS)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("dk,dv", [(32, 32), (64, 64), (128, 128), (64, 128), (128, 32)])
+def test_ragged_varlen_small(algo, dtype, dk, dv):
+    lengths = [1, 15, 16, 17, 100, 0, 257, 64]
+    inp = _cuda(prefill_inputs(lengths, 3, dk, dv, dtype, seed=dk + dv, s0_std=0.02))
+    o, S = _run(inp, algo)
+    torch.cuda.synchronize()
+    _check_all(inp, o, S, TOL_F32 if dtype == "f32" else TOL_BF16)
+
+
+@pytest.mark.parametrize("algo", PREFILL_ALGOS)
+def test_prefill_4k_full(algo):
+    inp = _cuda(config_inputs(CONFIGS["prefill_4k"]))
+    o, S = _run(inp, algo)
+    torch.cuda.synchronize()
+    _check_all(inp, o, S, TOL_BF16)
+
+
+@pytest.mark.parametrize("algo", PREFILL_ALGOS)
+def test_prefill_32k_sampled_heads(algo):
+    cfg = CONFIGS["prefill_32k"]
+    inp = config_inputs(cfg, device="cuda")
+    o, S = _run(inp, algo)
+    torch.cuda.synchronize()
+    heads = [0, 47, 95]
+    ref_o, ref_S, tok = oracle_subset(inp, [0], heads)
+    got_o, got_S = gpu_subset(o, S, tok, [0], heads)
+    assert relerr(got_o, ref_o) <= TOL_BF16
+    assert relerr(got_S, ref_S) <= TOL_BF16
+    assert torch.isfinite(o).all()
+
+
+@pytest.mark.parametrize("algo", PREFILL_ALGOS)
+def test_varlen_resume_sampled(algo):
+    cfg = CONFIGS["varlen_resume"]
+    inp = config_inputs(cfg, device="cuda")
+    o, S = _run(inp, algo)
+    torch.cuda.synchronize()
+    lens = inp["lengths"]
+    seqs = sorted({int(np.argmax(lens)), int(np.argmin(lens)), 5})
+    heads = [0, 95]
+    ref_o, ref_S, tok = oracle_subset(inp, seqs, heads)
+    got_o, got_S = gpu_subset(o, S, tok, seqs, heads)
+    assert relerr(got_o, ref_o) <= TOL_BF16
+    assert relerr(got_S, ref_S) <= TOL_BF16
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+
+
+@pytest.mark.parametrize("algo", PREFILL_ALGOS)
+@pytest.mark.parametrize("case", ["saturated", "alpha_one_beta_one", "slow_decay"])
+def test_gate_edge_cases(algo, case):
+    lengths = [48, 17, 33]
+    kw = dict(saturated=dict(z_mean=1e4, z_std=0.0),
+              alpha_one_beta_one=dict(z_mean=-1e4, z_std=0.0, beta_value=1.0),
+              slow_decay=dict(z_mean=-4.0))[case]
+    inp = _cuda(prefill_inputs(lengths, 2, 128, 128, "bf16", seed=7, s0_std=0.02, **kw))
+    o, S = _run(inp, algo)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    _check_all(inp, o, S, TOL_BF16)
+
+
+@pytest.mark.parametrize("algo", PREFILL_ALGOS)
+def test_empty_sequences_pass_state_through(algo):
+    lengths = [0, 0, 5, 0, 40]
+    inp = _cuda(prefill_inputs(lengths, 2, 64, 64, "bf16", seed=8, s0_std=0.5))
+    o, S = _run(inp, algo)
+    torch.cuda.synchronize()
+    for n in (0, 1, 3):
+        assert torch.equal(S[n], inp["initial_state"][n])
+    _check_all(inp, o, S, TOL_BF16)
+
+
+@pytest.mark.parametrize("algo", PREFILL_ALGOS)
+def test_in_place_resume_and_split_equivalence(algo):
+    """Prefix-cache resume: prefill(x[:t1]) -> S, then prefill(x[t1:], S0 = S)
+    with final_state aliasing initial_state, equals prefill(x)."""
+    L = 300
+    full = _cuda(prefill_inputs([L], 2, 128, 128, "bf16", seed=9, s0_std=0.02))
+    o_full, S_full = _run(full, algo)
+    for t1 in (16, 77, 128):
+        def part(lo, hi, s0):
+            d = {key: full[key][lo:hi] for key in ("q", "k", "v", "z", "beta")}
+            cu = torch.tensor([0, hi - lo], dtype=torch.int32)
+            return dict(d, A=full["A"], cu_seqlens=cu.cuda(), cu_seqlens_host=cu,
+                        initial_state=s0, lengths=[hi - lo])
+        a = part(0, t1, full["initial_state"].clone())
+        oa, sa = _run(a, algo, final_state=a["initial_state"])
+        assert sa.data_ptr() == a["initial_state"].data_ptr()
+        b = part(t1, L, sa)
+        ob, sb = _run(b, algo, final_state=sa)
+        torch.cuda.synchronize()
+        assert relerr(to_np(torch.cat([oa, ob])), to_np(o_full)) <= TOL_BF16
+        assert relerr(to_np(sb), to_np(S_full)) <= TOL_BF16
+    _check_all(full, o_full, S_full, TOL_BF16)
+
+
+@pytest.mark.parametrize("algo", PREFILL_ALGOS)
+def test_outputs_stay_inside_their_buffers(algo):
+    """Guard regions around o and the final state are left untouched."""
+    lengths = [5, 31, 16]
+    inp = _cuda(prefill_inputs(lengths, 2, 64, 64, "bf16", seed=10))
+    T, H, dv, dk, N = sum(lengths), 2, 64, 64, 3
+    guard = 4096
+    obuf = torch.full((guard * 2 + T * H * dv,), 7.0, dtype=torch.bfloat16, device="cuda")
+    sbuf = torch.full((guard * 2 + N * H * dk * dv,), 7.0, dtype=torch.float32, device="cuda")
+    o = obuf[guard:guard + T * H * dv].view(T, H, dv)
+    S = sbuf[guard:guard + N * H * dk * dv].view(N, H, dk, dv)
+    _run(inp, algo, o=o, final_state=S)
+    torch.cuda.synchronize()
+    assert torch.all(obuf[:guard] == 7.0) and torch.all(obuf[-guard:] == 7.0)
+    assert torch.all(sbuf[:guard] == 7.0) and torch.all(sbuf[-guard:] == 7.0)
+    _check_all(inp, o, S, TOL_BF16)
+
+
+# ------------------------------------------------------------------ decode ----
+
+@pytest.mark.parametrize("dtype,tol", [("bf16", TOL_BF16), ("f32", TOL_F32)])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 32), (32, 128)])
+def test_decode_step_with_slots(dtype, tol, dk, dv):
+    B, H, P = 37, 3, 50
+    d = decode_inputs(B, H, dk, dv, dtype, seed=11, nsets=2, pool=P, permute_slots=True,
+                      device="cuda")
+    pool0 = d["state"].clone()
+    o = K.kda_decode_step(d["q"][0], d["k"][0], d["v"][0], d["z"][0], d["A"], d["beta"][0],
+                          d["state"], d["slots"])
+    torch.cuda.synchronize()
+    ref_o, ref_new = oracle.decode_step(d["q"][0], d["k"][0], d["v"][0], d["z"][0], d["A"],
+                                        d["beta"][0], pool0, d["slots"])
+    assert relerr(to_np(o), ref_o) <= tol
+    assert relerr(to_np(d["state"]), ref_new) <= tol
+    untouched = sorted(set(range(P)) - set(d["slots"].cpu().tolist()))
+    assert torch.equal(d["state"][untouched], pool0[untouched])
+
+
+def test_decode_full_batch_first_steps():
+    cfg = CONFIGS["decode_256"]
+    d = decode_inputs(cfg.B, cfg.H, cfg.dk, cfg.dv, cfg.dtype, seed=cfg.seed, nsets=cfg.nsets,
+                      device="cuda")
+    ref_state = to_np(d["state"])
+    for s in range(2):
+        o = K.kda_decode_step(d["q"][s], d["k"][s], d["v"][s], d["z"][s], d["A"], d["beta"][s],
+                              d["state"])
+        torch.cuda.synchronize()
+        ref_o, ref_state = oracle.decode_step(d["q"][s], d["k"][s], d["v"][s], d["z"][s], d["A"],
+                                              d["beta"][s], ref_state)
+        assert relerr(to_np(o), ref_o) <= TOL_BF16
+        assert relerr(to_np(d["state"]), ref_state) <= TOL_BF16
+
+
+def test_decode_1000_steps_sampled_pairs():
+    """The timed decode workload: 1000 in-place steps (step s uses input set
+    s mod 16); sampled (sequence, head) pairs are replayed by the oracle."""
+    cfg = CONFIGS["decode_256"]
+    d = decode_inputs(cfg.B, cfg.H, cfg.dk, cfg.dv, cfg.dtype, seed=cfg.seed, nsets=cfg.nsets,
+                      device="cuda")
+    bsel, hsel = np.array([0, 101, 255]), np.array([0, 50, 95])
+    ref_state = to_np(d["state"])[bsel][:, hsel]
+    subsets = [{key: to_np(d[key][i])[bsel][:, hsel] for key in ("q", "k", "v", "z", "beta")}
+               for i in range(cfg.nsets)]
+    A_sub = to_np(d["A"])[hsel]
+    for s in range(cfg.steps):
+        i = s % cfg.nsets
+        o = K.kda_decode_step(d["q"][i], d["k"][i], d["v"][i], d["z"][i], d["A"], d["beta"][i],
+                              d["state"])
+        sub = subsets[i]
+        ref_o, ref_state = oracle.decode_step(sub["q"], sub["k"], sub["v"], sub["z"], A_sub,
+                                              sub["beta"], ref_state)
+    torch.cuda.synchronize()
+    got_o = to_np(o)[bsel][:, hsel]
+    got_S = to_np(d["state"])[bsel][:, hsel]
+    assert relerr(got_o, ref_o) <= TOL_BF16
+    assert relerr(got_S, ref_state) <= TOL_BF16
+
+
+@pytest.mark.parametrize("algo", PREFILL_ALGOS)
+def test_prefill_then_decode_equals_longer_prefill(algo):
+    L = 70
+    full = _cuda(prefill_inputs([L + 1], 3, 128, 128, "bf16", seed=12, s0_std=0.02))
+    o_full, S_full = _run(full, algo)
+    head = {key: full[key][:L] for key in ("q", "k", "v", "z", "beta")}
+    cu = torch.tensor([0, L], dtype=torch.int32)
+    _, S = _run(dict(head, A=full["A"], cu_seqlens=cu.cuda(), cu_seqlens_host=cu,
+                     initial_state=full["initial_state"], lengths=[L]), algo)
+    o = K.kda_decode_step(*(full[key][L:L + 1].contiguous() for key in ("q", "k", "v", "z")),
+                          full["A"], full["beta"][L:L + 1].contiguous(), S)
+    torch.cuda.synchronize()
+    assert relerr(to_np(o[0]), to_np(o_full[L])) <= TOL_BF16
+    assert relerr(to_np(S), to_np(S_full)) <= TOL_BF16
