@@ -34,6 +34,15 @@ METRIC = "KDA prefill tokens/s + TFLOP/s (H=96,d=128,T=32K); decode-step GB/s vs
 BYTES_PER_TOKEN_HEAD = 1284        # q,k,v,z bf16 (4*256) + beta fp32 (4) + o bf16 (256)
 FLOPS_PER_TOKEN_HEAD = 108544      # 6*dk*dv + 16*(3*dk + 2*dv) at dk = dv = 128
 FALLBACK_HBM_GBS = 6650.0
+# Kernels per prefill call -> (names, algorithmic bytes per token-head of each,
+# source file).  Tensor-core path: the intra kernel reads q, k, v, z (bf16) and
+# beta and writes a 74,240-byte block per (64-token chunk, head), i.e. 1,160 B
+# per token-head; the state kernel reads that block and writes o (bf16).
+KERNELS = {
+    1: (["prefill_cuda_core_kernel"], [BYTES_PER_TOKEN_HEAD], "kda_prefill_cuda_core.cu"),
+    3: (["plan_kernel", "intra_kernel", "state_kernel"], [0, 1028 + 1160, 1160 + 256],
+        "kda_prefill_tc.cu"),
+}
 FALLBACK_BF16_TFLOPS = 1590.0
 
 
@@ -104,17 +113,17 @@ def _source_sha(name: str) -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def _traffic(kernel_file: str, units: int):
+def _traffic(kernel_file: str, kernel: str, units: int):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current source of the kernel; else None."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        rec = json.load(f).get(kernel_file)
+        rec = json.load(f).get(kernel)
     if not rec or rec.get("source_sha") != _source_sha(kernel_file):
         return None
-    return rec["dram_bytes_per_unit"] * units
+    return rec["dram_bytes_per_token_head"] * units
 
 
 def cpu_oracle_sample(inp, target_s: float, max_heads: int = 96):
@@ -123,7 +132,7 @@ def cpu_oracle_sample(inp, target_s: float, max_heads: int = 96):
     so the timed run takes about target_s seconds.  Returns a dict."""
     from oracle import oracle
     cores = oracle.max_threads()
-    h = min(max_heads, inp["q"].shape[1], max(1, cores))
+    h = min(max_heads, inp["q"].shape[1])
 
     def sample(L):
         sl = slice(0, L)
@@ -193,6 +202,10 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="prefill_32k", choices=["prefill_32k", "prefill_4k"],
+                    help="prefill_4k is the small case used for profiler captures")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="skip the decode, end-to-end and CPU legs (profiler captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
@@ -225,7 +238,7 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    cfg = CONFIGS["prefill_32k"]
+    cfg = CONFIGS[args.workload]
     from dataclasses import replace
     inp = config_inputs(replace(cfg, seed=cfg.seed + 1000 * rank), device=dev)
     T, H, dk, dv = inp["q"].shape[0], cfg.H, cfg.dk, cfg.dv
@@ -235,30 +248,36 @@ def main():
     ws_bytes = K.kda_prefill_workspace_size(T, 1, H, dk, dv, torch.bfloat16, args.algo)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
 
-    def step():
+    nk = K.kda_prefill_kernel_count(dk, dv, torch.bfloat16, args.algo)
+    kernel_names, kernel_bytes_per_th, kernel_file = KERNELS[nk]
+
+    def step(events=None):
         K.kda_prefill(inp["q"], inp["k"], inp["v"], inp["z"], inp["A"], inp["beta"],
                       inp["cu_seqlens"], inp["cu_seqlens_host"], None, final_state=S, o=o,
-                      workspace=ws, algo=args.algo, stream=stream)
+                      workspace=ws, algo=args.algo, stream=stream, stage_events=events)
 
     for _ in range(args.warmup):
         step()
+    # One event per kernel boundary per timed step (created by a first record).
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+    for row in evs:
+        for e in row:
+            e.record(stream)
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    evs[0].record(stream)
     for i in range(args.steps):
-        step()
-        evs[i + 1].record(stream)
+        step(evs[i])
     torch.cuda.synchronize()
     clocks = sampler.stop()
     barrier()
     torch.cuda.synchronize()
-    per_launch = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
-    total_ms = evs[0].elapsed_time(evs[-1])
+    total_ms = evs[0][0].elapsed_time(evs[-1][-1])
+    per_kernel_ms = [statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+                     for j in range(nk)]
     total_ms = max_over_ranks(total_ms)
     ms_per_step = total_ms / args.steps
     tokens = T * world
@@ -267,84 +286,91 @@ def main():
     tflops = th * FLOPS_PER_TOKEN_HEAD * world / (ms_per_step / 1e3) / 1e12
 
     hbm_peak, tc_peak, peak_src = _peaks()
-    # The step is one kernel launch on the CUDA-core path: its event pair is the launch.
-    launch_ms = statistics.mean(per_launch)
-    alg_bytes = th * BYTES_PER_TOKEN_HEAD
+    dom = max(range(nk), key=lambda j: per_kernel_ms[j])
+    launch_ms = per_kernel_ms[dom]
+    alg_bytes = th * kernel_bytes_per_th[dom]
     achieved = alg_bytes / (launch_ms / 1e3) / 1e9
-    kernel_file = "kda_prefill_cuda_core.cu"
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": _traffic(kernel_file, th),
-                "kernel": "prefill_cuda_core_kernel", "peak_source": peak_src,
+                "frac": achieved / hbm_peak,
+                "traffic": _traffic(kernel_file, kernel_names[dom], th),
+                "kernel": kernel_names[dom], "peak_source": peak_src,
                 "algorithmic_bytes_per_launch": alg_bytes,
-                "tensor_frac": (th * FLOPS_PER_TOKEN_HEAD / (launch_ms / 1e3) / 1e12) / tc_peak}
-    launches = args.steps
+                "algorithmic_bytes_per_token_head": kernel_bytes_per_th[dom],
+                "kernels_ms": dict(zip(kernel_names, per_kernel_ms))}
+    path_gbs = th * BYTES_PER_TOKEN_HEAD / (ms_per_step / 1e3) / 1e9
+    path = {"bytes_per_token_head": BYTES_PER_TOKEN_HEAD, "achieved_gbs": path_gbs,
+            "hbm_frac": path_gbs / hbm_peak, "tensor_tflops": tflops / world,
+            "tensor_frac": tflops / world / tc_peak, "tensor_peak": tc_peak,
+            "roofline_ms": th * BYTES_PER_TOKEN_HEAD / hbm_peak / 1e6}
+    launches = args.steps * nk
 
-    # Decode step: B=256 cached states, H=96, updated in place; GB/s of state traffic.
-    dcfg = CONFIGS["decode_256"]
-    d = decode_inputs(dcfg.B, dcfg.H, dcfg.dk, dcfg.dv, dcfg.dtype, seed=dcfg.seed + 1000 * rank,
-                      nsets=dcfg.nsets, device=dev)
-    od = torch.empty(dcfg.B, dcfg.H, dcfg.dv, dtype=torch.bfloat16, device=dev)
+    decode = e2e = cpu = None
+    if not args.prefill_only:
+        # Decode step: B=256 cached states, H=96, updated in place; GB/s of state traffic.
+        dcfg = CONFIGS["decode_256"]
+        d = decode_inputs(dcfg.B, dcfg.H, dcfg.dk, dcfg.dv, dcfg.dtype, seed=dcfg.seed + 1000 * rank,
+                          nsets=dcfg.nsets, device=dev)
+        od = torch.empty(dcfg.B, dcfg.H, dcfg.dv, dtype=torch.bfloat16, device=dev)
 
-    def dstep(i):
-        j = i % dcfg.nsets
-        K.kda_decode_step(d["q"][j], d["k"][j], d["v"][j], d["z"][j], d["A"], d["beta"][j],
-                          d["state"], None, o=od, stream=stream)
+        def dstep(i):
+            j = i % dcfg.nsets
+            K.kda_decode_step(d["q"][j], d["k"][j], d["v"][j], d["z"][j], d["A"], d["beta"][j],
+                              d["state"], None, o=od, stream=stream)
 
-    for i in range(args.warmup):
-        dstep(i)
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.decode_steps):
-        dstep(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    dms = max_over_ranks(e0.elapsed_time(e1)) / args.decode_steps
-    state_bytes = 2 * dcfg.B * dcfg.H * dcfg.dk * dcfg.dv * 4
-    dgbs = state_bytes / (dms / 1e3) / 1e9
-    decode = {"config": dcfg.name, "ms_per_step": dms, "state_gbs": dgbs,
-              "frac_of_hbm": dgbs / hbm_peak, "steps": args.decode_steps,
-              "state_bytes_per_step": state_bytes, "gpu_launches": args.decode_steps}
-    del d, od
+        for i in range(args.warmup):
+            dstep(i)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.decode_steps):
+            dstep(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dms = max_over_ranks(e0.elapsed_time(e1)) / args.decode_steps
+        state_bytes = 2 * dcfg.B * dcfg.H * dcfg.dk * dcfg.dv * 4
+        dgbs = state_bytes / (dms / 1e3) / 1e9
+        decode = {"config": dcfg.name, "ms_per_step": dms, "state_gbs": dgbs,
+                  "frac_of_hbm": dgbs / hbm_peak, "steps": args.decode_steps,
+                  "state_bytes_per_step": state_bytes, "gpu_launches": args.decode_steps}
+        del d, od
 
-    # End to end through the C ABI: pinned host inputs -> device, prefill, result -> host.
-    host = {key: inp[key].cpu().pin_memory() for key in ("q", "k", "v", "z", "beta", "A")}
-    host_cu = inp["cu_seqlens_host"].pin_memory()
-    dbuf = {key: torch.empty_like(inp[key]) for key in host}
-    cu_dev = torch.empty_like(inp["cu_seqlens"])
-    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    S_host = torch.empty(S.shape, dtype=S.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values()) + host_cu.numel() * 4
-    d2h = o_host.numel() * o_host.element_size() + S_host.numel() * 4
+        # End to end through the C ABI: pinned host inputs -> device, prefill, result -> host.
+        host = {key: inp[key].cpu().pin_memory() for key in ("q", "k", "v", "z", "beta", "A")}
+        host_cu = inp["cu_seqlens_host"].pin_memory()
+        dbuf = {key: torch.empty_like(inp[key]) for key in host}
+        cu_dev = torch.empty_like(inp["cu_seqlens"])
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        S_host = torch.empty(S.shape, dtype=S.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values()) + host_cu.numel() * 4
+        d2h = o_host.numel() * o_host.element_size() + S_host.numel() * 4
 
-    def e2e_step():
-        for key in host:
-            dbuf[key].copy_(host[key], non_blocking=True)
-        cu_dev.copy_(host_cu, non_blocking=True)
-        K.kda_prefill(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["z"], dbuf["A"], dbuf["beta"], cu_dev,
-                      inp["cu_seqlens_host"], None, final_state=S, o=o, workspace=ws,
-                      algo=args.algo, stream=stream)
-        o_host.copy_(o, non_blocking=True)
-        S_host.copy_(S, non_blocking=True)
+        def e2e_step():
+            for key in host:
+                dbuf[key].copy_(host[key], non_blocking=True)
+            cu_dev.copy_(host_cu, non_blocking=True)
+            K.kda_prefill(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["z"], dbuf["A"], dbuf["beta"], cu_dev,
+                          inp["cu_seqlens_host"], None, final_state=S, o=o, workspace=ws,
+                          algo=args.algo, stream=stream)
+            o_host.copy_(o, non_blocking=True)
+            S_host.copy_(S, non_blocking=True)
 
-    e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
         e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ems = max_over_ranks(e0.elapsed_time(e1)) / args.e2e_steps
-    e2e = {"value": tokens / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": args.e2e_steps}
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = max_over_ranks(e0.elapsed_time(e1)) / args.e2e_steps
+        e2e = {"value": tokens / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": args.e2e_steps}
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        r = cpu_oracle_sample(inp, args.cpu_seconds)
-        cpu = {"value": r["tokens_per_s"], "unit": "tokens/s", "cores": r["cores"],
-               "kind": "oracle", "sample": r["sample"], "seconds": r["seconds"]}
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            r = cpu_oracle_sample(inp, args.cpu_seconds)
+            cpu = {"value": r["tokens_per_s"], "unit": "tokens/s", "cores": r["cores"],
+                   "kind": "oracle", "sample": r["sample"], "seconds": r["seconds"]}
 
     if rank == 0:
         line = {
@@ -358,6 +384,7 @@ def main():
                        "l2": "inputs larger than L2 (q,k,v,z = 3.2 GB per step), no flush"},
             "tflops": tflops,
             "roofline": roofline,
+            "path_roofline": path,
             "decode": decode,
             "e2e": e2e,
             "gpu_launches": launches,

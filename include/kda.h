@@ -107,8 +107,15 @@ size_t kda_prefill_workspace_size(int32_t total_tokens, int32_t num_seqs, int32_
  *                   kda_prefill_workspace_size(T, N, H, dk, dv, dt, algo) bytes
  *                   (may be NULL when that size is 0); contents are scratch.
  *   algo            KDA_ALGO_AUTO, or a forced path; KDA_ALGO_TENSOR_CORE with
- *                   dt = KDA_DTYPE_F32 returns KDA_ERR_UNSUPPORTED.
- * kda_prefill is kda_prefill_ex with algo = KDA_ALGO_AUTO.
+ *                   dt = KDA_DTYPE_F32 or dk, dv != 128 returns KDA_ERR_UNSUPPORTED.
+ *   stage_events    optional instrumentation (NULL = none): an array of
+ *                   num_stage_events cudaEvent_t handles (as void*), owned by
+ *                   the caller.  events[0] is recorded on `stream` before the
+ *                   first kernel of the call and events[i] after its i-th
+ *                   kernel, so elapsed(events[i-1], events[i]) is the duration
+ *                   of kernel i.  Entries beyond kda_prefill_kernel_count() + 1
+ *                   are left untouched; fewer entries record fewer boundaries.
+ * kda_prefill is kda_prefill_ex with algo = KDA_ALGO_AUTO and no events.
  */
 kda_status kda_prefill(const void *q, const void *k, const void *v, const void *z,
                        const float *A, const float *beta,
@@ -124,7 +131,14 @@ kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const voi
                           int32_t num_seqs, int32_t total_tokens, int32_t H, int32_t dk,
                           int32_t dv, kda_dtype dt, const float *initial_state,
                           float *final_state, void *o, void *workspace,
-                          size_t workspace_bytes, kda_algo algo, void *stream);
+                          size_t workspace_bytes, kda_algo algo, void *stream,
+                          void *const *stage_events, int32_t num_stage_events);
+
+/*
+ * Number of kernels one kda_prefill_ex call launches for these sizes and
+ * algorithm (for a non-empty batch); 0 for invalid arguments.
+ */
+int32_t kda_prefill_kernel_count(int32_t dk, int32_t dv, kda_dtype dt, kda_algo algo);
 
 /*
  * One recurrent decode step for B sequences, one new token each ("Kimi K3:

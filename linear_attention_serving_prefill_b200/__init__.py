@@ -8,7 +8,8 @@ without a GPU; every compute entry point raises if the CUDA library is missing.
 from __future__ import annotations
 
 __all__ = ["kda_prefill", "kda_decode_step", "kda_prefill_workspace_size",
-           "kda_status_string", "library_path", "KdaError"]
+           "kda_status_string", "library_path", "KdaError", "kda_prefill_kernel_count",
+           "kda_device_status"]
 
 
 def __getattr__(name):

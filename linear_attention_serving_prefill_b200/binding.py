@@ -29,7 +29,8 @@ SIGNATURES = {
     "kda_status_string": ([_I32], ctypes.c_char_p),
     "kda_prefill_workspace_size": ([_I32, _I32, _I32, _I32, _I32, _I32, _I32], _SZ),
     "kda_prefill": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _P], _I32),
-    "kda_prefill_ex": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _I32, _P], _I32),
+    "kda_prefill_ex": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _I32, _P, _P, _I32], _I32),
+    "kda_prefill_kernel_count": ([_I32, _I32, _I32, _I32], _I32),
     "kda_decode_step": ([_P] * 6 + [_I32] * 5 + [_P, _I32, _P, _P, _P], _I32),
     "kda_device_status": ([_P, _P], _I32),
 }
@@ -94,14 +95,15 @@ def kda_prefill_workspace_size(total_tokens: int, num_seqs: int, H: int, dk: int
 
 def kda_prefill(q, k, v, z, A, beta, cu_seqlens, cu_seqlens_host=None, initial_state=None,
                 output_final_state: bool = True, final_state=None, o=None, workspace=None,
-                algo: str = "auto", stream=None):
+                algo: str = "auto", stream=None, stage_events=None):
     """Chunked KDA prefill over packed sequences; returns ``(o, final_state)``.
 
     q, k, z [T,H,dk], v [T,H,dv] (bf16 or fp32, one dtype); A [H,dk] fp32;
     beta [T,H] fp32; cu_seqlens [N+1] int32 on the device; cu_seqlens_host an
     optional CPU copy; initial_state [N,H,dk,dv] fp32 or None.  ``final_state``
     may be passed (e.g. ``initial_state`` itself, for in-place resume);
-    otherwise it is allocated when ``output_final_state``.
+    otherwise it is allocated when ``output_final_state``.  ``stage_events``
+    (a list of recorded ``torch.cuda.Event``) receives the kernel boundaries.
     """
     T, H, dk = q.shape
     dv = v.shape[2]
@@ -121,15 +123,23 @@ def kda_prefill(q, k, v, z, A, beta, cu_seqlens, cu_seqlens_host=None, initial_s
         ch = cu_seqlens_host.to(torch.int32).contiguous()
         host = ctypes.c_void_p(ch.data_ptr())
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    ev_arr, n_ev = None, 0
+    if stage_events:
+        ev_arr = (ctypes.c_void_p * len(stage_events))(*[e.cuda_event for e in stage_events])
+        n_ev = len(stage_events)
     code = _lib.kda_prefill_ex(
         _dev(q, "q", dt), _dev(k, "k", dt), _dev(v, "v", dt), _dev(z, "z", dt),
         _dev(A, "A", torch.float32), _dev(beta, "beta", torch.float32),
         _dev(cu_seqlens, "cu_seqlens", torch.int32), host, N, T, H, dk, dv, KDA_DTYPE[dt],
         _dev(initial_state, "initial_state", torch.float32),
         _dev(final_state, "final_state", torch.float32), _dev(o, "o", dt),
-        _dev(workspace, "workspace"), ws_bytes, KDA_ALGO[algo], _stream_ptr(stream))
+        _dev(workspace, "workspace"), ws_bytes, KDA_ALGO[algo], _stream_ptr(stream), ev_arr, n_ev)
     _check(code, "kda_prefill")
     return o, final_state
+
+
+def kda_prefill_kernel_count(dk: int, dv: int, dtype=torch.bfloat16, algo: str = "auto") -> int:
+    return int(_lib.kda_prefill_kernel_count(dk, dv, KDA_DTYPE[dtype], KDA_ALGO[algo]))
 
 
 def kda_decode_step(q, k, v, z, A, beta, state, slots=None, o=None, stream=None):

@@ -7,6 +7,7 @@
 
 #include "kda.h"
 #include "kda_internal.h"
+#include "kda_prefill_tc.h"
 
 // Device status word: kernels with bounded on-chip waits record a timeout here
 // instead of hanging.  One instance per device that loads the library.
@@ -45,8 +46,18 @@ kda_status check_prefill_sizes(int32_t total_tokens, int32_t num_seqs, int32_t H
         return KDA_ERR_INVALID_ARG;
     if (dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
-    if (algo == KDA_ALGO_TENSOR_CORE) return KDA_ERR_UNSUPPORTED;  // not in this build yet
+    if (algo == KDA_ALGO_TENSOR_CORE && (dt != KDA_DTYPE_BF16 || dk != 128 || dv != 128))
+        return KDA_ERR_UNSUPPORTED;
     return KDA_OK;
+}
+
+// The path a call takes: tensor cores for bf16 with dk = dv = 128 unless the
+// CUDA-core path is forced; the fp32 CUDA-core path otherwise.
+bool use_tensor_core(int32_t dk, int32_t dv, kda_dtype dt, kda_algo algo)
+{
+    if (algo == KDA_ALGO_TENSOR_CORE) return true;
+    if (algo == KDA_ALGO_CUDA_CORE) return false;
+    return dt == KDA_DTYPE_BF16 && dk == 128 && dv == 128;
 }
 
 }  // namespace
@@ -70,6 +81,7 @@ extern "C" size_t kda_prefill_workspace_size(int32_t total_tokens, int32_t num_s
                                              int32_t dk, int32_t dv, kda_dtype dt, kda_algo algo)
 {
     if (check_prefill_sizes(total_tokens, num_seqs, H, dk, dv, dt, algo) != KDA_OK) return 0;
+    if (use_tensor_core(dk, dv, dt, algo)) return kda::tc_workspace_bytes(total_tokens, num_seqs, H);
     return 0;  // the CUDA-core path keeps everything on chip
 }
 
@@ -80,14 +92,15 @@ extern "C" kda_status kda_prefill_ex(const void *q, const void *k, const void *v
                                      int32_t total_tokens, int32_t H, int32_t dk, int32_t dv,
                                      kda_dtype dt, const float *initial_state,
                                      float *final_state, void *o, void *workspace,
-                                     size_t workspace_bytes, kda_algo algo, void *stream)
+                                     size_t workspace_bytes, kda_algo algo, void *stream,
+                                     void *const *stage_events, int32_t num_stage_events)
 {
     kda_status st = check_prefill_sizes(total_tokens, num_seqs, H, dk, dv, dt, algo);
     if (st != KDA_OK) return st;
     if (num_seqs > 0 && !cu_seqlens_dev) return KDA_ERR_INVALID_ARG;
     if (total_tokens > 0 && (!q || !k || !v || !z || !A || !beta || !o)) return KDA_ERR_INVALID_ARG;
     for (const void *p : {q, k, v, z, (const void *)o, (const void *)initial_state,
-                          (const void *)final_state})
+                          (const void *)final_state, (const void *)workspace})
         if (p && !aligned(p, 16)) return KDA_ERR_INVALID_ARG;
     if ((A && !aligned(A, 4)) || (beta && !aligned(beta, 4)) ||
         (cu_seqlens_dev && !aligned(cu_seqlens_dev, 4)))
@@ -98,9 +111,9 @@ extern "C" kda_status kda_prefill_ex(const void *q, const void *k, const void *v
         for (int32_t i = 0; i < num_seqs; ++i)
             if (cu_seqlens_host[i + 1] < cu_seqlens_host[i]) return KDA_ERR_INVALID_ARG;
     }
+    if (num_seqs == 0) return KDA_OK;
     const size_t need = kda_prefill_workspace_size(total_tokens, num_seqs, H, dk, dv, dt, algo);
     if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
-    if (num_seqs == 0) return KDA_OK;
 
     int32_t *status = nullptr;
     if ((st = status_word(&status)) != KDA_OK) return st;
@@ -112,8 +125,11 @@ extern "C" kda_status kda_prefill_ex(const void *q, const void *k, const void *v
     a.bf16 = (dt == KDA_DTYPE_BF16);
     a.initial_state = initial_state; a.final_state = final_state; a.o = o;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.status = status;
+    a.events = stage_events; a.num_events = stage_events ? num_stage_events : 0;
 
-    cudaError_t err = kda::launch_prefill_cuda_core(a, (cudaStream_t)stream);
+    cudaError_t err = use_tensor_core(dk, dv, dt, algo)
+                          ? kda::launch_prefill_tensor_core(a, (cudaStream_t)stream)
+                          : kda::launch_prefill_cuda_core(a, (cudaStream_t)stream);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -127,7 +143,13 @@ extern "C" kda_status kda_prefill(const void *q, const void *k, const void *v, c
 {
     return kda_prefill_ex(q, k, v, z, A, beta, cu_seqlens_dev, cu_seqlens_host, num_seqs,
                           total_tokens, H, dk, dv, dt, initial_state, final_state, o, workspace,
-                          workspace_bytes, KDA_ALGO_AUTO, stream);
+                          workspace_bytes, KDA_ALGO_AUTO, stream, nullptr, 0);
+}
+
+extern "C" int32_t kda_prefill_kernel_count(int32_t dk, int32_t dv, kda_dtype dt, kda_algo algo)
+{
+    if (check_prefill_sizes(0, 0, 1, dk, dv, dt, algo) != KDA_OK) return 0;
+    return use_tensor_core(dk, dv, dt, algo) ? 3 : 1;
 }
 
 extern "C" kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *z,

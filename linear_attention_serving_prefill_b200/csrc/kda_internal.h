@@ -21,6 +21,12 @@ struct PrefillArgs {
     void *workspace;
     size_t workspace_bytes;
     int32_t *status;                // device status word
+    void *const *events;            // optional cudaEvent_t per kernel boundary
+    int32_t num_events;
+    // Records boundary i (0 = before the first kernel) when the caller asked for it.
+    void mark(int i, cudaStream_t stream) const {
+        if (events && i < num_events && events[i]) cudaEventRecord((cudaEvent_t)events[i], stream);
+    }
 };
 
 struct DecodeArgs {

@@ -208,9 +208,11 @@ cudaError_t launch_typed(const PrefillArgs &a, cudaStream_t stream)
     if (err != cudaSuccess) return err;
     const long long blocks = (long long)a.num_seqs * a.H * (a.dv / kDVS);
     if (blocks == 0) return cudaSuccess;
+    a.mark(0, stream);
     kern<<<(unsigned)blocks, kThreads, smem, stream>>>(
         (const TIn *)a.q, (const TIn *)a.k, (const TIn *)a.v, (const TIn *)a.z, a.A, a.beta,
         a.cu_seqlens, a.H, a.dv, a.initial_state, a.final_state, (TIn *)a.o);
+    a.mark(1, stream);
     return cudaGetLastError();
 }
 

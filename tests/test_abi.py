@@ -56,7 +56,7 @@ def _prefill(**kw):
     return B._lib.kda_prefill_ex(a["q"], a["k"], a["v"], a["z"], a["A"], a["beta"], a["cu"],
                                  a["cu_host"], a["N"], a["T"], a["H"], a["dk"], a["dv"], a["dt"],
                                  a["s0"], a["sf"], a["o"], a["ws"], a["ws_bytes"], a["algo"],
-                                 a["stream"])
+                                 a["stream"], None, 0)
 
 
 def _host_cu(vals):
@@ -74,6 +74,15 @@ def test_prefill_rejects_bad_sizes():
     assert _prefill(dt=7) == INVALID
     assert _prefill(algo=9) == INVALID
     assert _prefill(algo=TC, dt=F32) == UNSUPPORTED
+    assert _prefill(algo=TC, dk=64, dv=64) == UNSUPPORTED
+
+
+def test_kernel_count():
+    assert B._lib.kda_prefill_kernel_count(128, 128, BF16, AUTO) == 3
+    assert B._lib.kda_prefill_kernel_count(128, 128, BF16, CORE) == 1
+    assert B._lib.kda_prefill_kernel_count(64, 64, BF16, AUTO) == 1
+    assert B._lib.kda_prefill_kernel_count(128, 128, F32, AUTO) == 1
+    assert B._lib.kda_prefill_kernel_count(96, 128, BF16, AUTO) == 0
 
 
 def test_prefill_rejects_null_and_misaligned_pointers():
@@ -139,7 +148,8 @@ def test_decode_rejects_bad_arguments():
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
 def test_valid_call_without_gpu_reports_cuda_error():
     p, keep = _host_cu([0, 4, 10])
-    assert _prefill(cu_host=p) == CUDA
+    need = B._lib.kda_prefill_workspace_size(10, 2, 4, 128, 128, BF16, AUTO)
+    assert _prefill(cu_host=p, ws=_fake(), ws_bytes=need) == CUDA
     out = ctypes.c_int32(0)
     assert B._lib.kda_device_status(None, ctypes.byref(out)) == CUDA
 

@@ -17,7 +17,12 @@ from tests.kda_testutil import (TOL_BF16, TOL_F32, gpu_subset, oracle_subset, re
 
 pytestmark = pytest.mark.gpu
 
-PREFILL_ALGOS = ["cuda_core"]
+PREFILL_ALGOS = ["cuda_core", "tensor_core"]
+
+
+def _supported(algo, dtype="bf16", dk=128, dv=128):
+    if algo == "tensor_core" and (dtype != "bf16" or dk != 128 or dv != 128):
+        pytest.skip("the tensor-core path covers bf16 with dk = dv = 128")
 
 
 def _cuda(inp):
@@ -53,6 +58,7 @@ def test_tiny_f32_config():
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("dk,dv", [(32, 32), (64, 64), (128, 128), (64, 128), (128, 32)])
 def test_ragged_varlen_small(algo, dtype, dk, dv):
+    _supported(algo, dtype, dk, dv)
     lengths = [1, 15, 16, 17, 100, 0, 257, 64]
     inp = _cuda(prefill_inputs(lengths, 3, dk, dv, dtype, seed=dk + dv, s0_std=0.02))
     o, S = _run(inp, algo)
@@ -115,7 +121,7 @@ def test_gate_edge_cases(algo, case):
 @pytest.mark.parametrize("algo", PREFILL_ALGOS)
 def test_empty_sequences_pass_state_through(algo):
     lengths = [0, 0, 5, 0, 40]
-    inp = _cuda(prefill_inputs(lengths, 2, 64, 64, "bf16", seed=8, s0_std=0.5))
+    inp = _cuda(prefill_inputs(lengths, 2, 128, 128, "bf16", seed=8, s0_std=0.5))
     o, S = _run(inp, algo)
     torch.cuda.synchronize()
     for n in (0, 1, 3):
@@ -150,9 +156,9 @@ def test_in_place_resume_and_split_equivalence(algo):
 @pytest.mark.parametrize("algo", PREFILL_ALGOS)
 def test_outputs_stay_inside_their_buffers(algo):
     """Guard regions around o and the final state are left untouched."""
-    lengths = [5, 31, 16]
-    inp = _cuda(prefill_inputs(lengths, 2, 64, 64, "bf16", seed=10))
-    T, H, dv, dk, N = sum(lengths), 2, 64, 64, 3
+    lengths = [5, 31, 16, 70]
+    inp = _cuda(prefill_inputs(lengths, 2, 128, 128, "bf16", seed=10))
+    T, H, dv, dk, N = sum(lengths), 2, 128, 128, 4
     guard = 4096
     obuf = torch.full((guard * 2 + T * H * dv,), 7.0, dtype=torch.bfloat16, device="cuda")
     sbuf = torch.full((guard * 2 + N * H * dk * dv,), 7.0, dtype=torch.float32, device="cuda")
