@@ -141,6 +141,37 @@ kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const voi
 int32_t kda_prefill_kernel_count(int32_t dk, int32_t dv, kda_dtype dt, kda_algo algo);
 
 /*
+ * kda_prefill without a workspace argument, for callers that cannot allocate
+ * device memory at call time (for example a serving engine that gives all free
+ * HBM to its cache pool at start-up and forbids later allocations, code running
+ * under another framework's allocator, or a latency-critical loop that cannot
+ * pay for the device synchronisation of cudaMalloc / cudaFree).  It has no
+ * counterpart in the source pages; it is a deployment convenience.
+ *
+ * Same arguments and results as kda_prefill on the tensor-core path (bf16,
+ * dk = dv = 128; other types or sizes return KDA_ERR_UNSUPPORTED).  The scratch
+ * memory is one file-scope device array of 64 MiB that the library holds on
+ * every GPU where this entry point's module is loaded, until the process exits.
+ * A call whose kda_prefill_workspace_size(..., KDA_ALGO_TENSOR_CORE) exceeds
+ * 64 MiB (about 900 chunk-head tiles of 64 tokens, e.g. one 576-token sequence
+ * at 96 heads) returns KDA_ERR_WORKSPACE and launches nothing.  It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *
+ * The first call on each device looks up the array's device address; make
+ * that first call before any stream capture.  Every call on a device shares the
+ * one array and leaves its contents behind; the kernels overwrite every scratch
+ * byte they later read, so nothing needs clearing.  Calls whose work overlaps
+ * on the GPU (different streams, or several host threads) race on the array:
+ * the caller must serialise them, e.g. by issuing them all on one stream.
+ */
+kda_status kda_prefill_noalloc(const void *q, const void *k, const void *v, const void *z,
+                               const float *A, const float *beta,
+                               const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                               int32_t num_seqs, int32_t total_tokens, int32_t H, int32_t dk,
+                               int32_t dv, kda_dtype dt, const float *initial_state,
+                               float *final_state, void *o, void *stream);
+
+/*
  * One recurrent decode step for B sequences, one new token each ("Kimi K3:
  * Architecture, Training, and Million-Token Agentic RL", section 3.2 edit
  * order: Sbar = Diag(alpha) S; vhat = Sbar^T k; S = Sbar + beta k (v - vhat)^T;

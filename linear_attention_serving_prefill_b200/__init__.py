@@ -9,7 +9,7 @@ from __future__ import annotations
 
 __all__ = ["kda_prefill", "kda_decode_step", "kda_prefill_workspace_size",
            "kda_status_string", "library_path", "KdaError", "kda_prefill_kernel_count",
-           "kda_device_status"]
+           "kda_device_status", "kda_prefill_noalloc"]
 
 
 def __getattr__(name):

@@ -31,6 +31,7 @@ SIGNATURES = {
     "kda_prefill": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _P], _I32),
     "kda_prefill_ex": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _I32, _P, _P, _I32], _I32),
     "kda_prefill_kernel_count": ([_I32, _I32, _I32, _I32], _I32),
+    "kda_prefill_noalloc": ([_P] * 8 + [_I32] * 6 + [_P] * 4, _I32),
     "kda_decode_step": ([_P] * 6 + [_I32] * 5 + [_P, _I32, _P, _P, _P], _I32),
     "kda_device_status": ([_P, _P], _I32),
 }
@@ -135,6 +136,39 @@ def kda_prefill(q, k, v, z, A, beta, cu_seqlens, cu_seqlens_host=None, initial_s
         _dev(final_state, "final_state", torch.float32), _dev(o, "o", dt),
         _dev(workspace, "workspace"), ws_bytes, KDA_ALGO[algo], _stream_ptr(stream), ev_arr, n_ev)
     _check(code, "kda_prefill")
+    return o, final_state
+
+
+def kda_prefill_noalloc(q, k, v, z, A, beta, cu_seqlens, cu_seqlens_host=None,
+                        initial_state=None, output_final_state: bool = True, final_state=None,
+                        o=None, stream=None):
+    """kda_prefill with the library's fixed scratch array instead of a workspace.
+
+    For callers that must not allocate device memory during the call: pass
+    preallocated ``o`` (and ``final_state``) to keep this function from
+    allocating them.  Returns ``(o, final_state)``.
+    """
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = cu_seqlens.shape[0] - 1
+    dt = q.dtype
+    if dt not in KDA_DTYPE:
+        raise ValueError(f"unsupported dtype {dt}")
+    if o is None:
+        o = torch.empty(T, H, dv, dtype=dt, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+    host = None
+    if cu_seqlens_host is not None:
+        ch = cu_seqlens_host.to(torch.int32).contiguous()
+        host = ctypes.c_void_p(ch.data_ptr())
+    code = _lib.kda_prefill_noalloc(
+        _dev(q, "q", dt), _dev(k, "k", dt), _dev(v, "v", dt), _dev(z, "z", dt),
+        _dev(A, "A", torch.float32), _dev(beta, "beta", torch.float32),
+        _dev(cu_seqlens, "cu_seqlens", torch.int32), host, N, T, H, dk, dv, KDA_DTYPE[dt],
+        _dev(initial_state, "initial_state", torch.float32),
+        _dev(final_state, "final_state", torch.float32), _dev(o, "o", dt), _stream_ptr(stream))
+    _check(code, "kda_prefill_noalloc")
     return o, final_state
 
 

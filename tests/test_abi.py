@@ -159,3 +159,11 @@ def test_binding_rejects_cpu_tensors():
     with pytest.raises(ValueError):
         B.kda_decode_step(x, x, x, x, torch.zeros(2, 32), torch.zeros(4, 2),
                           torch.zeros(4, 2, 32, 32))
+
+
+def test_noalloc_rejects_calls_beyond_its_scratch_limit():
+    # 64 MiB of scratch holds about 900 chunk-head tiles; 96 heads x 16 chunks do not fit.
+    args = [_fake()] * 6 + [_fake(), None, 1, 16 * 64, 96, 128, 128, BF16, None, None, _fake(), None]
+    assert B._lib.kda_prefill_noalloc(*args) == WORKSPACE
+    args = [_fake()] * 6 + [_fake(), None, 1, 64, 1, 64, 64, BF16, None, None, _fake(), None]
+    assert B._lib.kda_prefill_noalloc(*args) == UNSUPPORTED
