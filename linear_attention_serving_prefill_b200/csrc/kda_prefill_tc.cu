@@ -9,7 +9,7 @@
 //
 // Three launches per call:
 //   1. plan:   per-sequence chunk offsets and a longest-first order.
-//   2. intra:  one CTA per (64-token chunk, head).  Gate and cumulative
+//   2. intra:  persistent, one CTA per SM over the (64-token chunk, head) items.  Gate and cumulative
 //              log-decay G in fp32, then on the tensor cores
 //                A = strictly_lower(Diag(beta) Kt Kh^T), P = lower(Qt Kh^T)
 //              (16-token sub-tiles, each with its own reference point), the
@@ -31,7 +31,10 @@
 //   O  = Qt S_in + P Dl,   S_out = Diag(e^{G_C}) S_in + Kd^T Dl,
 // the recurrence unrolled over the chunk (the derivation is restated in the
 // oracle's chunkwise module).
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
+#include <mutex>
 
 #include "kda_common.cuh"
 #include "kda_internal.h"
@@ -45,7 +48,6 @@ using namespace tc;
 
 constexpr int kDK = 128, kDV = 128;
 constexpr int kChunk = 64;         // state-passing chunk
-constexpr int kSub = 16;           // sub-tile with its own decay reference
 constexpr uint64_t kWaitNs = 2000000000ull;  // per-wait limit: 2 s
 
 // Per (chunk, head) block written by the intra kernel, read by the state kernel.
@@ -114,20 +116,52 @@ plan_kernel(const int32_t *__restrict__ cu, int N, int32_t *__restrict__ chunk_o
 
 // ------------------------------------------------------------------ intra --
 
-constexpr int kIntraThreads = 128;
-// Shared memory of the intra kernel (offsets from a 1024-aligned base).
-constexpr uint32_t kIRbig = 0;        // 2 x 160 rows x 128 B: A/P A-operands R^(I)
-constexpr uint32_t kIKQ = 40960;      // 2 x 128 rows x 128 B: [Kt_I; Qt_I] per sub-tile
-constexpr uint32_t kIBWU = 73728;     // 256 rows x 128 B: [beta K e^G ; beta V]^T
-constexpr uint32_t kISmem = 106496;
-// Reused after the A/P products are read back:
-constexpr uint32_t kIAf = 0;          // fp32 A [64][65]
-constexpr uint32_t kITf = 16640;      // fp32 T [64][65]
-constexpr uint32_t kIXf = 33280;      // fp32 scratch [32][33]
-constexpr uint32_t kITop = kIKQ;      // bf16 T operand 64 rows x 128 B
+// Persistent: one CTA per SM walks (chunk, head) items b, b + gridDim.x, ...;
+// item w is chunk w / H of head w % H.  While an item is computed, warp 0
+// prefetches the next item's raw k, q, v, z rows (256 B each) into the other
+// stage of a two-stage ring with bulk copies, and its beta values with
+// cp.async.  Thread (cp, I) owns channels 2 cp, 2 cp + 1 of sub-tile I = warp / 2
+// (rows 16 I .. 16 I + 15), so the sub-tile index is uniform across a warp.
+constexpr int kIntraCompute = 256;
+constexpr int kIntraThreads = kIntraCompute;
+constexpr uint32_t kRawTile = kChunk * kDK * 2;    // one [64][128] bf16 tile, 16 KiB
+constexpr uint32_t kRawStage = 4 * kRawTile;       // k, q, v, z
+constexpr uint32_t kRawK = 0, kRawQ = kRawTile, kRawV = 2 * kRawTile, kRawZ = 3 * kRawTile;
+// Shared memory (offsets from a 1024-aligned base).
+constexpr uint32_t kIRaw = 0;                      // 2 raw stages
+constexpr uint32_t kIRbig = 2 * kRawStage;         // 2 x 160 rows x 128 B: A-operands R^(I)
+constexpr uint32_t kIKQ = kIRbig + 40960;          // [Kt_I; Qt_I] per sub-tile, then [bK e^G; bV]^T
+constexpr uint32_t kISmem = kIKQ + 32768;
+// Reused inside Rbig once the A/P products are read back:
+constexpr uint32_t kIAf = kIRbig;                  // fp32 A [64][65]
+constexpr uint32_t kITf = kIRbig + 16640;          // fp32 T [64][65]
+constexpr uint32_t kIXf = kIRbig + 33280;          // fp32 scratch [32][33]
 constexpr int kLd = 65;
 // First row of R^(I) in Rbig: 16 * (0 + 1 + ... + I) = 0, 16, 48, 96.
 __host__ __device__ constexpr int row_base(int I) { return 8 * I * (I + 1); }
+
+struct IntraItem { int t0, len, g, h; };
+
+// One 3-D tile load: the box {128 channels, 1 head, 64 tokens} at (0, h, t0)
+// of a [T][H][128] bf16 tensor; rows past T arrive as zeros.
+__device__ __forceinline__ void tma_rows(void *smem_dst, const CUtensorMap *map, int h, int t0,
+                                         uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(h), "r"(t0),
+          "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void compute_sync() { __syncthreads(); }
+
+__device__ __forceinline__ void cp_async_4(void *smem_dst, const void *gmem_src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ int find_seq(const int32_t *chunk_off, int N, int g) {
     int lo = 0, hi = N - 1;  // largest n with chunk_off[n] <= g
@@ -138,254 +172,358 @@ __device__ __forceinline__ int find_seq(const int32_t *chunk_off, int N, int g) 
     return lo;
 }
 
-__global__ void __launch_bounds__(kIntraThreads)
-intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-             const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ z,
+__device__ __forceinline__ float2 ld_bf16x2_smem(const uint8_t *base, uint32_t off) {
+    return __bfloat1622float2(*(const __nv_bfloat162 *)(base + off));
+}
+
+__device__ __forceinline__ uint32_t bf16_bits(float x) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+// The gate with the fast exponential and division (a few ulp; the bf16 path's
+// tolerance is far looser).  Limits as in gate_log_decay: exp(A) z -> +inf gives
+// g_min, -> -inf gives 0 (1 / +inf through the fast division is 0).
+__device__ __forceinline__ float gate_log_decay_fast(float expA, float z) {
+    return __fdividef(kGMin, 1.0f + __expf(-expA * z));
+}
+
+__global__ void __launch_bounds__(kIntraThreads, 1)
+intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_z,
              const float *__restrict__ A, const float *__restrict__ beta,
              const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_off, int N, int H,
              uint8_t *__restrict__ blocks, int64_t max_chunks, int32_t *status)
 {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t bar;
+    __shared__ uint64_t full[2], mma_bar;
     __shared__ uint32_t tbase;
-    __shared__ float sBeta[kChunk];
-    __shared__ int sAbort;
+    __shared__ IntraItem info[2];
+    __shared__ float sBeta[2][kChunk];
+    __shared__ float sTot[4][kDK];
+    __shared__ volatile int sAbort;
 
-    const int g = blockIdx.x, h = blockIdx.y, c = threadIdx.x;
-    const int total = chunk_off[N];
-    if (g >= total) return;
-    const int n = find_seq(chunk_off, N, g);
-    const int t0 = cu[n] + (g - chunk_off[n]) * kChunk;
-    const int len = min(kChunk, cu[n + 1] - t0);
-    uint8_t *blk = blocks + ((size_t)h * max_chunks + g) * kBlockBytes;
-    const size_t rs = (size_t)H * kDK;                  // token stride (elements)
-    const size_t base = (size_t)t0 * rs + (size_t)h * kDK + c;
-    const int warp = c >> 5, lane = c & 31;
-
-    if (c == 0) {
-        mbar_init(&bar, 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int total_items = chunk_off[N] * H;
+    if ((int)blockIdx.x >= total_items) return;
+    if (tid == 0) {
+        for (int s = 0; s < 2; ++s) mbar_init(&full[s], 1);
+        mbar_init(&mma_bar, 1);
         fence_mbar_init();
         sAbort = 0;
     }
-    if (c < kChunk) sBeta[c] = c < len ? beta[(size_t)(t0 + c) * H + h] : 0.f;
     if (warp == 0) { tmem_alloc(&tbase, 256); tmem_relinquish(); }
-
-    // Pass 1: gate and cumulative log-decay for key channel c, all 64 rows.
-    const float eA = expf(A[(size_t)h * kDK + c]);
-    float G[kChunk];
-    {
-        float acc = 0.f;
-#pragma unroll
-        for (int r = 0; r < kChunk; ++r) {
-            const float zz = r < len ? __bfloat162float(z[base + (size_t)r * rs]) : 0.f;
-            acc += r < len ? gate_log_decay(eA, zz) : 0.f;
-            G[r] = acc;
-        }
-    }
-    // Sub-tile references m_I = G at the end of sub-tile I-1 (m_0 = 0) and
-    // the factors that carry a column operand from its own sub-tile's
-    // reference to a later sub-tile's: f[I'][I] = e^{m_I' - m_I} <= 1.
-    const float m1 = G[15], m2 = G[31], m3 = G[47], GC = G[63];
-    const float mref[4] = {0.f, m1, m2, m3};
-    float f[4][4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) f[a][b] = (a > b) ? __expf(mref[a] - mref[b]) : 1.f;
-    float emref[4];
-#pragma unroll
-    for (int I = 0; I < 4; ++I) emref[I] = __expf(mref[I]);
-    const float eGC[4] = {__expf(GC - mref[0]), __expf(GC - mref[1]), __expf(GC - mref[2]),
-                          __expf(GC - mref[3])};
-    __syncthreads();  // sBeta visible
-
-    // Pass 2: scaled operands for channel c.
-    uint8_t *sR = sm + kIRbig, *sKQ = sm + kIKQ, *sB = sm + kIBWU;
-    uint32_t bufK[4], bufV[4], bufD[4];
-#pragma unroll
-    for (int r = 0; r < kChunk; ++r) {
-        const int I = r / kSub, ri = r % kSub;
-        const bool valid = r < len;
-        const float kv = valid ? __bfloat162float(k[base + (size_t)r * rs]) : 0.f;
-        const float qv = valid ? __bfloat162float(q[base + (size_t)r * rs]) : 0.f;
-        const float vv = valid ? __bfloat162float(v[(size_t)(t0 + r) * H * kDV + (size_t)h * kDV + c]) : 0.f;
-        const float e1 = __expf(G[r] - mref[I]);   // in [e^-80, 1]
-        const float e2 = __expf(mref[I] - G[r]);   // in [1, e^80]
-        const float br = sBeta[r];
-        // B operand of the A/P products: Kt and Qt scaled to the row sub-tile reference.
-        *(__nv_bfloat16 *)(sKQ + sw128_offset(32 * I + ri, c, 128)) = __float2bfloat16_rn(kv * e1);
-        *(__nv_bfloat16 *)(sKQ + sw128_offset(32 * I + 16 + ri, c, 128)) = __float2bfloat16_rn(qv * e1);
-        // A operands R^(I') for every later sub-tile I' >= I: k e^{m_I' - G_r}.
-        const float kb = kv * e2;
-#pragma unroll
-        for (int Ip = 0; Ip < 4; ++Ip)
-            if (Ip >= I)
-                *(__nv_bfloat16 *)(sR + sw128_offset(row_base(Ip) + r, c, 160)) =
-                    __float2bfloat16_rn(kb * f[Ip][I]);
-        // Qt with the chunk-start reference -> rows 64.. of the [W; Qt] tile.
-        *(__nv_bfloat16 *)(blk + kOffWQ + sw128_offset(64 + r, c, 128)) =
-            __float2bfloat16_rn(qv * e1 * emref[I]);
-        // Transposed operands, 8 tokens per 16-byte store.
-        const uint32_t hk = __bfloat16_as_ushort(__float2bfloat16_rn(br * kv * e1 * emref[I]));
-        const uint32_t hv = __bfloat16_as_ushort(__float2bfloat16_rn(br * vv));
-        const uint32_t hd = __bfloat16_as_ushort(__float2bfloat16_rn(kv * e2 * eGC[I]));
-        const int slot = (r & 7) >> 1;
-        if ((r & 1) == 0) {
-            bufK[slot] = hk; bufV[slot] = hv; bufD[slot] = hd;
-        } else {
-            bufK[slot] |= hk << 16; bufV[slot] |= hv << 16; bufD[slot] |= hd << 16;
-        }
-        if ((r & 7) == 7) {
-            const int r0 = r - 7;
-            *(uint4 *)(sB + sw128_offset(c, r0, 256)) = make_uint4(bufK[0], bufK[1], bufK[2], bufK[3]);
-            *(uint4 *)(sB + sw128_offset(128 + c, r0, 256)) = make_uint4(bufV[0], bufV[1], bufV[2], bufV[3]);
-            *(uint4 *)(blk + kOffKd + sw128_offset(c, r0, 128)) = make_uint4(bufD[0], bufD[1], bufD[2], bufD[3]);
-        }
-    }
-    ((float *)(blk + kOffDecay))[c] = __expf(GC);
-
-    // A/P products on the tensor cores: for sub-tile I, D[s][32I + j] =
-    // R^(I)_s . Kt_{16I+j} (j < 16) and R^(I)_s . Qt_{16I+j-16} (j >= 16).
-    fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tb = tbase;
-    const uint64_t deadline = globaltimer_ns() + kWaitNs;
-    if (c == 0) {
-        const uint32_t id = idesc_bf16_f32(64, 32);
-#pragma unroll
-        for (int I = 0; I < 4; ++I)
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t kb2 = ks >> 2, kin = ks & 3;
-                const uint32_t a = smem_u32(sR) + kb2 * 160 * 128 + row_base(I) * 128 + kin * 32;
-                const uint32_t b = smem_u32(sKQ) + kb2 * 128 * 128 + 32 * I * 128 + kin * 32;
-                mma_ss(tmem_addr(tb, 0, 32 * I), desc_kmajor_sw128(a), desc_kmajor_sw128(b), id, ks > 0);
-            }
-        mma_commit(&bar);
-    }
-    if (!mbar_wait(&bar, 0, deadline)) { record_timeout(status); sAbort = 1; }
-    tc_fence_after_sync();
 
-    float *Af = (float *)(sm + kIAf), *Tf = (float *)(sm + kITf), *Xf = (float *)(sm + kIXf);
-    // Read back (M = 64 layout: row s -> lane 16 * (s / 16) ... warp w lanes 0-15).
+    // Warp 0: request item wn into stage sn (raw rows by bulk copy, beta by cp.async).
+    auto issue = [&](int wn, int sn) {
+        const int g = wn / H, h = wn % H;
+        const int n = find_seq(chunk_off, N, g);
+        const int t0 = cu[n] + (g - chunk_off[n]) * kChunk;
+        const int len = min(kChunk, cu[n + 1] - t0);
+        for (int r = lane; r < kChunk; r += 32) {
+            if (r < len) cp_async_4(&sBeta[sn][r], beta + (size_t)(t0 + r) * H + h);
+            else sBeta[sn][r] = 0.f;
+        }
+        cp_async_commit();
+        if (lane == 0) {
+            info[sn] = IntraItem{t0, len, g, h};
+            mbar_arrive_expect_tx(&full[sn], kRawStage);
+            uint8_t *stn = sm + kIRaw + sn * kRawStage;
+            tma_rows(stn + kRawK, &tm_k, h, t0, &full[sn]);
+            tma_rows(stn + kRawQ, &tm_q, h, t0, &full[sn]);
+            tma_rows(stn + kRawV, &tm_v, h, t0, &full[sn]);
+            tma_rows(stn + kRawZ, &tm_z, h, t0, &full[sn]);
+        }
+        __syncwarp();
+    };
+    if (warp == 0) issue(blockIdx.x, 0);
+    int issued = 1;  // items requested so far (meaningful in warp 0)
+
     {
-        uint32_t rr[32];
-        const int s = 16 * warp + lane;
-#pragma unroll
-        for (int I = 0; I < 4; ++I) {
-            tmem_ld32(tmem_addr(tb, 32 * warp, 32 * I), rr);
-            tmem_ld_wait();
-            if (lane < 16) {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int r = 16 * I + j;
-                    Af[r * kLd + s] = s < r ? sBeta[r] * __uint_as_float(rr[j]) : 0.f;
-                    const float pv = s <= r ? __uint_as_float(rr[16 + j]) : 0.f;
-                    *(__nv_bfloat16 *)(blk + kOffP + sw128_offset(r, s, 64)) = __float2bfloat16_rn(pv);
+        // Thread (cp, I): channels c0 = 2 cp and c0 + 1, sub-tile I = warp / 2.
+        const int cp = ((warp & 1) << 5) | lane, c0 = 2 * cp, I = warp >> 1;
+        uint32_t mma_count = 0;
+        int it = 0;
+        for (int w = blockIdx.x; w < total_items && !sAbort; w += gridDim.x, ++it) {
+            const int s = it & 1;
+            if (warp == 0) {
+                cp_async_wait_all();  // this item's beta values
+                if (w + (int)gridDim.x < total_items) {
+                    issue(w + gridDim.x, s ^ 1);
+                    issued = it + 2;
                 }
             }
-        }
-    }
-    tc_fence_before_sync();
-    __syncthreads();
+            if (!mbar_wait(&full[s], (it >> 1) & 1, globaltimer_ns() + kWaitNs)) {
+                if (tid == 0) record_timeout(status);
+                sAbort = 1;
+                break;
+            }
+            const IntraItem inf = info[s];
+            const int len = inf.len, h = inf.h;
+            const uint8_t *st = sm + kIRaw + s * kRawStage;
+            uint8_t *blk = blocks + ((size_t)h * max_chunks + inf.g) * kBlockBytes;
+            const float2 eA = make_float2(__expf(A[(size_t)h * kDK + c0]), __expf(A[(size_t)h * kDK + c0 + 1]));
 
-    // T = (I + A)^-1 by blocks of 16: diagonal blocks by forward substitution,
-    // then T_ij = -T_ii A_ij T_jj doubled from 16 to 32 to 64.
-    if (c < 64) {
-        const int I = c >> 4, j = c & 15, o = 16 * I;
-        float col[16];
+            // Pass 1: gate and cumulative log-decay of channels c0, c0 + 1 over this
+            // thread's sub-tile I (rows 16 I .. 16 I + 15), relative to the sub-tile
+            // start: L_r = G_r - m_I.
+            float2 L[16];
+            float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float x = (r == j) ? 1.f : 0.f;
+            for (int i = 0; i < 16; ++i) {
+                const int r = 16 * I + i;
+                if (r < len) {
+                    const float2 zz = ld_bf16x2_smem(st, kRawZ + r * 256 + 4 * cp);
+                    acc.x += gate_log_decay_fast(eA.x, zz.x);
+                    acc.y += gate_log_decay_fast(eA.y, zz.y);
+                }
+                L[i] = acc;
+            }
+            sTot[I][c0] = acc.x;
+            sTot[I][c0 + 1] = acc.y;
+            compute_sync();
+            // Sub-tile references m_J = G at the end of sub-tile J - 1 (m_0 = 0), G_C.
+            float2 mref[5];
+            mref[0] = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int s2 = 0; s2 < r; ++s2) x -= Af[(o + r) * kLd + o + s2] * col[s2];
-            col[r] = r < j ? 0.f : x;
-        }
-        for (int r = 0; r < 64; ++r) Tf[r * kLd + o + j] = (r >= o && r < o + 16) ? col[r - o] : 0.f;
-    }
-    __syncthreads();
-    // Level 1: blocks (1,0) and (3,2).  X = A_ij T_jj, then T_ij = -T_ii X.
-    for (int e = c; e < 2 * 256; e += kIntraThreads) {
-        const int p = e >> 8, r = (e >> 4) & 15, s2 = e & 15;
-        const int oi = 32 * p + 16, oj = 32 * p;
-        float x = 0.f;
+            for (int J = 0; J < 4; ++J)
+                mref[J + 1] = make_float2(mref[J].x + sTot[J][c0], mref[J].y + sTot[J][c0 + 1]);
+            const float2 mI = I == 0 ? mref[0] : I == 1 ? mref[1] : I == 2 ? mref[2] : mref[3];
+            const float2 GC = mref[4];
+            const float2 emI = make_float2(__expf(mI.x), __expf(mI.y));
+            const float2 egc = make_float2(__expf(GC.x - mI.x), __expf(GC.y - mI.y));
+            // fac[Ip] = e^{m_Ip - m_I} carries a column operand from sub-tile I's
+            // reference to a later sub-tile's (1 for Ip = I).
+            float2 fac[4];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) x += Af[(oi + r) * kLd + oj + t] * Tf[(oj + t) * kLd + oj + s2];
-        Xf[(16 * p + r) * 33 + s2] = x;
-    }
-    __syncthreads();
-    for (int e = c; e < 2 * 256; e += kIntraThreads) {
-        const int p = e >> 8, r = (e >> 4) & 15, s2 = e & 15;
-        const int oi = 32 * p + 16, oj = 32 * p;
-        float x = 0.f;
+            for (int Ip = 0; Ip < 4; ++Ip)
+                fac[Ip] = Ip > I ? make_float2(__expf(mref[Ip].x - mI.x), __expf(mref[Ip].y - mI.y))
+                                 : make_float2(1.f, 1.f);
+
+            // Pass 2: scaled operands of channels c0, c0 + 1 for the 16 rows.
+            uint8_t *sR = sm + kIRbig, *sKQ = sm + kIKQ;
+            uint32_t pk0[8], pk1[8], pv0[8], pv1[8], kd0[4], kd1[4];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) x += Tf[(oi + r) * kLd + oi + t] * Xf[(16 * p + t) * 33 + s2];
-        Tf[(oi + r) * kLd + oj + s2] = -x;
-    }
-    __syncthreads();
-    // Level 2: block rows 32..63, columns 0..31.
-    for (int e = c; e < 1024; e += kIntraThreads) {
-        const int r = e >> 5, s2 = e & 31;
-        float x = 0.f;
-#pragma unroll 8
-        for (int t = 0; t < 32; ++t) x += Af[(32 + r) * kLd + t] * Tf[t * kLd + s2];
-        Xf[r * 33 + s2] = x;
-    }
-    __syncthreads();
-    for (int e = c; e < 1024; e += kIntraThreads) {
-        const int r = e >> 5, s2 = e & 31;
-        float x = 0.f;
-#pragma unroll 8
-        for (int t = 0; t < 32; ++t) x += Tf[(32 + r) * kLd + 32 + t] * Xf[t * 33 + s2];
-        Tf[(32 + r) * kLd + s2] = -x;
-    }
-    __syncthreads();
-    // T as the bf16 A operand of the W/U product (64 rows x 64 K).
-    uint8_t *sT = sm + kITop;
-    for (int e = c; e < 64 * 64; e += kIntraThreads) {
-        const int r = e >> 6, s2 = e & 63;
-        *(__nv_bfloat16 *)(sT + sw128_offset(r, s2, 64)) = __float2bfloat16_rn(Tf[r * kLd + s2]);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-    if (c == 0 && !sAbort) {
-        const uint32_t id = idesc_bf16_f32(64, 256);
+            for (int i = 0; i < 16; ++i) {
+                const int r = 16 * I + i;
+                const bool valid = r < len;
+                const float2 kv = valid ? ld_bf16x2_smem(st, kRawK + r * 256 + 4 * cp) : make_float2(0.f, 0.f);
+                const float2 qv = valid ? ld_bf16x2_smem(st, kRawQ + r * 256 + 4 * cp) : make_float2(0.f, 0.f);
+                const float2 vv = valid ? ld_bf16x2_smem(st, kRawV + r * 256 + 4 * cp) : make_float2(0.f, 0.f);
+                const float2 e1 = make_float2(__expf(L[i].x), __expf(L[i].y));    // in [e^-80, 1]
+                const float2 e2 = make_float2(__expf(-L[i].x), __expf(-L[i].y));  // in [1, e^80]
+                const float br = sBeta[s][r];
+                *(uint32_t *)(sKQ + sw128_offset(32 * I + i, c0, 128)) = pack_bf16(kv.x * e1.x, kv.y * e1.y);
+                *(uint32_t *)(sKQ + sw128_offset(32 * I + 16 + i, c0, 128)) = pack_bf16(qv.x * e1.x, qv.y * e1.y);
+                const float2 kb = make_float2(kv.x * e2.x, kv.y * e2.y);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-            mma_ss(tmem_addr(tb, 0, 0), desc_kmajor_sw128(smem_u32(sT) + ks * 32),
-                   desc_kmajor_sw128(smem_u32(sB) + ks * 32), id, ks > 0);
-        mma_commit(&bar);
-    }
-    bool ok = !sAbort && mbar_wait(&bar, 1, deadline + kWaitNs);
-    if (!ok && !sAbort) record_timeout(status);
-    tc_fence_after_sync();
-    if (ok) {
-        // W -> rows 0..63 of the [W; Qt] tile, U -> row-major U.
-        uint32_t rr[32];
-        const int r = 16 * warp + lane;
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-            tmem_ld32(tmem_addr(tb, 32 * warp, 32 * q4), rr);
-            tmem_ld_wait();
-            if (lane < 16) {
-#pragma unroll
-                for (int cc = 0; cc < 32; cc += 8) {
-                    const uint4 w4 = make_uint4(pack_bf16(__uint_as_float(rr[cc]), __uint_as_float(rr[cc + 1])),
-                                                pack_bf16(__uint_as_float(rr[cc + 2]), __uint_as_float(rr[cc + 3])),
-                                                pack_bf16(__uint_as_float(rr[cc + 4]), __uint_as_float(rr[cc + 5])),
-                                                pack_bf16(__uint_as_float(rr[cc + 6]), __uint_as_float(rr[cc + 7])));
-                    const int col = 32 * q4 + cc;
-                    if (col < 128)
-                        *(uint4 *)(blk + kOffWQ + sw128_offset(r, col, 128)) = w4;
-                    else
-                        *(uint4 *)(blk + kOffU + (size_t)(r * 128 + col - 128) * 2) = w4;
+                for (int Ip = 0; Ip < 4; ++Ip)
+                    if (Ip >= I)
+                        *(uint32_t *)(sR + sw128_offset(row_base(Ip) + r, c0, 160)) =
+                            pack_bf16(kb.x * fac[Ip].x, kb.y * fac[Ip].y);
+                *(uint32_t *)(blk + kOffWQ + sw128_offset(64 + r, c0, 128)) =
+                    pack_bf16(qv.x * e1.x * emI.x, qv.y * e1.y * emI.y);
+                const uint32_t hk0 = bf16_bits(br * kv.x * e1.x * emI.x), hk1 = bf16_bits(br * kv.y * e1.y * emI.y);
+                const uint32_t hv0 = bf16_bits(br * vv.x), hv1 = bf16_bits(br * vv.y);
+                const uint32_t hd0 = bf16_bits(kb.x * egc.x), hd1 = bf16_bits(kb.y * egc.y);
+                if ((i & 1) == 0) {
+                    pk0[i >> 1] = hk0; pk1[i >> 1] = hk1; pv0[i >> 1] = hv0; pv1[i >> 1] = hv1;
+                    kd0[(i & 7) >> 1] = hd0; kd1[(i & 7) >> 1] = hd1;
+                } else {
+                    pk0[i >> 1] |= hk0 << 16; pk1[i >> 1] |= hk1 << 16;
+                    pv0[i >> 1] |= hv0 << 16; pv1[i >> 1] |= hv1 << 16;
+                    kd0[(i & 7) >> 1] |= hd0 << 16; kd1[(i & 7) >> 1] |= hd1 << 16;
+                }
+                if ((i & 7) == 7) {
+                    const int r0 = r - 7;
+                    *(uint4 *)(blk + kOffKd + sw128_offset(c0, r0, 128)) = make_uint4(kd0[0], kd0[1], kd0[2], kd0[3]);
+                    *(uint4 *)(blk + kOffKd + sw128_offset(c0 + 1, r0, 128)) = make_uint4(kd1[0], kd1[1], kd1[2], kd1[3]);
                 }
             }
+            if (I == 0) {
+                ((float *)(blk + kOffDecay))[c0] = __expf(GC.x);
+                ((float *)(blk + kOffDecay))[c0 + 1] = __expf(GC.y);
+            }
+
+            // A/P products: D[s][32 I + j] = R^(I)_s . Kt_{16I+j} (j < 16) and . Qt (j >= 16).
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            compute_sync();
+            tc_fence_after_sync();
+            if (tid == 0) {
+                const uint32_t id = idesc_bf16_f32(64, 32);
+#pragma unroll
+                for (int I = 0; I < 4; ++I)
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t kb2 = ks >> 2, kin = ks & 3;
+                        const uint32_t a = smem_u32(sR) + kb2 * 160 * 128 + row_base(I) * 128 + kin * 32;
+                        const uint32_t b = smem_u32(sKQ) + kb2 * 128 * 128 + 32 * I * 128 + kin * 32;
+                        mma_ss(tmem_addr(tb, 0, 32 * I), desc_kmajor_sw128(a), desc_kmajor_sw128(b), id, ks > 0);
+                    }
+                mma_commit(&mma_bar);
+            }
+            if (!mbar_wait(&mma_bar, mma_count & 1, globaltimer_ns() + kWaitNs)) {
+                if (tid == 0) record_timeout(status);
+                sAbort = 1;
+                break;
+            }
+            ++mma_count;
+            tc_fence_after_sync();
+
+            float *Af = (float *)(sm + kIAf), *Tf = (float *)(sm + kITf), *Xf = (float *)(sm + kIXf);
+            {
+                // M = 64 layout: warp (w % 4) lanes 0-15 hold rows s = 16 (w % 4) + lane;
+                // warps 0-3 read sub-tiles 0, 1 and warps 4-7 sub-tiles 2, 3.
+                uint32_t rr[32];
+                const int wq = warp & 3, sidx = 16 * wq + lane;
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    const int I = 2 * (warp >> 2) + jj;
+                    tmem_ld32(tmem_addr(tb, 32 * wq, 32 * I), rr);
+                    tmem_ld_wait();
+                    if (lane < 16) {
+#pragma unroll
+                        for (int jr = 0; jr < 16; ++jr) {
+                            const int r = 16 * I + jr;
+                            Af[r * kLd + sidx] = sidx < r ? sBeta[s][r] * __uint_as_float(rr[jr]) : 0.f;
+                            const float pvv = sidx <= r ? __uint_as_float(rr[16 + jr]) : 0.f;
+                            *(__nv_bfloat16 *)(blk + kOffP + sw128_offset(r, sidx, 64)) = __float2bfloat16_rn(pvv);
+                        }
+                    }
+                }
+            }
+            // [beta K e^G ; beta V]^T (256 rows x 64 tokens) into the freed [Kt; Qt] region.
+#pragma unroll
+            for (int g8 = 0; g8 < 2; ++g8) {
+                const int r0 = 16 * I + 8 * g8;
+                *(uint4 *)(sKQ + sw128_offset(c0, r0, 256)) =
+                    make_uint4(pk0[4 * g8], pk0[4 * g8 + 1], pk0[4 * g8 + 2], pk0[4 * g8 + 3]);
+                *(uint4 *)(sKQ + sw128_offset(c0 + 1, r0, 256)) =
+                    make_uint4(pk1[4 * g8], pk1[4 * g8 + 1], pk1[4 * g8 + 2], pk1[4 * g8 + 3]);
+                *(uint4 *)(sKQ + sw128_offset(128 + c0, r0, 256)) =
+                    make_uint4(pv0[4 * g8], pv0[4 * g8 + 1], pv0[4 * g8 + 2], pv0[4 * g8 + 3]);
+                *(uint4 *)(sKQ + sw128_offset(128 + c0 + 1, r0, 256)) =
+                    make_uint4(pv1[4 * g8], pv1[4 * g8 + 1], pv1[4 * g8 + 2], pv1[4 * g8 + 3]);
+            }
+            tc_fence_before_sync();
+            compute_sync();
+
+            // T = (I + A)^-1 by blocks of 16: diagonal blocks by forward
+            // substitution, then T_ij = -T_ii A_ij T_jj doubled from 16 to 32 to 64.
+            if (tid < 64) {
+                const int I = tid >> 4, jc = tid & 15, o = 16 * I;
+                float col[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    float x = (r == jc) ? 1.f : 0.f;
+#pragma unroll
+                    for (int s2 = 0; s2 < r; ++s2) x -= Af[(o + r) * kLd + o + s2] * col[s2];
+                    col[r] = r < jc ? 0.f : x;
+                }
+#pragma unroll
+                for (int blkr = 0; blkr < 4; ++blkr)
+#pragma unroll
+                    for (int r = 0; r < 16; ++r)
+                        Tf[(16 * blkr + r) * kLd + o + jc] = (blkr == I) ? col[r] : 0.f;
+            }
+            compute_sync();
+            for (int e = tid; e < 2 * 256; e += kIntraCompute) {
+                const int p = e >> 8, r = (e >> 4) & 15, s2 = e & 15;
+                const int oi = 32 * p + 16, oj = 32 * p;
+                float x = 0.f;
+#pragma unroll
+                for (int t = 0; t < 16; ++t) x += Af[(oi + r) * kLd + oj + t] * Tf[(oj + t) * kLd + oj + s2];
+                Xf[(16 * p + r) * 33 + s2] = x;
+            }
+            compute_sync();
+            for (int e = tid; e < 2 * 256; e += kIntraCompute) {
+                const int p = e >> 8, r = (e >> 4) & 15, s2 = e & 15;
+                const int oi = 32 * p + 16, oj = 32 * p;
+                float x = 0.f;
+#pragma unroll
+                for (int t = 0; t < 16; ++t) x += Tf[(oi + r) * kLd + oi + t] * Xf[(16 * p + t) * 33 + s2];
+                Tf[(oi + r) * kLd + oj + s2] = -x;
+            }
+            compute_sync();
+            for (int e = tid; e < 1024; e += kIntraCompute) {
+                const int r = e >> 5, s2 = e & 31;
+                float x = 0.f;
+#pragma unroll 8
+                for (int t = 0; t < 32; ++t) x += Af[(32 + r) * kLd + t] * Tf[t * kLd + s2];
+                Xf[r * 33 + s2] = x;
+            }
+            compute_sync();
+            for (int e = tid; e < 1024; e += kIntraCompute) {
+                const int r = e >> 5, s2 = e & 31;
+                float x = 0.f;
+#pragma unroll 8
+                for (int t = 0; t < 32; ++t) x += Tf[(32 + r) * kLd + 32 + t] * Xf[t * 33 + s2];
+                Tf[(32 + r) * kLd + s2] = -x;
+            }
+            compute_sync();
+            // T as the bf16 A operand (64 rows x 64 K) in the item's raw z tile.
+            uint8_t *sT = sm + kIRaw + s * kRawStage + kRawZ;
+            for (int e = tid; e < 64 * 64; e += kIntraCompute) {
+                const int r = e >> 6, s2 = e & 63;
+                *(__nv_bfloat16 *)(sT + sw128_offset(r, s2, 64)) = __float2bfloat16_rn(Tf[r * kLd + s2]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            compute_sync();
+            tc_fence_after_sync();
+            if (tid == 0) {
+                const uint32_t id = idesc_bf16_f32(64, 256);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_ss(tmem_addr(tb, 0, 0), desc_kmajor_sw128(smem_u32(sT) + ks * 32),
+                           desc_kmajor_sw128(smem_u32(sKQ) + ks * 32), id, ks > 0);
+                mma_commit(&mma_bar);
+            }
+            if (!mbar_wait(&mma_bar, mma_count & 1, globaltimer_ns() + kWaitNs)) {
+                if (tid == 0) record_timeout(status);
+                sAbort = 1;
+                break;
+            }
+            ++mma_count;
+            tc_fence_after_sync();
+            {
+                // W (columns 0..127, warps 0-3) -> rows 0..63 of [W; Qt]; U (128..255, warps 4-7).
+                uint32_t rr[32];
+                const int wq = warp & 3, r = 16 * wq + lane, part = warp >> 2;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    tmem_ld32(tmem_addr(tb, 32 * wq, 128 * part + 32 * q4), rr);
+                    tmem_ld_wait();
+                    if (lane < 16) {
+#pragma unroll
+                        for (int cc = 0; cc < 32; cc += 8) {
+                            const uint4 w4 = make_uint4(
+                                pack_bf16(__uint_as_float(rr[cc]), __uint_as_float(rr[cc + 1])),
+                                pack_bf16(__uint_as_float(rr[cc + 2]), __uint_as_float(rr[cc + 3])),
+                                pack_bf16(__uint_as_float(rr[cc + 4]), __uint_as_float(rr[cc + 5])),
+                                pack_bf16(__uint_as_float(rr[cc + 6]), __uint_as_float(rr[cc + 7])));
+                            const int col = 32 * q4 + cc;
+                            if (part == 0)
+                                *(uint4 *)(blk + kOffWQ + sw128_offset(r, col, 128)) = w4;
+                            else
+                                *(uint4 *)(blk + kOffU + (size_t)(r * 128 + col) * 2) = w4;
+                        }
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            compute_sync();
+        }
+        // Drain: every requested copy has landed before the CTA may exit.
+        if (warp == 0) {
+            cp_async_wait_all();
+            for (int d = it; d < issued; ++d)
+                mbar_wait(&full[d & 1], (d >> 1) & 1, globaltimer_ns() + kWaitNs);
         }
     }
     tc_fence_before_sync();
@@ -639,6 +777,37 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
     if (warp == 0) tmem_dealloc(tb, 512);
 }
 
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime (no
+// link-time dependency on libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+    });
+    return fn;
+}
+
+// [T][H][128] bf16 rows viewed as a 3-D tensor (channel, head, token) with a
+// {128, 1, 64} box: one chunk of one head per load, no swizzle.
+bool encode_rows_map(CUtensorMap *map, const void *base, int32_t T, int32_t H)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)kDK, (cuuint64_t)H, (cuuint64_t)(T > 0 ? T : 1)};
+    const cuuint64_t strides[2] = {(cuuint64_t)kDK * 2, (cuuint64_t)H * kDK * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)kDK, 1, (cuuint32_t)kChunk};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 size_t tc_workspace_bytes(int32_t total_tokens, int32_t num_seqs, int32_t H)
@@ -672,12 +841,18 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
 
-    const int ismem = kISmem + 1024;
     if (max_chunks > 0) {
-        dim3 grid((unsigned)max_chunks, (unsigned)a.H);
-        intra_kernel<<<grid, kIntraThreads, ismem, stream>>>(
-            (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.v,
-            (const __nv_bfloat16 *)a.z, a.A, a.beta, a.cu_seqlens, chunk_off, a.num_seqs, a.H,
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int64_t items = max_chunks * a.H;
+        const unsigned grid = (unsigned)(items < sms ? items : sms);
+        CUtensorMap mk, mq, mv, mz;
+        if (!encode_rows_map(&mk, a.k, a.total_tokens, a.H) || !encode_rows_map(&mq, a.q, a.total_tokens, a.H) ||
+            !encode_rows_map(&mv, a.v, a.total_tokens, a.H) || !encode_rows_map(&mz, a.z, a.total_tokens, a.H))
+            return cudaErrorInvalidValue;
+        intra_kernel<<<grid, kIntraThreads, kISmem + 1024, stream>>>(
+            mk, mq, mv, mz, a.A, a.beta, a.cu_seqlens, chunk_off, a.num_seqs, a.H,
             blocks, max_chunks, a.status);
         err = cudaGetLastError();
         if (err != cudaSuccess) return err;
