@@ -120,9 +120,10 @@ plan_kernel(const int32_t *__restrict__ cu, int N, int32_t *__restrict__ chunk_o
 // item w is chunk w / H of head w % H.  While an item is computed, warp 0
 // prefetches the next item's raw k, q, v, z rows (256 B each) into the other
 // stage of a two-stage ring with bulk copies, and its beta values with
-// cp.async.  Thread (cp, I) owns channels 2 cp, 2 cp + 1 of sub-tile I = warp / 2
-// (rows 16 I .. 16 I + 15), so the sub-tile index is uniform across a warp.
-constexpr int kIntraCompute = 256;
+// cp.async.  Thread (cp, q8) owns channels 2 cp, 2 cp + 1 of the eight rows
+// 8 q8 .. 8 q8 + 7 (q8 = warp / 2), inside sub-tile I = q8 / 2, so the
+// sub-tile index is uniform across a warp.
+constexpr int kIntraCompute = 512;
 constexpr int kIntraThreads = kIntraCompute;
 constexpr uint32_t kRawTile = kChunk * kDK * 2;    // one [64][128] bf16 tile, 16 KiB
 constexpr uint32_t kRawStage = 4 * kRawTile;       // k, q, v, z
@@ -200,7 +201,7 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     __shared__ uint32_t tbase;
     __shared__ IntraItem info[2];
     __shared__ float sBeta[2][kChunk];
-    __shared__ float sTot[4][kDK];
+    __shared__ float sTot[8][kDK];
     __shared__ volatile int sAbort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -244,19 +245,13 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     int issued = 1;  // items requested so far (meaningful in warp 0)
 
     {
-        // Thread (cp, I): channels c0 = 2 cp and c0 + 1, sub-tile I = warp / 2.
-        const int cp = ((warp & 1) << 5) | lane, c0 = 2 * cp, I = warp >> 1;
+        // Thread (cp, q8): channels c0 = 2 cp and c0 + 1, rows 8 q8 .. 8 q8 + 7, sub-tile I.
+        const int cp = ((warp & 1) << 5) | lane, c0 = 2 * cp, q8 = warp >> 1, I = q8 >> 1;
         uint32_t mma_count = 0;
         int it = 0;
         for (int w = blockIdx.x; w < total_items && !sAbort; w += gridDim.x, ++it) {
             const int s = it & 1;
-            if (warp == 0) {
-                cp_async_wait_all();  // this item's beta values
-                if (w + (int)gridDim.x < total_items) {
-                    issue(w + gridDim.x, s ^ 1);
-                    issued = it + 2;
-                }
-            }
+            if (warp == 0) cp_async_wait_all();  // this item's beta values (issued one item ago)
             if (!mbar_wait(&full[s], (it >> 1) & 1, globaltimer_ns() + kWaitNs)) {
                 if (tid == 0) record_timeout(status);
                 sAbort = 1;
@@ -268,14 +263,13 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             uint8_t *blk = blocks + ((size_t)h * max_chunks + inf.g) * kBlockBytes;
             const float2 eA = make_float2(__expf(A[(size_t)h * kDK + c0]), __expf(A[(size_t)h * kDK + c0 + 1]));
 
-            // Pass 1: gate and cumulative log-decay of channels c0, c0 + 1 over this
-            // thread's sub-tile I (rows 16 I .. 16 I + 15), relative to the sub-tile
-            // start: L_r = G_r - m_I.
-            float2 L[16];
+            // Pass 1: gate and cumulative log-decay of channels c0, c0 + 1 over the
+            // eight rows, then relative to the sub-tile start: L_r = G_r - m_I.
+            float2 L[8];
             float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = 16 * I + i;
+            for (int i = 0; i < 8; ++i) {
+                const int r = 8 * q8 + i;
                 if (r < len) {
                     const float2 zz = ld_bf16x2_smem(st, kRawZ + r * 256 + 4 * cp);
                     acc.x += gate_log_decay_fast(eA.x, zz.x);
@@ -283,15 +277,21 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 }
                 L[i] = acc;
             }
-            sTot[I][c0] = acc.x;
-            sTot[I][c0 + 1] = acc.y;
+            sTot[q8][c0] = acc.x;
+            sTot[q8][c0 + 1] = acc.y;
             compute_sync();
+            if (q8 & 1) {
+                const float ox = sTot[q8 - 1][c0], oy = sTot[q8 - 1][c0 + 1];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) { L[i].x += ox; L[i].y += oy; }
+            }
             // Sub-tile references m_J = G at the end of sub-tile J - 1 (m_0 = 0), G_C.
             float2 mref[5];
             mref[0] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int J = 0; J < 4; ++J)
-                mref[J + 1] = make_float2(mref[J].x + sTot[J][c0], mref[J].y + sTot[J][c0 + 1]);
+                mref[J + 1] = make_float2(mref[J].x + sTot[2 * J][c0] + sTot[2 * J + 1][c0],
+                                          mref[J].y + sTot[2 * J][c0 + 1] + sTot[2 * J + 1][c0 + 1]);
             const float2 mI = I == 0 ? mref[0] : I == 1 ? mref[1] : I == 2 ? mref[2] : mref[3];
             const float2 GC = mref[4];
             const float2 emI = make_float2(__expf(mI.x), __expf(mI.y));
@@ -304,12 +304,12 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 fac[Ip] = Ip > I ? make_float2(__expf(mref[Ip].x - mI.x), __expf(mref[Ip].y - mI.y))
                                  : make_float2(1.f, 1.f);
 
-            // Pass 2: scaled operands of channels c0, c0 + 1 for the 16 rows.
+            // Pass 2: scaled operands of channels c0, c0 + 1 for the eight rows.
             uint8_t *sR = sm + kIRbig, *sKQ = sm + kIKQ;
-            uint32_t pk0[8], pk1[8], pv0[8], pv1[8], kd0[4], kd1[4];
+            uint32_t pk0[4], pk1[4], pv0[4], pv1[4], kd0[4], kd1[4];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = 16 * I + i;
+            for (int i = 0; i < 8; ++i) {
+                const int r = 8 * q8 + i, ri = r & 15;
                 const bool valid = r < len;
                 const float2 kv = valid ? ld_bf16x2_smem(st, kRawK + r * 256 + 4 * cp) : make_float2(0.f, 0.f);
                 const float2 qv = valid ? ld_bf16x2_smem(st, kRawQ + r * 256 + 4 * cp) : make_float2(0.f, 0.f);
@@ -317,8 +317,8 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 const float2 e1 = make_float2(__expf(L[i].x), __expf(L[i].y));    // in [e^-80, 1]
                 const float2 e2 = make_float2(__expf(-L[i].x), __expf(-L[i].y));  // in [1, e^80]
                 const float br = sBeta[s][r];
-                *(uint32_t *)(sKQ + sw128_offset(32 * I + i, c0, 128)) = pack_bf16(kv.x * e1.x, kv.y * e1.y);
-                *(uint32_t *)(sKQ + sw128_offset(32 * I + 16 + i, c0, 128)) = pack_bf16(qv.x * e1.x, qv.y * e1.y);
+                *(uint32_t *)(sKQ + sw128_offset(32 * I + ri, c0, 128)) = pack_bf16(kv.x * e1.x, kv.y * e1.y);
+                *(uint32_t *)(sKQ + sw128_offset(32 * I + 16 + ri, c0, 128)) = pack_bf16(qv.x * e1.x, qv.y * e1.y);
                 const float2 kb = make_float2(kv.x * e2.x, kv.y * e2.y);
 #pragma unroll
                 for (int Ip = 0; Ip < 4; ++Ip)
@@ -332,19 +332,16 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 const uint32_t hd0 = bf16_bits(kb.x * egc.x), hd1 = bf16_bits(kb.y * egc.y);
                 if ((i & 1) == 0) {
                     pk0[i >> 1] = hk0; pk1[i >> 1] = hk1; pv0[i >> 1] = hv0; pv1[i >> 1] = hv1;
-                    kd0[(i & 7) >> 1] = hd0; kd1[(i & 7) >> 1] = hd1;
+                    kd0[i >> 1] = hd0; kd1[i >> 1] = hd1;
                 } else {
                     pk0[i >> 1] |= hk0 << 16; pk1[i >> 1] |= hk1 << 16;
                     pv0[i >> 1] |= hv0 << 16; pv1[i >> 1] |= hv1 << 16;
-                    kd0[(i & 7) >> 1] |= hd0 << 16; kd1[(i & 7) >> 1] |= hd1 << 16;
-                }
-                if ((i & 7) == 7) {
-                    const int r0 = r - 7;
-                    *(uint4 *)(blk + kOffKd + sw128_offset(c0, r0, 128)) = make_uint4(kd0[0], kd0[1], kd0[2], kd0[3]);
-                    *(uint4 *)(blk + kOffKd + sw128_offset(c0 + 1, r0, 128)) = make_uint4(kd1[0], kd1[1], kd1[2], kd1[3]);
+                    kd0[i >> 1] |= hd0 << 16; kd1[i >> 1] |= hd1 << 16;
                 }
             }
-            if (I == 0) {
+            *(uint4 *)(blk + kOffKd + sw128_offset(c0, 8 * q8, 128)) = make_uint4(kd0[0], kd0[1], kd0[2], kd0[3]);
+            *(uint4 *)(blk + kOffKd + sw128_offset(c0 + 1, 8 * q8, 128)) = make_uint4(kd1[0], kd1[1], kd1[2], kd1[3]);
+            if (q8 == 0) {
                 ((float *)(blk + kOffDecay))[c0] = __expf(GC.x);
                 ((float *)(blk + kOffDecay))[c0 + 1] = __expf(GC.y);
             }
@@ -367,6 +364,12 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                     }
                 mma_commit(&mma_bar);
             }
+            // While the products run, warp 0 requests the next item into the other
+            // stage (free: its previous item finished with it).
+            if (warp == 0 && w + (int)gridDim.x < total_items) {
+                issue(w + gridDim.x, s ^ 1);
+                issued = it + 2;
+            }
             if (!mbar_wait(&mma_bar, mma_count & 1, globaltimer_ns() + kWaitNs)) {
                 if (tid == 0) record_timeout(status);
                 sAbort = 1;
@@ -378,99 +381,106 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             float *Af = (float *)(sm + kIAf), *Tf = (float *)(sm + kITf), *Xf = (float *)(sm + kIXf);
             {
                 // M = 64 layout: warp (w % 4) lanes 0-15 hold rows s = 16 (w % 4) + lane;
-                // warps 0-3 read sub-tiles 0, 1 and warps 4-7 sub-tiles 2, 3.
+                // warp w reads sub-tile w / 4.
                 uint32_t rr[32];
-                const int wq = warp & 3, sidx = 16 * wq + lane;
+                const int wq = warp & 3, sidx = 16 * wq + lane, Ia = warp >> 2;
+                tmem_ld32(tmem_addr(tb, 32 * wq, 32 * Ia), rr);
+                tmem_ld_wait();
+                if (lane < 16) {
 #pragma unroll
-                for (int jj = 0; jj < 2; ++jj) {
-                    const int I = 2 * (warp >> 2) + jj;
-                    tmem_ld32(tmem_addr(tb, 32 * wq, 32 * I), rr);
-                    tmem_ld_wait();
-                    if (lane < 16) {
-#pragma unroll
-                        for (int jr = 0; jr < 16; ++jr) {
-                            const int r = 16 * I + jr;
-                            Af[r * kLd + sidx] = sidx < r ? sBeta[s][r] * __uint_as_float(rr[jr]) : 0.f;
-                            const float pvv = sidx <= r ? __uint_as_float(rr[16 + jr]) : 0.f;
-                            *(__nv_bfloat16 *)(blk + kOffP + sw128_offset(r, sidx, 64)) = __float2bfloat16_rn(pvv);
-                        }
+                    for (int jr = 0; jr < 16; ++jr) {
+                        const int r = 16 * Ia + jr;
+                        Af[r * kLd + sidx] = sidx < r ? sBeta[s][r] * __uint_as_float(rr[jr]) : 0.f;
+                        const float pvv = sidx <= r ? __uint_as_float(rr[16 + jr]) : 0.f;
+                        *(__nv_bfloat16 *)(blk + kOffP + sw128_offset(r, sidx, 64)) = __float2bfloat16_rn(pvv);
                     }
                 }
             }
             // [beta K e^G ; beta V]^T (256 rows x 64 tokens) into the freed [Kt; Qt] region.
-#pragma unroll
-            for (int g8 = 0; g8 < 2; ++g8) {
-                const int r0 = 16 * I + 8 * g8;
-                *(uint4 *)(sKQ + sw128_offset(c0, r0, 256)) =
-                    make_uint4(pk0[4 * g8], pk0[4 * g8 + 1], pk0[4 * g8 + 2], pk0[4 * g8 + 3]);
-                *(uint4 *)(sKQ + sw128_offset(c0 + 1, r0, 256)) =
-                    make_uint4(pk1[4 * g8], pk1[4 * g8 + 1], pk1[4 * g8 + 2], pk1[4 * g8 + 3]);
-                *(uint4 *)(sKQ + sw128_offset(128 + c0, r0, 256)) =
-                    make_uint4(pv0[4 * g8], pv0[4 * g8 + 1], pv0[4 * g8 + 2], pv0[4 * g8 + 3]);
-                *(uint4 *)(sKQ + sw128_offset(128 + c0 + 1, r0, 256)) =
-                    make_uint4(pv1[4 * g8], pv1[4 * g8 + 1], pv1[4 * g8 + 2], pv1[4 * g8 + 3]);
-            }
+            *(uint4 *)(sKQ + sw128_offset(c0, 8 * q8, 256)) = make_uint4(pk0[0], pk0[1], pk0[2], pk0[3]);
+            *(uint4 *)(sKQ + sw128_offset(c0 + 1, 8 * q8, 256)) = make_uint4(pk1[0], pk1[1], pk1[2], pk1[3]);
+            *(uint4 *)(sKQ + sw128_offset(128 + c0, 8 * q8, 256)) = make_uint4(pv0[0], pv0[1], pv0[2], pv0[3]);
+            *(uint4 *)(sKQ + sw128_offset(128 + c0 + 1, 8 * q8, 256)) = make_uint4(pv1[0], pv1[1], pv1[2], pv1[3]);
             tc_fence_before_sync();
             compute_sync();
 
+            // T, rounded to bf16, is also the A operand of the W/U product
+            // (64 rows x 64 K), written into the item's raw z tile as it is formed.
+            uint8_t *sT = sm + kIRaw + s * kRawStage + kRawZ;
             // T = (I + A)^-1 by blocks of 16: diagonal blocks by forward
             // substitution, then T_ij = -T_ii A_ij T_jj doubled from 16 to 32 to 64.
+            // Only the lower triangle is used; the two upper blocks that the
+            // doubling products read, (0,1) and (2,3), are set to zero.
             if (tid < 64) {
-                const int I = tid >> 4, jc = tid & 15, o = 16 * I;
+                const int Ib = tid >> 4, jc = tid & 15, o = 16 * Ib;
                 float col[16];
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
                     float x = (r == jc) ? 1.f : 0.f;
 #pragma unroll
-                    for (int s2 = 0; s2 < r; ++s2) x -= Af[(o + r) * kLd + o + s2] * col[s2];
+                    for (int s2 = 0; s2 < r; ++s2) x = fmaf(-Af[(o + r) * kLd + o + s2], col[s2], x);
                     col[r] = r < jc ? 0.f : x;
                 }
 #pragma unroll
-                for (int blkr = 0; blkr < 4; ++blkr)
-#pragma unroll
-                    for (int r = 0; r < 16; ++r)
-                        Tf[(16 * blkr + r) * kLd + o + jc] = (blkr == I) ? col[r] : 0.f;
+                for (int r = 0; r < 16; ++r) {
+                    Tf[(o + r) * kLd + o + jc] = col[r];
+                    *(__nv_bfloat16 *)(sT + sw128_offset(o + r, o + jc, 64)) = __float2bfloat16_rn(col[r]);
+                }
+            } else {
+                const int e = tid - 64;  // the other threads zero the upper blocks
+                for (int f = e; f < 512; f += kIntraCompute - 64) {
+                    const int blkz = f >> 8, r = (f >> 4) & 15, cz = f & 15;
+                    const int ro = 32 * blkz, co = 32 * blkz + 16;
+                    Tf[(ro + r) * kLd + co + cz] = 0.f;   // read by the doubling products
+                }
+                for (int f = e; f < 6 * 256; f += kIntraCompute - 64) {
+                    const int bz = f >> 8, r = (f >> 4) & 15, cz = f & 15;
+                    // upper blocks (0,1) (0,2) (0,3) (1,2) (1,3) (2,3) of the bf16 operand
+                    const int bi = bz < 3 ? 0 : bz < 5 ? 1 : 2;
+                    const int bj = bz < 3 ? bz + 1 : bz < 5 ? bz - 1 : 3;
+                    *(__nv_bfloat16 *)(sT + sw128_offset(16 * bi + r, 16 * bj + cz, 64)) = __float2bfloat16_rn(0.f);
+                }
             }
             compute_sync();
-            for (int e = tid; e < 2 * 256; e += kIntraCompute) {
-                const int p = e >> 8, r = (e >> 4) & 15, s2 = e & 15;
+            {
+                // Level 1, blocks (1,0) and (3,2): X = A_ij T_jj, one output per thread.
+                const int p = tid >> 8, r = (tid >> 4) & 15, sb = tid & 15;
                 const int oi = 32 * p + 16, oj = 32 * p;
-                float x = 0.f;
+                float x0 = 0.f;
 #pragma unroll
-                for (int t = 0; t < 16; ++t) x += Af[(oi + r) * kLd + oj + t] * Tf[(oj + t) * kLd + oj + s2];
-                Xf[(16 * p + r) * 33 + s2] = x;
-            }
-            compute_sync();
-            for (int e = tid; e < 2 * 256; e += kIntraCompute) {
-                const int p = e >> 8, r = (e >> 4) & 15, s2 = e & 15;
-                const int oi = 32 * p + 16, oj = 32 * p;
-                float x = 0.f;
+                for (int t = 0; t < 16; ++t) x0 = fmaf(Af[(oi + r) * kLd + oj + t], Tf[(oj + t) * kLd + oj + sb], x0);
+                Xf[(16 * p + r) * 33 + sb] = x0;
+                compute_sync();
+                float y0 = 0.f;
 #pragma unroll
-                for (int t = 0; t < 16; ++t) x += Tf[(oi + r) * kLd + oi + t] * Xf[(16 * p + t) * 33 + s2];
-                Tf[(oi + r) * kLd + oj + s2] = -x;
+                for (int t = 0; t < 16; ++t) y0 = fmaf(Tf[(oi + r) * kLd + oi + t], Xf[(16 * p + t) * 33 + sb], y0);
+                Tf[(oi + r) * kLd + oj + sb] = -y0;
+                *(__nv_bfloat16 *)(sT + sw128_offset(oi + r, oj + sb, 64)) = __float2bfloat16_rn(-y0);
             }
             compute_sync();
-            for (int e = tid; e < 1024; e += kIntraCompute) {
-                const int r = e >> 5, s2 = e & 31;
-                float x = 0.f;
+            {
+                // Level 2, block rows 32..63 x columns 0..31: two outputs per thread.
+                const int r = tid >> 4, sb = tid & 15;
+                float x[2] = {0.f, 0.f};
 #pragma unroll 8
-                for (int t = 0; t < 32; ++t) x += Af[(32 + r) * kLd + t] * Tf[t * kLd + s2];
-                Xf[r * 33 + s2] = x;
-            }
-            compute_sync();
-            for (int e = tid; e < 1024; e += kIntraCompute) {
-                const int r = e >> 5, s2 = e & 31;
-                float x = 0.f;
+                for (int t = 0; t < 32; ++t) {
+                    const float a = Af[(32 + r) * kLd + t];
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) x[jj] = fmaf(a, Tf[t * kLd + sb + 16 * jj], x[jj]);
+                }
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) Xf[r * 33 + sb + 16 * jj] = x[jj];
+                compute_sync();
+                float y[2] = {0.f, 0.f};
 #pragma unroll 8
-                for (int t = 0; t < 32; ++t) x += Tf[(32 + r) * kLd + 32 + t] * Xf[t * 33 + s2];
-                Tf[(32 + r) * kLd + s2] = -x;
-            }
-            compute_sync();
-            // T as the bf16 A operand (64 rows x 64 K) in the item's raw z tile.
-            uint8_t *sT = sm + kIRaw + s * kRawStage + kRawZ;
-            for (int e = tid; e < 64 * 64; e += kIntraCompute) {
-                const int r = e >> 6, s2 = e & 63;
-                *(__nv_bfloat16 *)(sT + sw128_offset(r, s2, 64)) = __float2bfloat16_rn(Tf[r * kLd + s2]);
+                for (int t = 0; t < 32; ++t) {
+                    const float tt = Tf[(32 + r) * kLd + 32 + t];
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) y[jj] = fmaf(tt, Xf[t * 33 + sb + 16 * jj], y[jj]);
+                }
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj)
+                    *(__nv_bfloat16 *)(sT + sw128_offset(32 + r, sb + 16 * jj, 64)) = __float2bfloat16_rn(-y[jj]);
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
@@ -492,12 +502,14 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             ++mma_count;
             tc_fence_after_sync();
             {
-                // W (columns 0..127, warps 0-3) -> rows 0..63 of [W; Qt]; U (128..255, warps 4-7).
+                // W (columns 0..127) -> rows 0..63 of [W; Qt]; U (columns 128..255).
+                // Warp w: lane quadrant w % 4, columns 64 (w / 4) .. + 63.
                 uint32_t rr[32];
-                const int wq = warp & 3, r = 16 * wq + lane, part = warp >> 2;
+                const int wq = warp & 3, r = 16 * wq + lane, cg = warp >> 2;
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    tmem_ld32(tmem_addr(tb, 32 * wq, 128 * part + 32 * q4), rr);
+                for (int q4 = 0; q4 < 2; ++q4) {
+                    const int colbase = 64 * cg + 32 * q4;
+                    tmem_ld32(tmem_addr(tb, 32 * wq, colbase), rr);
                     tmem_ld_wait();
                     if (lane < 16) {
 #pragma unroll
@@ -507,11 +519,11 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                                 pack_bf16(__uint_as_float(rr[cc + 2]), __uint_as_float(rr[cc + 3])),
                                 pack_bf16(__uint_as_float(rr[cc + 4]), __uint_as_float(rr[cc + 5])),
                                 pack_bf16(__uint_as_float(rr[cc + 6]), __uint_as_float(rr[cc + 7])));
-                            const int col = 32 * q4 + cc;
-                            if (part == 0)
+                            const int col = colbase + cc;
+                            if (col < 128)
                                 *(uint4 *)(blk + kOffWQ + sw128_offset(r, col, 128)) = w4;
                             else
-                                *(uint4 *)(blk + kOffU + (size_t)(r * 128 + col) * 2) = w4;
+                                *(uint4 *)(blk + kOffU + (size_t)(r * 128 + col - 128) * 2) = w4;
                         }
                     }
                 }
