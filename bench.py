@@ -121,9 +121,24 @@ def _traffic(kernel_file: str, kernel: str, units: int):
         return None
     with open(path) as f:
         rec = json.load(f).get(kernel)
-    if not rec or rec.get("source_sha") != _source_sha(kernel_file):
+    if not isinstance(rec, dict) or rec.get("source_sha") != _source_sha(kernel_file):
         return None
     return rec["dram_bytes_per_token_head"] * units
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Seed of rank `rank`'s independent problem (weak scaling: one problem per GPU)."""
+    return base + 1000 * rank
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The slowest rank's time; every rank takes part (same collective order)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def cpu_oracle_sample(inp, target_s: float, max_heads: int = 96):
@@ -231,16 +246,9 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     cfg = CONFIGS[args.workload]
     from dataclasses import replace
-    inp = config_inputs(replace(cfg, seed=cfg.seed + 1000 * rank), device=dev)
+    inp = config_inputs(replace(cfg, seed=rank_seed(cfg.seed, rank)), device=dev)
     T, H, dk, dv = inp["q"].shape[0], cfg.H, cfg.dk, cfg.dv
     stream = torch.cuda.current_stream()
     o = torch.empty(T, H, dv, dtype=torch.bfloat16, device=dev)
@@ -278,7 +286,7 @@ def main():
     total_ms = evs[0][0].elapsed_time(evs[-1][-1])
     per_kernel_ms = [statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
                      for j in range(nk)]
-    total_ms = max_over_ranks(total_ms)
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
     tokens = T * world
     value = tokens / (ms_per_step / 1e3)
@@ -308,7 +316,7 @@ def main():
     if not args.prefill_only:
         # Decode step: B=256 cached states, H=96, updated in place; GB/s of state traffic.
         dcfg = CONFIGS["decode_256"]
-        d = decode_inputs(dcfg.B, dcfg.H, dcfg.dk, dcfg.dv, dcfg.dtype, seed=dcfg.seed + 1000 * rank,
+        d = decode_inputs(dcfg.B, dcfg.H, dcfg.dk, dcfg.dv, dcfg.dtype, seed=rank_seed(dcfg.seed, rank),
                           nsets=dcfg.nsets, device=dev)
         od = torch.empty(dcfg.B, dcfg.H, dcfg.dv, dtype=torch.bfloat16, device=dev)
 
@@ -327,7 +335,7 @@ def main():
             dstep(i)
         e1.record(stream)
         torch.cuda.synchronize()
-        dms = max_over_ranks(e0.elapsed_time(e1)) / args.decode_steps
+        dms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.decode_steps
         state_bytes = 2 * dcfg.B * dcfg.H * dcfg.dk * dcfg.dv * 4
         dgbs = state_bytes / (dms / 1e3) / 1e9
         decode = {"config": dcfg.name, "ms_per_step": dms, "state_gbs": dgbs,
@@ -363,7 +371,7 @@ def main():
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = max_over_ranks(e0.elapsed_time(e1)) / args.e2e_steps
+        ems = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.e2e_steps
         e2e = {"value": tokens / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": args.e2e_steps}
 

@@ -197,6 +197,16 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
  */
 kda_status kda_device_status(void *stream, int32_t *status_out);
 
+/*
+ * Failure-detection self-test (a diagnostic with no counterpart in the source
+ * pages).  Enqueues one CTA whose mbarrier wait has nothing to complete it; the
+ * wait gives up after limit_ns (1 ms .. 10 s, else KDA_ERR_INVALID_ARG), writes
+ * KDA_ERR_TIMEOUT into the device status word and the kernel exits normally, so
+ * the context stays usable.  kda_device_status then reports KDA_ERR_TIMEOUT.
+ * It exercises the same bounded-wait path every tensor-core kernel uses.
+ */
+kda_status kda_selftest_wait_timeout(int64_t limit_ns, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -34,6 +34,7 @@ SIGNATURES = {
     "kda_prefill_noalloc": ([_P] * 8 + [_I32] * 6 + [_P] * 4, _I32),
     "kda_decode_step": ([_P] * 6 + [_I32] * 5 + [_P, _I32, _P, _P, _P], _I32),
     "kda_device_status": ([_P, _P], _I32),
+    "kda_selftest_wait_timeout": ([ctypes.c_int64, _P], _I32),
 }
 
 
@@ -190,6 +191,12 @@ def kda_decode_step(q, k, v, z, A, beta, state, slots=None, o=None, stream=None)
         _dev(slots, "slots", torch.int32), _dev(o, "o", dt), _stream_ptr(stream))
     _check(code, "kda_decode_step")
     return o
+
+
+def kda_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Enqueue the bounded-wait self-test; read the result with kda_device_status()."""
+    _check(_lib.kda_selftest_wait_timeout(int(limit_ns), _stream_ptr(stream)),
+           "kda_selftest_wait_timeout")
 
 
 def kda_device_status(stream=None) -> int:

@@ -192,3 +192,14 @@ extern "C" kda_status kda_device_status(void *stream, int32_t *status_out)
     *status_out = v;
     return KDA_OK;
 }
+
+extern "C" kda_status kda_selftest_wait_timeout(int64_t limit_ns, void *stream)
+{
+    if (limit_ns < 1000000LL || limit_ns > 10000000000LL) return KDA_ERR_INVALID_ARG;
+    int32_t *word = nullptr;
+    kda_status st = status_word(&word);
+    if (st != KDA_OK) return st;
+    return kda::launch_wait_timeout_selftest(word, limit_ns, (cudaStream_t)stream) == cudaSuccess
+               ? KDA_OK
+               : KDA_ERR_CUDA;
+}

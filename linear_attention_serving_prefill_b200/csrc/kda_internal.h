@@ -42,6 +42,9 @@ struct DecodeArgs {
 // Fused chunked prefill on CUDA cores, all arithmetic in fp32 (16-token chunks).
 cudaError_t launch_prefill_cuda_core(const PrefillArgs &a, cudaStream_t stream);
 
+// One-CTA kernel whose bounded mbarrier wait is never satisfied (records a timeout).
+cudaError_t launch_wait_timeout_selftest(int32_t *status, int64_t limit_ns, cudaStream_t stream);
+
 // Single-token decode step (HBM-bound, one CTA per (sequence, head)).
 cudaError_t launch_decode_step(const DecodeArgs &a, cudaStream_t stream);
 

@@ -167,3 +167,8 @@ def test_noalloc_rejects_calls_beyond_its_scratch_limit():
     assert B._lib.kda_prefill_noalloc(*args) == WORKSPACE
     args = [_fake()] * 6 + [_fake(), None, 1, 64, 1, 64, 64, BF16, None, None, _fake(), None]
     assert B._lib.kda_prefill_noalloc(*args) == UNSUPPORTED
+
+
+def test_selftest_rejects_out_of_range_limits():
+    assert B._lib.kda_selftest_wait_timeout(0, None) == INVALID
+    assert B._lib.kda_selftest_wait_timeout(20_000_000_000, None) == INVALID
