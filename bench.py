@@ -312,8 +312,36 @@ def main():
             "roofline_ms": th * BYTES_PER_TOKEN_HEAD / hbm_peak / 1e6}
     launches = args.steps * nk
 
-    decode = e2e = cpu = None
+    decode = e2e = cpu = ckpt = None
     if not args.prefill_only:
+        # Prefix-cache checkpoints every 512 tokens (the pages' hash block) on the same
+        # workload: the cost of writing 64 KiB per (checkpoint, head) from the state pass.
+        every = 512
+        n_ck = K.kda_checkpoint_count(inp["cu_seqlens_host"], every)
+        ckbuf = torch.empty(max(n_ck, 1), H, dk, dv, dtype=torch.float32, device=dev)
+
+        def cstep():
+            K.kda_prefill_checkpointed(inp["q"], inp["k"], inp["v"], inp["z"], inp["A"], inp["beta"],
+                                       inp["cu_seqlens"], inp["cu_seqlens_host"], every,
+                                       final_state=S, o=o, checkpoints=ckbuf, workspace=ws,
+                                       algo=args.algo, stream=stream)
+
+        for _ in range(args.warmup):
+            cstep()
+        torch.cuda.synchronize()
+        barrier()
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(args.steps):
+            cstep()
+        c1.record(stream)
+        torch.cuda.synchronize()
+        cms = max_over_ranks(c0.elapsed_time(c1), world, dev) / args.steps
+        ckpt = {"every": every, "checkpoints_per_step": n_ck * H, "ms_per_step": cms,
+                "overhead_vs_plain": cms / ms_per_step - 1.0,
+                "extra_bytes_per_step": n_ck * H * dk * dv * 4}
+        del ckbuf
+
         # Decode step: B=256 cached states, H=96, updated in place; GB/s of state traffic.
         dcfg = CONFIGS["decode_256"]
         d = decode_inputs(dcfg.B, dcfg.H, dcfg.dk, dcfg.dv, dcfg.dtype, seed=rank_seed(dcfg.seed, rank),
@@ -394,6 +422,7 @@ def main():
             "roofline": roofline,
             "path_roofline": path,
             "decode": decode,
+            "checkpoints": ckpt,
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clocks,

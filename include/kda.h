@@ -135,6 +135,41 @@ kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const voi
                           void *const *stage_events, int32_t num_stage_events);
 
 /*
+ * kda_prefill_ex that also writes state checkpoints for prefix caching ("Kimi
+ * K3 Under the Hood", section "Serving two incompatible cache types": prefix
+ * hashes every 512 tokens, KDA states kept only at selected boundaries, a hit
+ * copies the cached state into the running state and resumes prefill).
+ *
+ *   checkpoint_every  0 = none (checkpoints may be NULL), else a positive
+ *                     multiple of 64: checkpoint j (j = 1 .. L_n / every) of
+ *                     sequence n is the state after its first j * every tokens.
+ *   checkpoints       device fp32 [kda_checkpoint_count(...), H, dk, dv]; row
+ *                     (sum_{m<n} L_m / every) + j - 1 holds checkpoint j of
+ *                     sequence n (a checkpoint at a sequence's last token equals
+ *                     its final state).  16-byte aligned, caller-owned.
+ * Other arguments, results and errors as kda_prefill_ex; a bad checkpoint_every
+ * or a NULL checkpoints with checkpoint_every > 0 is KDA_ERR_INVALID_ARG.
+ */
+kda_status kda_prefill_checkpointed(const void *q, const void *k, const void *v, const void *z,
+                                    const float *A, const float *beta,
+                                    const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                                    int32_t num_seqs, int32_t total_tokens, int32_t H, int32_t dk,
+                                    int32_t dv, kda_dtype dt, const float *initial_state,
+                                    float *final_state, void *o, void *workspace,
+                                    size_t workspace_bytes, kda_algo algo, void *stream,
+                                    void *const *stage_events, int32_t num_stage_events,
+                                    int32_t checkpoint_every, float *checkpoints);
+
+/*
+ * Rows of the checkpoint tensor for these HOST offsets: sum over sequences of
+ * L_n / checkpoint_every.  Returns -1 for invalid arguments (NULL offsets with
+ * num_seqs > 0, checkpoint_every not a positive multiple of 64, decreasing
+ * offsets).
+ */
+int64_t kda_checkpoint_count(const int32_t *cu_seqlens_host, int32_t num_seqs,
+                             int32_t checkpoint_every);
+
+/*
  * Number of kernels one kda_prefill_ex call launches for these sizes and
  * algorithm (for a non-empty batch); 0 for invalid arguments.
  */

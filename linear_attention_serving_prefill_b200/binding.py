@@ -31,6 +31,9 @@ SIGNATURES = {
     "kda_prefill": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _P], _I32),
     "kda_prefill_ex": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _I32, _P, _P, _I32], _I32),
     "kda_prefill_kernel_count": ([_I32, _I32, _I32, _I32], _I32),
+    "kda_prefill_checkpointed": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _I32, _P, _P, _I32, _I32, _P],
+                                 _I32),
+    "kda_checkpoint_count": ([_P, _I32, _I32], ctypes.c_int64),
     "kda_prefill_noalloc": ([_P] * 8 + [_I32] * 6 + [_P] * 4, _I32),
     "kda_decode_step": ([_P] * 6 + [_I32] * 5 + [_P, _I32, _P, _P, _P], _I32),
     "kda_device_status": ([_P, _P], _I32),
@@ -138,6 +141,48 @@ def kda_prefill(q, k, v, z, A, beta, cu_seqlens, cu_seqlens_host=None, initial_s
         _dev(workspace, "workspace"), ws_bytes, KDA_ALGO[algo], _stream_ptr(stream), ev_arr, n_ev)
     _check(code, "kda_prefill")
     return o, final_state
+
+
+def kda_checkpoint_count(cu_seqlens_host, checkpoint_every: int) -> int:
+    """Rows of the checkpoint tensor: sum over sequences of L_n // checkpoint_every."""
+    ch = cu_seqlens_host.to(torch.int32).contiguous()
+    n = _lib.kda_checkpoint_count(ctypes.c_void_p(ch.data_ptr()), ch.numel() - 1, checkpoint_every)
+    if n < 0:
+        raise KdaError(1, "kda_checkpoint_count")
+    return int(n)
+
+
+def kda_prefill_checkpointed(q, k, v, z, A, beta, cu_seqlens, cu_seqlens_host, checkpoint_every,
+                             initial_state=None, final_state=None, o=None, checkpoints=None,
+                             workspace=None, algo: str = "auto", stream=None):
+    """kda_prefill plus the state after every ``checkpoint_every`` tokens of each
+    sequence; returns ``(o, final_state, checkpoints [count, H, dk, dv])``."""
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = cu_seqlens.shape[0] - 1
+    dt = q.dtype
+    if o is None:
+        o = torch.empty(T, H, dv, dtype=dt, device=q.device)
+    if final_state is None:
+        final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+    count = kda_checkpoint_count(cu_seqlens_host, checkpoint_every)
+    if checkpoints is None:
+        checkpoints = torch.empty(max(count, 1), H, dk, dv, dtype=torch.float32, device=q.device)
+    need = kda_prefill_workspace_size(T, N, H, dk, dv, dt, algo)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ch = cu_seqlens_host.to(torch.int32).contiguous()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    code = _lib.kda_prefill_checkpointed(
+        _dev(q, "q", dt), _dev(k, "k", dt), _dev(v, "v", dt), _dev(z, "z", dt),
+        _dev(A, "A", torch.float32), _dev(beta, "beta", torch.float32),
+        _dev(cu_seqlens, "cu_seqlens", torch.int32), ctypes.c_void_p(ch.data_ptr()), N, T, H, dk,
+        dv, KDA_DTYPE[dt], _dev(initial_state, "initial_state", torch.float32),
+        _dev(final_state, "final_state", torch.float32), _dev(o, "o", dt),
+        _dev(workspace, "workspace"), ws_bytes, KDA_ALGO[algo], _stream_ptr(stream), None, 0,
+        int(checkpoint_every), _dev(checkpoints, "checkpoints", torch.float32))
+    _check(code, "kda_prefill_checkpointed")
+    return o, final_state, checkpoints[:count]
 
 
 def kda_prefill_noalloc(q, k, v, z, A, beta, cu_seqlens, cu_seqlens_host=None,

@@ -85,18 +85,32 @@ extern "C" size_t kda_prefill_workspace_size(int32_t total_tokens, int32_t num_s
     return 0;  // the CUDA-core path keeps everything on chip
 }
 
-extern "C" kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const void *z,
-                                     const float *A, const float *beta,
-                                     const int32_t *cu_seqlens_dev,
-                                     const int32_t *cu_seqlens_host, int32_t num_seqs,
-                                     int32_t total_tokens, int32_t H, int32_t dk, int32_t dv,
-                                     kda_dtype dt, const float *initial_state,
-                                     float *final_state, void *o, void *workspace,
-                                     size_t workspace_bytes, kda_algo algo, void *stream,
-                                     void *const *stage_events, int32_t num_stage_events)
+extern "C" int64_t kda_checkpoint_count(const int32_t *cu_seqlens_host, int32_t num_seqs,
+                                        int32_t checkpoint_every)
+{
+    if (num_seqs < 0 || checkpoint_every <= 0 || checkpoint_every % 64 != 0) return -1;
+    if (num_seqs > 0 && !cu_seqlens_host) return -1;
+    int64_t total = 0;
+    for (int32_t i = 0; i < num_seqs; ++i) {
+        const int32_t L = cu_seqlens_host[i + 1] - cu_seqlens_host[i];
+        if (L < 0) return -1;
+        total += L / checkpoint_every;
+    }
+    return total;
+}
+
+extern "C" kda_status kda_prefill_checkpointed(
+    const void *q, const void *k, const void *v, const void *z, const float *A, const float *beta,
+    const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host, int32_t num_seqs,
+    int32_t total_tokens, int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+    const float *initial_state, float *final_state, void *o, void *workspace,
+    size_t workspace_bytes, kda_algo algo, void *stream, void *const *stage_events,
+    int32_t num_stage_events, int32_t checkpoint_every, float *checkpoints)
 {
     kda_status st = check_prefill_sizes(total_tokens, num_seqs, H, dk, dv, dt, algo);
     if (st != KDA_OK) return st;
+    if (checkpoint_every < 0 || checkpoint_every % 64 != 0) return KDA_ERR_INVALID_ARG;
+    if (checkpoint_every > 0 && (!checkpoints || !aligned(checkpoints, 16))) return KDA_ERR_INVALID_ARG;
     if (num_seqs > 0 && !cu_seqlens_dev) return KDA_ERR_INVALID_ARG;
     if (total_tokens > 0 && (!q || !k || !v || !z || !A || !beta || !o)) return KDA_ERR_INVALID_ARG;
     for (const void *p : {q, k, v, z, (const void *)o, (const void *)initial_state,
@@ -126,11 +140,28 @@ extern "C" kda_status kda_prefill_ex(const void *q, const void *k, const void *v
     a.initial_state = initial_state; a.final_state = final_state; a.o = o;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.status = status;
     a.events = stage_events; a.num_events = stage_events ? num_stage_events : 0;
+    a.ckpt_every = checkpoint_every; a.checkpoints = checkpoint_every > 0 ? checkpoints : nullptr;
 
     cudaError_t err = use_tensor_core(dk, dv, dt, algo)
                           ? kda::launch_prefill_tensor_core(a, (cudaStream_t)stream)
                           : kda::launch_prefill_cuda_core(a, (cudaStream_t)stream);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+extern "C" kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const void *z,
+                                     const float *A, const float *beta,
+                                     const int32_t *cu_seqlens_dev,
+                                     const int32_t *cu_seqlens_host, int32_t num_seqs,
+                                     int32_t total_tokens, int32_t H, int32_t dk, int32_t dv,
+                                     kda_dtype dt, const float *initial_state,
+                                     float *final_state, void *o, void *workspace,
+                                     size_t workspace_bytes, kda_algo algo, void *stream,
+                                     void *const *stage_events, int32_t num_stage_events)
+{
+    return kda_prefill_checkpointed(q, k, v, z, A, beta, cu_seqlens_dev, cu_seqlens_host,
+                                    num_seqs, total_tokens, H, dk, dv, dt, initial_state,
+                                    final_state, o, workspace, workspace_bytes, algo, stream,
+                                    stage_events, num_stage_events, 0, nullptr);
 }
 
 extern "C" kda_status kda_prefill(const void *q, const void *k, const void *v, const void *z,

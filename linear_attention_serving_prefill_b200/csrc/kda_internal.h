@@ -21,6 +21,8 @@ struct PrefillArgs {
     void *workspace;
     size_t workspace_bytes;
     int32_t *status;                // device status word
+    int32_t ckpt_every;             // 0 = no checkpoints, else a multiple of 64
+    float *checkpoints;             // [count, H, dk, dv] or nullptr
     void *const *events;            // optional cudaEvent_t per kernel boundary
     int32_t num_events;
     // Records boundary i (0 = before the first kernel) when the caller asked for it.

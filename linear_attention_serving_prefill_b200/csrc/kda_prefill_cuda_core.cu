@@ -42,7 +42,8 @@ prefill_cuda_core_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                          const TIn *__restrict__ v, const TIn *__restrict__ z,
                          const float *__restrict__ A, const float *__restrict__ beta,
                          const int32_t *__restrict__ cu_seqlens, int H, int dv,
-                         const float *S0, float *Sf, TIn *__restrict__ o)
+                         const float *S0, float *Sf, TIn *__restrict__ o, int ckpt_every,
+                         float *__restrict__ ckpts)
 {
     constexpr int LD = CudaCoreSmem<DK>::LD;
     extern __shared__ float sm[];
@@ -68,6 +69,14 @@ prefill_cuda_core_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     const int tid = threadIdx.x;
     const int t_begin = cu_seqlens[n], t_end = cu_seqlens[n + 1];
     const size_t state_base = ((size_t)n * H + h) * DK * dv + j0;
+    // Row of this sequence's first checkpoint: sum over earlier sequences of L / every.
+    __shared__ long long sCkBase;
+    if (tid == 0) {
+        long long b = 0;
+        if (ckpt_every > 0)
+            for (int m = 0; m < n; ++m) b += (cu_seqlens[m + 1] - cu_seqlens[m]) / ckpt_every;
+        sCkBase = b;
+    }
 
     for (int c = tid; c < DK; c += kThreads) sEA[c] = expf(A[(size_t)h * DK + c]);
     for (int e = tid; e < DK * kDVS; e += kThreads) {
@@ -188,6 +197,15 @@ prefill_cuda_core_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
             }
         }
         __syncthreads();
+        // Checkpoint: the state after the first `pos` tokens, when pos is a multiple of every.
+        const int pos = tc + len - t_begin;
+        if (ckpt_every > 0 && pos % ckpt_every == 0) {
+            const size_t row = (size_t)(sCkBase + pos / ckpt_every - 1);
+            for (int e = tid; e < DK * kDVS; e += kThreads) {
+                const int c = e / kDVS, j = e % kDVS;
+                ckpts[(row * H + h) * DK * dv + (size_t)c * dv + j0 + j] = sS[e];
+            }
+        }
     }
 
     if (Sf) {
@@ -211,7 +229,8 @@ cudaError_t launch_typed(const PrefillArgs &a, cudaStream_t stream)
     a.mark(0, stream);
     kern<<<(unsigned)blocks, kThreads, smem, stream>>>(
         (const TIn *)a.q, (const TIn *)a.k, (const TIn *)a.v, (const TIn *)a.z, a.A, a.beta,
-        a.cu_seqlens, a.H, a.dv, a.initial_state, a.final_state, (TIn *)a.o);
+        a.cu_seqlens, a.H, a.dv, a.initial_state, a.final_state, (TIn *)a.o, a.ckpt_every,
+        a.checkpoints);
     a.mark(1, stream);
     return cudaGetLastError();
 }

@@ -71,35 +71,49 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // ------------------------------------------------------------------- plan --
 
 // chunk_off[n] = sum_{m<n} ceil(L_m / 64); chunk_off[N] = total chunks.
+// ckpt_off[n] = sum_{m<n} L_m / every (checkpoint rows), when every > 0.
 // order[i] = sequence index with the i-th largest length (ties by index)
 // when N <= kMaxSorted, else the identity.
 constexpr int kPlanThreads = 1024;
 constexpr int kMaxSorted = 4096;
 
 __global__ void __launch_bounds__(kPlanThreads)
-plan_kernel(const int32_t *__restrict__ cu, int N, int32_t *__restrict__ chunk_off,
-            int32_t *__restrict__ order)
+plan_kernel(const int32_t *__restrict__ cu, int N, int every, int32_t *__restrict__ chunk_off,
+            int32_t *__restrict__ ckpt_off, int32_t *__restrict__ order)
 {
-    __shared__ int32_t part[kPlanThreads];
+    __shared__ int32_t part[2][kPlanThreads];
     const int tid = threadIdx.x;
     const int per = (N + kPlanThreads - 1) / kPlanThreads;
     const int lo = min(N, tid * per), hi = min(N, lo + per);
-    int32_t acc = 0;
-    for (int n = lo; n < hi; ++n) acc += (cu[n + 1] - cu[n] + kChunk - 1) / kChunk;
-    part[tid] = acc;
+    int32_t acc = 0, acck = 0;
+    for (int n = lo; n < hi; ++n) {
+        const int32_t L = cu[n + 1] - cu[n];
+        acc += (L + kChunk - 1) / kChunk;
+        acck += every > 0 ? L / every : 0;
+    }
+    part[0][tid] = acc;
+    part[1][tid] = acck;
     __syncthreads();
     for (int off = 1; off < kPlanThreads; off <<= 1) {
-        const int32_t v = tid >= off ? part[tid - off] : 0;
+        const int32_t v0 = tid >= off ? part[0][tid - off] : 0;
+        const int32_t v1 = tid >= off ? part[1][tid - off] : 0;
         __syncthreads();
-        part[tid] += v;
+        part[0][tid] += v0;
+        part[1][tid] += v1;
         __syncthreads();
     }
-    int32_t run = part[tid] - acc;  // exclusive prefix
+    int32_t run = part[0][tid] - acc, runk = part[1][tid] - acck;  // exclusive prefixes
     for (int n = lo; n < hi; ++n) {
+        const int32_t L = cu[n + 1] - cu[n];
         chunk_off[n] = run;
-        run += (cu[n + 1] - cu[n] + kChunk - 1) / kChunk;
+        ckpt_off[n] = runk;
+        run += (L + kChunk - 1) / kChunk;
+        runk += every > 0 ? L / every : 0;
     }
-    if (tid == kPlanThreads - 1) chunk_off[N] = part[tid];
+    if (tid == kPlanThreads - 1) {
+        chunk_off[N] = part[0][tid];
+        ckpt_off[N] = part[1][tid];
+    }
     for (int n = tid; n < N; n += kPlanThreads) {
         int rank = n;
         if (N <= kMaxSorted) {
@@ -562,7 +576,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_off,
              const int32_t *__restrict__ order, int N, int H,
              const uint8_t *__restrict__ blocks, int64_t max_chunks,
-             const float *S0, float *Sf, __nv_bfloat16 *__restrict__ o, int32_t *status)
+             const float *S0, float *Sf, __nv_bfloat16 *__restrict__ o, int32_t *status,
+             int ckpt_every, const int32_t *__restrict__ ckpt_off, float *__restrict__ ckpts)
 {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
@@ -727,11 +742,21 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
                 }
                 dec = (const float *)(sm + s1 * kStageBytes + kOffDecay);
             }
+            // Checkpoint when the state after `pos` tokens falls on a multiple of every.
+            const int pos = min((c + 1) * kChunk, tend - tbeg);
+            float *ck = nullptr;
+            if (ckpt_every > 0 && pos % ckpt_every == 0)
+                ck = ckpts + ((size_t)(ckpt_off[n] + pos / ckpt_every - 1) * H + h) * kDK * kDV;
             // S_out -> bf16 copy for the next chunk, and pre-decayed fp32 state.
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
                 tmem_ld32(tmem_addr(tb, lq, kTS + 32 * q4), r32);
                 tmem_ld_wait();
+                if (ck) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        ck[(size_t)(32 * q4 + i) * kDV + j] = __uint_as_float(r32[i]);
+                }
                 if (last) {
                     if (Sf) {
 #pragma unroll
@@ -826,7 +851,7 @@ size_t tc_workspace_bytes(int32_t total_tokens, int32_t num_seqs, int32_t H)
 {
     if (num_seqs <= 0) return 0;
     const int64_t max_chunks = ((int64_t)total_tokens + 63LL * num_seqs) / kChunk;
-    const size_t plan = (((size_t)(2 * num_seqs + 2) * sizeof(int32_t)) + 1023) & ~(size_t)1023;
+    const size_t plan = (((size_t)(3 * num_seqs + 3) * sizeof(int32_t)) + 1023) & ~(size_t)1023;
     return plan + (size_t)H * max_chunks * kBlockBytes;
 }
 
@@ -835,8 +860,9 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
     if (a.dk != kDK || a.dv != kDV || !a.bf16) return cudaErrorInvalidValue;
     const int64_t max_chunks = ((int64_t)a.total_tokens + 63LL * a.num_seqs) / kChunk;
     int32_t *chunk_off = (int32_t *)a.workspace;
-    int32_t *order = chunk_off + a.num_seqs + 1;
-    const size_t plan = (((size_t)(2 * a.num_seqs + 2) * sizeof(int32_t)) + 1023) & ~(size_t)1023;
+    int32_t *ckpt_off = chunk_off + a.num_seqs + 1;
+    int32_t *order = ckpt_off + a.num_seqs + 1;
+    const size_t plan = (((size_t)(3 * a.num_seqs + 3) * sizeof(int32_t)) + 1023) & ~(size_t)1023;
     uint8_t *blocks = (uint8_t *)a.workspace + plan;
     cudaError_t err;
 
@@ -848,7 +874,8 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
     if (err != cudaSuccess) return err;
 
     a.mark(0, stream);
-    plan_kernel<<<1, kPlanThreads, 0, stream>>>(a.cu_seqlens, a.num_seqs, chunk_off, order);
+    plan_kernel<<<1, kPlanThreads, 0, stream>>>(a.cu_seqlens, a.num_seqs, a.ckpt_every, chunk_off,
+                                                ckpt_off, order);
     a.mark(1, stream);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
@@ -872,7 +899,7 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
     a.mark(2, stream);
     state_kernel<<<(unsigned)(a.num_seqs * a.H), kStateThreads, kStateSmem, stream>>>(
         a.cu_seqlens, chunk_off, order, a.num_seqs, a.H, blocks, max_chunks, a.initial_state,
-        a.final_state, (__nv_bfloat16 *)a.o, a.status);
+        a.final_state, (__nv_bfloat16 *)a.o, a.status, a.ckpt_every, ckpt_off, a.checkpoints);
     a.mark(3, stream);
     return cudaGetLastError();
 }

@@ -101,6 +101,13 @@ void kda_oracle_gate(const double *z, const double *A, int64_t T, int H, int dk,
                             g + ((size_t)t * H + h) * dk);
 }
 
+int kda_oracle_prefill_ckpt(const double *q, const double *k, const double *v,
+                            const double *z, const double *A, const double *beta,
+                            const int32_t *cu_seqlens, int num_seqs, int H, int dk,
+                            int dv, const double *initial_state, double *o,
+                            double *final_state, int every, double *checkpoints,
+                            int nthreads);
+
 /*
  * Prefill over packed variable-length sequences: for every sequence n and head
  * h, start from initial_state[n,h] (zeros when initial_state is NULL), run the
@@ -114,6 +121,25 @@ int kda_oracle_prefill(const double *q, const double *k, const double *v,
                        const int32_t *cu_seqlens, int num_seqs, int H, int dk,
                        int dv, const double *initial_state, double *o,
                        double *final_state, int nthreads)
+{
+    return kda_oracle_prefill_ckpt(q, k, v, z, A, beta, cu_seqlens, num_seqs, H, dk, dv,
+                                   initial_state, o, final_state, 0, NULL, nthreads);
+}
+
+/*
+ * Prefill that also records state checkpoints for prefix caching ("Kimi K3
+ * Under the Hood", section "Serving two incompatible cache types": KDA states
+ * are kept at selected prefix-hash boundaries).  With every > 0, checkpoint j
+ * (j = 1 .. L_n / every) of sequence n is the state after its first j * every
+ * tokens, stored at row (sum_{m<n} L_m / every) + j - 1 of checkpoints
+ * [count, H, dk, dv].
+ */
+int kda_oracle_prefill_ckpt(const double *q, const double *k, const double *v,
+                            const double *z, const double *A, const double *beta,
+                            const int32_t *cu_seqlens, int num_seqs, int H, int dk,
+                            int dv, const double *initial_state, double *o,
+                            double *final_state, int every, double *checkpoints,
+                            int nthreads)
 {
     int failed = 0;
 #ifdef _OPENMP
@@ -139,11 +165,21 @@ int kda_oracle_prefill(const double *q, const double *k, const double *v,
                     memcpy(S, initial_state + sidx, sizeof(double) * (size_t)dk * dv);
                 else
                     memset(S, 0, sizeof(double) * (size_t)dk * dv);
+                int64_t ck_base = 0;
+                if (every > 0)
+                    for (int m = 0; m < n; ++m)
+                        ck_base += (cu_seqlens[m + 1] - cu_seqlens[m]) / every;
                 for (int64_t t = cu_seqlens[n]; t < cu_seqlens[n + 1]; ++t) {
                     const size_t th = (size_t)t * H + h;
                     oracle_gate_row(z + th * dk, A + (size_t)h * dk, dk, g);
                     oracle_token_step(S, q + th * dk, k + th * dk, v + th * dv, g,
                                       beta[th], dk, dv, vhat, o + th * dv);
+                    const int64_t done = t + 1 - cu_seqlens[n];
+                    if (every > 0 && checkpoints && done % every == 0) {
+                        const size_t row = (size_t)(ck_base + done / every - 1);
+                        memcpy(checkpoints + (row * H + h) * (size_t)dk * dv, S,
+                               sizeof(double) * (size_t)dk * dv);
+                    }
                 }
                 if (final_state)
                     memcpy(final_state + sidx, S, sizeof(double) * (size_t)dk * dv);

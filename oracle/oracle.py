@@ -53,6 +53,9 @@ def _load():
         lib.kda_oracle_prefill.argtypes = [d, d, d, d, d, d, d, i32, i32, i32, i32,
                                            d, d, d, i32]
         lib.kda_oracle_prefill.restype = i32
+        lib.kda_oracle_prefill_ckpt.argtypes = [d, d, d, d, d, d, d, i32, i32, i32, i32,
+                                                d, d, d, i32, d, i32]
+        lib.kda_oracle_prefill_ckpt.restype = i32
         lib.kda_oracle_decode.argtypes = [d, d, d, d, d, d, i32, i32, i32, i32, d,
                                           d, d, i32]
         lib.kda_oracle_decode.restype = i32
@@ -117,6 +120,39 @@ def prefill(q, k, v, z, A, beta, cu_seqlens, initial_state=None, nthreads: int =
     if rc != 0:
         raise MemoryError("kda oracle: allocation failed")
     return o, sf
+
+
+def checkpoint_count(cu_seqlens, every: int) -> int:
+    """sum over sequences of L_n // every (0 when every <= 0)."""
+    cu = _i32(cu_seqlens)
+    if every <= 0:
+        return 0
+    return int(sum((int(cu[i + 1]) - int(cu[i])) // every for i in range(len(cu) - 1)))
+
+
+def prefill_checkpoints(q, k, v, z, A, beta, cu_seqlens, every: int, initial_state=None,
+                        nthreads: int = 0):
+    """As ``prefill``, plus the state after every ``every`` tokens of each sequence.
+
+    Returns ``(o, final_state, checkpoints [count, H, dk, dv])``; checkpoint j of
+    sequence n (j = 1 .. L_n // every) is at row sum_{m<n} L_m // every + j - 1.
+    """
+    q, k, v, z, A, beta = (_f64(t) for t in (q, k, v, z, A, beta))
+    cu = _i32(cu_seqlens)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    n = cu.shape[0] - 1
+    s0 = None if initial_state is None else _f64(initial_state)
+    o = np.zeros((T, H, dv), dtype=np.float64)
+    sf = np.zeros((n, H, dk, dv), dtype=np.float64)
+    ck = np.zeros((checkpoint_count(cu, every), H, dk, dv), dtype=np.float64)
+    rc = _load().kda_oracle_prefill_ckpt(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(A),
+                                         _ptr(beta), _ptr(cu), n, H, dk, dv, _ptr(s0),
+                                         _ptr(o), _ptr(sf), int(every),
+                                         _ptr(ck) if ck.size else None, nthreads)
+    if rc != 0:
+        raise MemoryError("kda oracle: allocation failed")
+    return o, sf, ck
 
 
 def decode_step(q, k, v, z, A, beta, state, slots=None, nthreads: int = 0):

@@ -172,3 +172,18 @@ def test_noalloc_rejects_calls_beyond_its_scratch_limit():
 def test_selftest_rejects_out_of_range_limits():
     assert B._lib.kda_selftest_wait_timeout(0, None) == INVALID
     assert B._lib.kda_selftest_wait_timeout(20_000_000_000, None) == INVALID
+
+
+def test_checkpoint_count_and_validation():
+    p, keep = _host_cu([0, 130, 130, 700])
+    assert B._lib.kda_checkpoint_count(p, 3, 64) == 2 + 0 + 8
+    assert B._lib.kda_checkpoint_count(p, 3, 128) == 1 + 0 + 4
+    assert B._lib.kda_checkpoint_count(p, 3, 100) == -1      # not a multiple of 64
+    assert B._lib.kda_checkpoint_count(None, 3, 64) == -1
+    args = dict(q=_fake(), k=_fake(), v=_fake(), z=_fake(), A=_fake(), beta=_fake())
+    common = [args[k] for k in ("q", "k", "v", "z", "A", "beta")] + [_fake(), None, 2, 10, 4, 64, 64,
+                                                                      BF16, None, None, _fake(), None,
+                                                                      0, AUTO, None, None, 0]
+    assert B._lib.kda_prefill_checkpointed(*common, 96, _fake()) == INVALID   # not a multiple of 64
+    assert B._lib.kda_prefill_checkpointed(*common, 64, None) == INVALID      # no buffer
+    assert B._lib.kda_prefill_checkpointed(*common, 64, _fake(0x10008)) == INVALID  # misaligned

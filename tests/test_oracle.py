@@ -350,3 +350,28 @@ def test_oracle_regression_fixture():
     o, sf = oracle.prefill(**arr, cu_seqlens=np.array(d["cu_seqlens"], np.int32))
     np.testing.assert_allclose(o, np.array(d["o"]), rtol=1e-13, atol=1e-15)
     np.testing.assert_allclose(sf, np.array(d["final_state"]), rtol=1e-13, atol=1e-15)
+
+
+def test_checkpoints_are_prefix_final_states():
+    """A checkpoint is, by definition, the final state of the sequence's prefix
+    of that length; the oracle's checkpoint output is checked against separate
+    prefix runs (and the plain prefill is unchanged by asking for checkpoints)."""
+    lengths = [130, 0, 64, 200, 63]
+    x = _inputs(lengths, H=2, dk=4, dv=3, seed=40)
+    for every in (16, 64, 100):
+        o, sf, ck = oracle.prefill_checkpoints(**x, every=every)
+        o2, sf2 = oracle.prefill(**x)
+        np.testing.assert_array_equal(o, o2)
+        np.testing.assert_array_equal(sf, sf2)
+        assert ck.shape[0] == sum(L // every for L in lengths)
+        row = 0
+        cu = x["cu_seqlens"]
+        for i, L in enumerate(lengths):
+            for j in range(1, L // every + 1):
+                sl = slice(cu[i], cu[i] + j * every)
+                _, s_pref = oracle.prefill(**{kk: x[kk][sl] for kk in ("q", "k", "v", "z", "beta")},
+                                          A=x["A"], cu_seqlens=np.array([0, j * every], np.int32),
+                                          initial_state=x["initial_state"][i:i + 1])
+                np.testing.assert_array_equal(ck[row], s_pref[0])
+                row += 1
+        assert row == ck.shape[0]

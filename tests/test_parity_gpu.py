@@ -245,3 +245,47 @@ def test_prefill_then_decode_equals_longer_prefill(algo):
     torch.cuda.synchronize()
     assert relerr(to_np(o[0]), to_np(o_full[L])) <= TOL_BF16
     assert relerr(to_np(S), to_np(S_full)) <= TOL_BF16
+
+
+# ------------------------------------------------------------- checkpoints ----
+
+@pytest.mark.parametrize("algo,dtype,tol", [("cuda_core", "f32", TOL_F32), ("cuda_core", "bf16", TOL_BF16),
+                                            ("tensor_core", "bf16", TOL_BF16)])
+@pytest.mark.parametrize("every", [64, 128, 512])
+def test_checkpoints_match_oracle(algo, dtype, tol, every):
+    """State checkpoints every `every` tokens (prefix-cache boundaries) equal the
+    oracle's, and asking for them leaves o and the final states unchanged."""
+    lengths = [700, 64, 129, 0, 1030, 511]
+    x = _cuda(prefill_inputs(lengths, 2, 128, 128, dtype, seed=50 + every, s0_std=0.02))
+    o, S, ck = K.kda_prefill_checkpointed(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"],
+                                          x["cu_seqlens"], x["cu_seqlens_host"], every,
+                                          initial_state=x["initial_state"], algo=algo)
+    o2, S2 = _run(x, algo)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(S, S2)
+    ref_o, ref_S, ref_ck = oracle.prefill_checkpoints(
+        x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"], x["cu_seqlens_host"], every,
+        x["initial_state"])
+    assert ck.shape[0] == sum(L // every for L in lengths) == ref_ck.shape[0]
+    assert relerr(to_np(ck), ref_ck) <= tol
+    assert relerr(to_np(S), ref_S) <= tol
+
+
+def test_checkpoints_full_size_varlen_sampled_heads():
+    """The 16-sequence varlen workload with checkpoints every 512 tokens (the
+    pages' prefix-hash block); two heads of every checkpoint row against the oracle."""
+    cfg = CONFIGS["varlen_resume"]
+    x = config_inputs(cfg, device="cuda")
+    o, S, ck = K.kda_prefill_checkpointed(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"],
+                                          x["cu_seqlens"], x["cu_seqlens_host"], 512,
+                                          initial_state=x["initial_state"])
+    torch.cuda.synchronize()
+    heads = [0, 77]
+    hs = torch.tensor(heads, device="cuda")
+    sub = {key: x[key].index_select(1, hs).cpu() for key in ("q", "k", "v", "z", "beta")}
+    _, ref_S, ref_ck = oracle.prefill_checkpoints(sub["q"], sub["k"], sub["v"], sub["z"],
+                                                  x["A"].index_select(0, hs).cpu(), sub["beta"],
+                                                  x["cu_seqlens_host"], 512,
+                                                  x["initial_state"].index_select(1, hs).cpu())
+    assert relerr(to_np(ck.index_select(1, hs)), ref_ck) <= TOL_BF16
+    assert relerr(to_np(S.index_select(1, hs)), ref_S) <= TOL_BF16
