@@ -18,7 +18,8 @@
 //              on the tensor cores.  Writes per (chunk, head) a block of
 //              MMA-ready tiles: [W; Q e^{G}], (K e^{G_C - G})^T, P, U, e^{G_C}.
 //   3. state:  one persistent CTA per (sequence, head), walking its chunks in
-//              order with the fp32 state transposed in tensor memory:
+//              order with the fp32 state transposed in tensor memory (two
+//              epilogue warpgroups split every pass by rows / key channels):
 //                D    = S^T [W; Qt]^T              (S^T as a TMEM operand)
 //                Dl^T = U^T - D[:, :64]            -> bf16 into TMEM
 //                S^T  = S^T Diag(e^{G_C}) + Dl^T Kd   (Kd = K e^{G_C - G})
@@ -559,18 +560,20 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
 
 // ------------------------------------------------------------------ state --
 
-constexpr int kStateThreads = 320;       // WG0: warps 0-3, WG1: warps 4-7, load: 8, mma: 9
+constexpr int kStateThreads = 320;       // epilogue: warps 0-7, load: 8, mma: 9
 constexpr uint32_t kStageBytes = 75776;  // block rounded up to 1 KiB
 constexpr int kStages = 2;
-constexpr uint32_t kStateSmem = kStages * kStageBytes + 1024;
+constexpr uint32_t kOStage = kStages * kStageBytes;  // 2 x [64][128] bf16 output staging
+constexpr uint32_t kStateSmem = kStages * kStageBytes + 2 * 16384 + 1024;
 // TMEM columns
 constexpr uint32_t kTS = 0, kTSbf = 128, kTDl = 192, kTD1 = 256;  // D1 double buffer: 256, 384
 
 struct StateBars {
     uint64_t full[kStages], empty[kStages];
-    uint64_t mma1, dl_ready, sbf_ready;
-    uint64_t mma2[2], d1_free[2];
+    uint64_t mma1, dl_ready, sbf_ready, sdec_ready;
+    uint64_t mma2[2], d1_free[2], ostaged[2];
 };
+constexpr uint32_t kEpi = 256;  // epilogue threads: two warpgroups
 
 __global__ void __launch_bounds__(kStateThreads, 1)
 state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_off,
@@ -597,11 +600,16 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
         return;
     }
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) { mbar_init(&bars.full[s], 1); mbar_init(&bars.empty[s], 129); }
+        for (int s = 0; s < kStages; ++s) { mbar_init(&bars.full[s], 1); mbar_init(&bars.empty[s], kEpi + 1); }
         mbar_init(&bars.mma1, 1);
-        mbar_init(&bars.dl_ready, 128);
-        mbar_init(&bars.sbf_ready, 128);
-        for (int b = 0; b < 2; ++b) { mbar_init(&bars.mma2[b], 1); mbar_init(&bars.d1_free[b], 128); }
+        mbar_init(&bars.dl_ready, kEpi);
+        mbar_init(&bars.sbf_ready, kEpi);
+        mbar_init(&bars.sdec_ready, kEpi);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars.mma2[b], 1);
+            mbar_init(&bars.d1_free[b], kEpi);
+            mbar_init(&bars.ostaged[b], kEpi);
+        }
         fence_mbar_init();
         sAbort = 0;
     }
@@ -651,7 +659,8 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
                            desc_kmajor_sw128(st + kOffWQ + (ks >> 2) * 128 * 128 + (ks & 3) * 32),
                            id128, ks > 0);
                 mma_commit(&bars.mma1);
-                if (!mbar_wait(&bars.dl_ready, c & 1, globaltimer_ns() + kWaitNs)) {
+                if (!mbar_wait(&bars.dl_ready, c & 1, globaltimer_ns() + kWaitNs) ||
+                    !mbar_wait(&bars.sdec_ready, c & 1, globaltimer_ns() + kWaitNs)) {
                     record_timeout(status); sAbort = 1; break;
                 }
                 tc_fence_after_sync();
@@ -670,12 +679,14 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
             // Drain: wait for the last committed MMAs before exit.
             if (c > 0) mbar_wait(&bars.mma2[(c - 1) & 1], ((c - 1) >> 1) & 1, globaltimer_ns() + kWaitNs);
         }
-    } else if (warp < 4) {
-        // ---- WG0: the delta and the state passes; thread j = value channel j ----
-        const int j = tid;
-        const uint32_t lq = 32 * warp;
-        uint32_t r32[32];
-        // Initial state: S^T row j = column j of S0; bf16 copy and pre-decay.
+    } else {
+        // ---- epilogue, warps 0-7: thread j = TMEM lane = value channel j; half hh
+        // takes delta rows 32 hh .., state columns 64 hh .. and output rows 32 hh .. ----
+        const int j = tid & 127, hh = warp >> 2;
+        const uint32_t lq = 32 * (warp & 3);
+        uint32_t ra[32], rb[32];
+        // Initial state: S^T row j = column j of S0 (this half's 64 key channels):
+        // fp32 master pre-multiplied by the first chunk's decay, and the bf16 copy.
         bool ok = true;
         const float *dec0 = nullptr;
         if (S0) {
@@ -683,22 +694,52 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
             if (!ok) { record_timeout(status); sAbort = 1; }
             dec0 = (const float *)(sm + kOffDecay);
         }
-        for (int q4 = 0; q4 < 4 && ok; ++q4) {
+        for (int q2 = 0; q2 < 2 && ok; ++q2) {
+            const int c0 = 64 * hh + 32 * q2;
             float sv[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                sv[i] = S0 ? S0[sbase + (size_t)(32 * q4 + i) * kDV + j] : 0.f;
+            for (int i = 0; i < 32; ++i) sv[i] = S0 ? S0[sbase + (size_t)(c0 + i) * kDV + j] : 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r32[i] = __float_as_uint(S0 ? sv[i] * dec0[32 * q4 + i] : 0.f);
-            tmem_st32(tmem_addr(tb, lq, kTS + 32 * q4), r32);
+            for (int i = 0; i < 32; ++i) ra[i] = __float_as_uint(S0 ? sv[i] * dec0[c0 + i] : 0.f);
+            tmem_st32(tmem_addr(tb, lq, kTS + c0), ra);
             uint32_t sb[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) sb[i] = pack_bf16(sv[2 * i], sv[2 * i + 1]);
-            tmem_st16(tmem_addr(tb, lq, kTSbf + 16 * q4), sb);
+            tmem_st16(tmem_addr(tb, lq, kTSbf + c0 / 2), sb);
         }
         tmem_st_wait();
         tc_fence_before_sync();
         mbar_arrive(&bars.sbf_ready);
+        mbar_arrive(&bars.sdec_ready);
+
+        // O^T rows of chunk cc -> o: each thread parks its 32 values in a [64][128]
+        // bf16 staging tile (double-buffered by chunk parity), then the 256
+        // threads write whole 256-byte token rows with 16-byte stores.
+        auto output = [&](int cc) {
+            const int bb = cc & 1;
+            const int t0 = tbeg + cc * kChunk;
+            const int len = min(kChunk, tend - t0);
+            __nv_bfloat16 *ost = (__nv_bfloat16 *)(sm + kOStage + bb * 16384);
+            tmem_ld32(tmem_addr(tb, lq, kTD1 + 128 * bb + 64 + 32 * hh), ra);
+            tmem_ld_wait();
+            tc_fence_before_sync();
+            mbar_arrive(&bars.d1_free[bb]);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ost[(32 * hh + i) * kDV + j] = __float2bfloat16_rn(__uint_as_float(ra[i]));
+            mbar_arrive(&bars.ostaged[bb]);
+            if (!mbar_wait(&bars.ostaged[bb], (cc >> 1) & 1, globaltimer_ns() + kWaitNs)) {
+                record_timeout(status);
+                sAbort = 1;
+                return;
+            }
+            const int r = tid >> 2, part = tid & 3;
+            if (r < len) {
+                const uint4 *src = (const uint4 *)(ost + r * kDV + 32 * part);
+                uint4 *dst = (uint4 *)(o + ((size_t)(t0 + r) * H + h) * kDV + 32 * part);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) dst[m] = src[m];
+            }
+        };
 
         for (int c = 0; c < nch && !sAbort; ++c) {
             const int s = c % kStages, b = c & 1;
@@ -708,106 +749,88 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
                 record_timeout(status); sAbort = 1; break;
             }
             tc_fence_after_sync();
-            // Dl^T[j][r] = U[r][j] - D1[j][r], r < 64 -> bf16 pairs into TMEM.
-            const __nv_bfloat16 *U = (const __nv_bfloat16 *)(st + kOffU);
-            uint32_t dl[32];
-#pragma unroll
-            for (int hlf = 0; hlf < 2; ++hlf) {
-                tmem_ld32(tmem_addr(tb, lq, kTD1 + 128 * b + 32 * hlf), r32);
+            // Dl^T[j][r] = U[r][j] - D1[j][r] for this half's 32 rows -> bf16 pairs into TMEM.
+            {
+                const __nv_bfloat16 *U = (const __nv_bfloat16 *)(st + kOffU);
+                tmem_ld32(tmem_addr(tb, lq, kTD1 + 128 * b + 32 * hh), ra);
                 tmem_ld_wait();
+                uint32_t dl[16];
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
-                    const int r = 32 * hlf + i;
-                    const float d0 = __bfloat162float(U[r * kDV + j]) - __uint_as_float(r32[i]);
-                    const float d1v = __bfloat162float(U[(r + 1) * kDV + j]) - __uint_as_float(r32[i + 1]);
-                    dl[16 * hlf + (i >> 1)] = pack_bf16(d0, d1v);
+                    const int r = 32 * hh + i;
+                    const float d0 = __bfloat162float(U[r * kDV + j]) - __uint_as_float(ra[i]);
+                    const float d1v = __bfloat162float(U[(r + 1) * kDV + j]) - __uint_as_float(ra[i + 1]);
+                    dl[i >> 1] = pack_bf16(d0, d1v);
                 }
+                tmem_st16(tmem_addr(tb, lq, kTDl + 16 * hh), dl);
+                tmem_st_wait();
             }
-            tmem_st32(tmem_addr(tb, lq, kTDl), dl);
-            tmem_st_wait();
             tc_fence_before_sync();
             mbar_arrive(&bars.dl_ready);
             mbar_arrive(&bars.empty[s]);  // done with U of this stage
+            // The previous chunk's output, off the critical path (its D1 buffer is
+            // only reused by the product two chunks later).
+            if (c > 0) output(c - 1);
 
             if (!mbar_wait(&bars.mma2[b], (c >> 1) & 1, globaltimer_ns() + kWaitNs)) {
                 record_timeout(status); sAbort = 1; break;
             }
             tc_fence_after_sync();
             const bool last = (c + 1 == nch);
-            const float *dec = nullptr;
-            if (!last) {
+            // S_out, this half's 64 key channels: two loads, one wait.
+            tmem_ld32(tmem_addr(tb, lq, kTS + 64 * hh), ra);
+            tmem_ld32(tmem_addr(tb, lq, kTS + 64 * hh + 32), rb);
+            tmem_ld_wait();
+            // Checkpoint when the state after `pos` tokens falls on a multiple of every.
+            const int pos = min((c + 1) * kChunk, tend - tbeg);
+            if (ckpt_every > 0 && pos % ckpt_every == 0) {
+                float *ck = ckpts + ((size_t)(ckpt_off[n] + pos / ckpt_every - 1) * H + h) * kDK * kDV;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    ck[(size_t)(64 * hh + i) * kDV + j] = __uint_as_float(ra[i]);
+                    ck[(size_t)(64 * hh + 32 + i) * kDV + j] = __uint_as_float(rb[i]);
+                }
+            }
+            if (last) {
+                if (Sf) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        Sf[sbase + (size_t)(64 * hh + i) * kDV + j] = __uint_as_float(ra[i]);
+                        Sf[sbase + (size_t)(64 * hh + 32 + i) * kDV + j] = __uint_as_float(rb[i]);
+                    }
+                }
+            } else {
+                // Critical: the bf16 copy that the next chunk's first product reads.
+                uint32_t sa[16], sbv[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    sa[i] = pack_bf16(__uint_as_float(ra[2 * i]), __uint_as_float(ra[2 * i + 1]));
+                    sbv[i] = pack_bf16(__uint_as_float(rb[2 * i]), __uint_as_float(rb[2 * i + 1]));
+                }
+                tmem_st16(tmem_addr(tb, lq, kTSbf + 32 * hh), sa);
+                tmem_st16(tmem_addr(tb, lq, kTSbf + 32 * hh + 16), sbv);
+                tmem_st_wait();
+                tc_fence_before_sync();
+                mbar_arrive(&bars.sbf_ready);
+                // Off the critical path: the fp32 master times the next chunk's decay.
                 const int s1 = (c + 1) % kStages;
                 if (!mbar_wait(&bars.full[s1], ((c + 1) / kStages) & 1, globaltimer_ns() + kWaitNs)) {
                     record_timeout(status); sAbort = 1; break;
                 }
-                dec = (const float *)(sm + s1 * kStageBytes + kOffDecay);
-            }
-            // Checkpoint when the state after `pos` tokens falls on a multiple of every.
-            const int pos = min((c + 1) * kChunk, tend - tbeg);
-            float *ck = nullptr;
-            if (ckpt_every > 0 && pos % ckpt_every == 0)
-                ck = ckpts + ((size_t)(ckpt_off[n] + pos / ckpt_every - 1) * H + h) * kDK * kDV;
-            // S_out -> bf16 copy for the next chunk, and pre-decayed fp32 state.
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                tmem_ld32(tmem_addr(tb, lq, kTS + 32 * q4), r32);
-                tmem_ld_wait();
-                if (ck) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        ck[(size_t)(32 * q4 + i) * kDV + j] = __uint_as_float(r32[i]);
-                }
-                if (last) {
-                    if (Sf) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            Sf[sbase + (size_t)(32 * q4 + i) * kDV + j] = __uint_as_float(r32[i]);
-                    }
-                    continue;
-                }
-                uint32_t sb[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    sb[i] = pack_bf16(__uint_as_float(r32[2 * i]), __uint_as_float(r32[2 * i + 1]));
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    r32[i] = __float_as_uint(__uint_as_float(r32[i]) * dec[32 * q4 + i]);
-                tmem_st32(tmem_addr(tb, lq, kTS + 32 * q4), r32);
-                tmem_st16(tmem_addr(tb, lq, kTSbf + 16 * q4), sb);
-            }
-            if (!last) {
-                tmem_st_wait();
-                tc_fence_before_sync();
-                mbar_arrive(&bars.sbf_ready);
-            }
-        }
-    } else {
-        // ---- WG1: outputs; thread j = value channel j ----
-        const int j = tid - 128;
-        const uint32_t lq = 32 * (warp - 4);
-        uint32_t r32[32];
-        for (int c = 0; c < nch && !sAbort; ++c) {
-            const int b = c & 1;
-            if (!mbar_wait(&bars.mma2[b], (c >> 1) & 1, globaltimer_ns() + kWaitNs)) {
-                record_timeout(status); sAbort = 1; break;
-            }
-            tc_fence_after_sync();
-            const int t0 = tbeg + c * kChunk;
-            const int len = min(kChunk, tend - t0);
-#pragma unroll
-            for (int hlf = 0; hlf < 2; ++hlf) {
-                tmem_ld32(tmem_addr(tb, lq, kTD1 + 128 * b + 64 + 32 * hlf), r32);
-                tmem_ld_wait();
+                const float *dec = (const float *)(sm + s1 * kStageBytes + kOffDecay) + 64 * hh;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const int r = 32 * hlf + i;
-                    if (r < len)
-                        o[((size_t)(t0 + r) * H + h) * kDV + j] = __float2bfloat16_rn(__uint_as_float(r32[i]));
+                    ra[i] = __float_as_uint(__uint_as_float(ra[i]) * dec[i]);
+                    rb[i] = __float_as_uint(__uint_as_float(rb[i]) * dec[32 + i]);
                 }
+                tmem_st32(tmem_addr(tb, lq, kTS + 64 * hh), ra);
+                tmem_st32(tmem_addr(tb, lq, kTS + 64 * hh + 32), rb);
+                tmem_st_wait();
+                tc_fence_before_sync();
+                mbar_arrive(&bars.sdec_ready);
             }
-            tc_fence_before_sync();
-            mbar_arrive(&bars.d1_free[b]);
         }
+        if (!sAbort) output(nch - 1);  // the last chunk's output
     }
     tc_fence_before_sync();
     __syncthreads();
