@@ -369,7 +369,37 @@ def main():
         decode = {"config": dcfg.name, "ms_per_step": dms, "state_gbs": dgbs,
                   "frac_of_hbm": dgbs / hbm_peak, "steps": args.decode_steps,
                   "state_bytes_per_step": state_bytes, "gpu_launches": args.decode_steps}
-        del d, od
+
+        # Speculative decoding on the same batch: verify 4 drafts per sequence (state
+        # read once, not written), then replay the accepted ones (here all 4).
+        Tq = 4
+        sq, sk, sv, sz = (d[key][:Tq].permute(1, 0, 2, 3).contiguous() for key in ("q", "k", "v", "z"))
+        sbeta = d["beta"][:Tq].permute(1, 0, 2).contiguous()
+        so = torch.empty(dcfg.B, Tq, dcfg.H, dcfg.dv, dtype=torch.bfloat16, device=dev)
+        for _ in range(args.warmup):
+            K.kda_decode_multi(sq, sk, sv, sz, d["A"], sbeta, d["state"], o=so, stream=stream)
+        torch.cuda.synchronize()
+        barrier()
+        reps = 50
+        e0.record(stream)
+        for _ in range(reps):
+            K.kda_decode_multi(sq, sk, sv, sz, d["A"], sbeta, d["state"], o=so, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        vms = max_over_ranks(e0.elapsed_time(e1), world, dev) / reps
+        e0.record(stream)
+        for _ in range(reps):
+            K.kda_decode_multi(sq, sk, sv, sz, d["A"], sbeta, d["state"], update_state=True,
+                               want_outputs=False, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        rms = max_over_ranks(e0.elapsed_time(e1), world, dev) / reps
+        decode["spec_verify"] = {"drafts": Tq, "ms": vms,
+                                 "state_read_gbs": state_bytes / 2 / (vms / 1e3) / 1e9,
+                                 "tokens_per_s": dcfg.B * Tq / (vms / 1e3)}
+        decode["spec_replay"] = {"accepted": Tq, "ms": rms,
+                                 "state_gbs": state_bytes / (rms / 1e3) / 1e9}
+        del d, od, so
 
         # End to end through the C ABI: pinned host inputs -> device, prefill, result -> host.
         host = {key: inp[key].cpu().pin_memory() for key in ("q", "k", "v", "z", "beta", "A")}

@@ -225,6 +225,33 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
                            void *stream);
 
 /*
+ * Speculative-decoding verify and replay ("Kimi K3 Under the Hood", section
+ * "Serving two incompatible cache types": rejected drafts must not advance the
+ * recurrent state; the projected inputs of the drafts are kept and the accepted
+ * tokens are replayed on-chip in one fused recurrence instead of saving a state
+ * per draft position).  Each (sequence, head) state is read once, the tokens run
+ * on-chip in the section 3.2 edit order, and the state is written at most once.
+ *
+ *   q, k, z [B, Tq, H, dk], v [B, Tq, H, dv] in dtype dt; beta [B, Tq, H] fp32;
+ *   the Tq tokens of sequence b are consecutive positions after its state.
+ *   state, pool_size, slots  as kda_decode_step (pool [P, H, dk, dv] fp32).
+ *   num_tokens   device int32 [B]: tokens of sequence b to apply (clamped to
+ *                [0, Tq]), or NULL for all Tq.
+ *   update_state 0 = verify: o receives every applied token's output and the
+ *                state in HBM is left untouched; 1 = replay/commit: the state of
+ *                each sequence is advanced by its num_tokens[b] tokens in place
+ *                (o is written too when non-NULL).
+ *   o            [B, Tq, H, dv] dtype dt, or NULL (then update_state must be 1).
+ * Tq in [1, 64].  Errors as kda_decode_step.
+ */
+kda_status kda_decode_multi(const void *q, const void *k, const void *v, const void *z,
+                            const float *A, const float *beta, int32_t B, int32_t Tq, int32_t H,
+                            int32_t dk, int32_t dv, kda_dtype dt, float *state,
+                            int32_t pool_size, const int32_t *slots,
+                            const int32_t *num_tokens, int32_t update_state, void *o,
+                            void *stream);
+
+/*
  * Reads and clears the library's device status word for the current device
  * (synchronises `stream` first).  Kernels that wait on an on-chip barrier
  * with an iteration limit record KDA_ERR_TIMEOUT there instead of hanging;

@@ -37,6 +37,7 @@ SIGNATURES = {
     "kda_prefill_noalloc": ([_P] * 8 + [_I32] * 6 + [_P] * 4, _I32),
     "kda_decode_step": ([_P] * 6 + [_I32] * 5 + [_P, _I32, _P, _P, _P], _I32),
     "kda_device_status": ([_P, _P], _I32),
+    "kda_decode_multi": ([_P] * 6 + [_I32] * 6 + [_P, _I32, _P, _P, _I32, _P, _P], _I32),
     "kda_selftest_wait_timeout": ([ctypes.c_int64, _P], _I32),
 }
 
@@ -235,6 +236,30 @@ def kda_decode_step(q, k, v, z, A, beta, state, slots=None, o=None, stream=None)
         KDA_DTYPE[dt], _dev(state, "state", torch.float32), state.shape[0],
         _dev(slots, "slots", torch.int32), _dev(o, "o", dt), _stream_ptr(stream))
     _check(code, "kda_decode_step")
+    return o
+
+
+def kda_decode_multi(q, k, v, z, A, beta, state, slots=None, num_tokens=None,
+                     update_state: bool = False, o=None, want_outputs: bool = True, stream=None):
+    """Speculative-decoding verify (update_state=False: outputs for every draft
+    token, state untouched) or replay (update_state=True: advance each sequence's
+    state by its first num_tokens[b] tokens in place).
+
+    q, k, z [B,Tq,H,dk], v [B,Tq,H,dv]; beta [B,Tq,H] fp32; state [P,H,dk,dv] fp32.
+    Returns o [B,Tq,H,dv] (or None when want_outputs is False in replay mode).
+    """
+    B, Tq, H, dk = q.shape
+    dv = v.shape[3]
+    dt = q.dtype
+    if o is None and (want_outputs or not update_state):
+        o = torch.empty(B, Tq, H, dv, dtype=dt, device=q.device)
+    code = _lib.kda_decode_multi(
+        _dev(q, "q", dt), _dev(k, "k", dt), _dev(v, "v", dt), _dev(z, "z", dt),
+        _dev(A, "A", torch.float32), _dev(beta, "beta", torch.float32), B, Tq, H, dk, dv,
+        KDA_DTYPE[dt], _dev(state, "state", torch.float32), state.shape[0],
+        _dev(slots, "slots", torch.int32), _dev(num_tokens, "num_tokens", torch.int32),
+        1 if update_state else 0, _dev(o, "o", dt), _stream_ptr(stream))
+    _check(code, "kda_decode_multi")
     return o
 
 

@@ -209,6 +209,37 @@ extern "C" kda_status kda_decode_step(const void *q, const void *k, const void *
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+extern "C" kda_status kda_decode_multi(const void *q, const void *k, const void *v, const void *z,
+                                       const float *A, const float *beta, int32_t B, int32_t Tq,
+                                       int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+                                       float *state, int32_t pool_size, const int32_t *slots,
+                                       const int32_t *num_tokens, int32_t update_state, void *o,
+                                       void *stream)
+{
+    if (B < 0 || H <= 0 || pool_size < 0 || Tq < 1 || Tq > 64) return KDA_ERR_INVALID_ARG;
+    if (dt != KDA_DTYPE_BF16 && dt != KDA_DTYPE_F32) return KDA_ERR_INVALID_ARG;
+    if (update_state != 0 && update_state != 1) return KDA_ERR_INVALID_ARG;
+    if (dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (B == 0) return KDA_OK;
+    if (!q || !k || !v || !z || !A || !beta || !state) return KDA_ERR_INVALID_ARG;
+    if (!o && !update_state) return KDA_ERR_INVALID_ARG;   // verify without outputs does nothing
+    if (!slots && pool_size < B) return KDA_ERR_INVALID_ARG;
+    for (const void *p : {q, k, v, z, (const void *)o, (const void *)state})
+        if (p && !aligned(p, 16)) return KDA_ERR_INVALID_ARG;
+    if (!aligned(A, 4) || !aligned(beta, 4) || (slots && !aligned(slots, 4)) ||
+        (num_tokens && !aligned(num_tokens, 4)))
+        return KDA_ERR_INVALID_ARG;
+
+    kda::DecodeMultiArgs a;
+    a.q = q; a.k = k; a.v = v; a.z = z; a.A = A; a.beta = beta;
+    a.B = B; a.Tq = Tq; a.H = H; a.dk = dk; a.dv = dv; a.bf16 = (dt == KDA_DTYPE_BF16);
+    a.state = state; a.slots = slots; a.num_tokens = num_tokens;
+    a.update_state = update_state != 0; a.o = o;
+    cudaError_t err = kda::launch_decode_multi(a, (cudaStream_t)stream);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 extern "C" kda_status kda_device_status(void *stream, int32_t *status_out)
 {
     if (!status_out) return KDA_ERR_INVALID_ARG;

@@ -41,6 +41,21 @@ struct DecodeArgs {
     void *o;
 };
 
+struct DecodeMultiArgs {
+    const void *q, *k, *v, *z;      // [B, Tq, H, d]
+    const float *A, *beta;          // beta [B, Tq, H]
+    int32_t B, Tq, H, dk, dv;
+    bool bf16;
+    float *state;
+    const int32_t *slots;
+    const int32_t *num_tokens;      // [B] or nullptr (= Tq)
+    bool update_state;
+    void *o;                        // [B, Tq, H, dv] or nullptr
+};
+
+// Tq tokens per sequence on a register-resident state (verify / replay).
+cudaError_t launch_decode_multi(const DecodeMultiArgs &a, cudaStream_t stream);
+
 // Fused chunked prefill on CUDA cores, all arithmetic in fp32 (16-token chunks).
 cudaError_t launch_prefill_cuda_core(const PrefillArgs &a, cudaStream_t stream);
 

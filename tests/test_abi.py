@@ -187,3 +187,20 @@ def test_checkpoint_count_and_validation():
     assert B._lib.kda_prefill_checkpointed(*common, 96, _fake()) == INVALID   # not a multiple of 64
     assert B._lib.kda_prefill_checkpointed(*common, 64, None) == INVALID      # no buffer
     assert B._lib.kda_prefill_checkpointed(*common, 64, _fake(0x10008)) == INVALID  # misaligned
+
+
+def test_decode_multi_rejects_bad_arguments():
+    def call(**kw):
+        a = dict(Bn=2, Tq=4, H=2, dk=128, dv=128, dt=BF16, state=_fake(), P=2, slots=None, nt=None,
+                 upd=0, o=_fake())
+        a.update(kw)
+        return B._lib.kda_decode_multi(_fake(), _fake(), _fake(), _fake(), _fake(), _fake(), a["Bn"],
+                                       a["Tq"], a["H"], a["dk"], a["dv"], a["dt"], a["state"], a["P"],
+                                       a["slots"], a["nt"], a["upd"], a["o"], None)
+    assert call(Tq=0) == INVALID
+    assert call(Tq=65) == INVALID
+    assert call(upd=2) == INVALID
+    assert call(o=None, upd=0) == INVALID      # verify needs outputs
+    assert call(dk=48) == UNSUPPORTED
+    assert call(nt=_fake(0x10002)) == INVALID
+    assert call(Bn=0) == OK

@@ -289,3 +289,85 @@ def test_checkpoints_full_size_varlen_sampled_heads():
                                                   x["initial_state"].index_select(1, hs).cpu())
     assert relerr(to_np(ck.index_select(1, hs)), ref_ck) <= TOL_BF16
     assert relerr(to_np(S.index_select(1, hs)), ref_S) <= TOL_BF16
+
+
+# ---------------------------------------------- speculative verify / replay ----
+
+def _spec_inputs(B, Tq, H, dk, dv, dtype, seed, pool):
+    x = prefill_inputs([Tq] * B, H, dk, dv, dtype, seed=seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    state = (torch.randn(pool, H, dk, dv, generator=g) * 0.3).cuda()
+    slots = torch.randperm(pool, generator=g)[:B].to(torch.int32).cuda()
+    shaped = {key: x[key].view(B, Tq, *x[key].shape[1:]).cuda() for key in ("q", "k", "v", "z", "beta")}
+    return x, shaped, state, slots
+
+
+@pytest.mark.parametrize("dtype,tol", [("bf16", TOL_BF16), ("f32", TOL_F32)])
+def test_spec_verify_leaves_state_and_matches_prefill(dtype, tol):
+    B, Tq, H, dk, dv, P = 37, 5, 3, 128, 128, 50
+    x, s, state, slots = _spec_inputs(B, Tq, H, dk, dv, dtype, 60, P)
+    before = state.clone()
+    o = K.kda_decode_multi(s["q"], s["k"], s["v"], s["z"], x["A"].cuda(), s["beta"], state, slots)
+    torch.cuda.synchronize()
+    assert torch.equal(state, before)                      # a verify writes no state
+    s0 = before[slots.long()].cpu()
+    ref_o, _ = oracle.prefill(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"], x["cu_seqlens_host"], s0)
+    assert relerr(to_np(o).reshape(B * Tq, H, dv), ref_o) <= tol
+
+
+@pytest.mark.parametrize("dtype,tol", [("bf16", TOL_BF16), ("f32", TOL_F32)])
+def test_spec_replay_commits_accepted_prefix(dtype, tol):
+    B, Tq, H, dk, dv, P = 37, 6, 3, 64, 128, 41
+    x, s, state, slots = _spec_inputs(B, Tq, H, dk, dv, dtype, 61, P)
+    before = state.clone()
+    g = torch.Generator().manual_seed(7)
+    acc = torch.randint(0, Tq + 1, (B,), generator=g).to(torch.int32)
+    acc[0], acc[1] = 0, Tq
+    K.kda_decode_multi(s["q"], s["k"], s["v"], s["z"], x["A"].cuda(), s["beta"], state, slots,
+                       num_tokens=acc.cuda(), update_state=True, want_outputs=False)
+    torch.cuda.synchronize()
+    sl = slots.long().cpu()
+    untouched = sorted(set(range(P)) - set(sl.tolist()))
+    assert torch.equal(state[untouched], before[untouched])
+    assert torch.equal(state[sl[0]], before[sl[0]])         # zero accepted tokens: unchanged
+    for b in range(B):
+        a = int(acc[b])
+        if a == 0:
+            continue
+        tok = slice(b * Tq, b * Tq + a)
+        _, ref_S = oracle.prefill(*(x[key][tok] for key in ("q", "k", "v", "z")), x["A"],
+                                  x["beta"][tok], np.array([0, a], np.int32),
+                                  before[sl[b]].cpu()[None])
+        assert relerr(to_np(state[sl[b]]), ref_S[0]) <= tol
+
+
+def test_spec_single_token_replay_equals_decode_step():
+    B, H = 16, 4
+    d = decode_inputs(B, H, 128, 128, "bf16", seed=62, nsets=1, device="cuda")
+    st1, st2 = d["state"].clone(), d["state"].clone()
+    o1 = K.kda_decode_step(d["q"][0], d["k"][0], d["v"][0], d["z"][0], d["A"], d["beta"][0], st1)
+    o2 = K.kda_decode_multi(d["q"][0][:, None], d["k"][0][:, None], d["v"][0][:, None],
+                            d["z"][0][:, None], d["A"], d["beta"][0][:, None], st2,
+                            update_state=True)
+    torch.cuda.synchronize()
+    assert torch.equal(st1, st2)
+    assert torch.equal(o1, o2[:, 0])
+
+
+def test_spec_full_batch_verify_then_replay():
+    """B = 256 sequences, H = 96, 4 drafts each: verify, then replay all four,
+    equals four decode steps; the verify outputs equal the steps' outputs."""
+    B, H, Tq = 256, 96, 4
+    d = decode_inputs(B, H, 128, 128, "bf16", seed=63, nsets=Tq, device="cuda")
+    q, k, v, z = (d[key].permute(1, 0, 2, 3).contiguous() for key in ("q", "k", "v", "z"))
+    beta = d["beta"].permute(1, 0, 2).contiguous()
+    st_steps = d["state"].clone()
+    outs = [K.kda_decode_step(d["q"][t], d["k"][t], d["v"][t], d["z"][t], d["A"], d["beta"][t], st_steps)
+            for t in range(Tq)]
+    st = d["state"].clone()
+    ov = K.kda_decode_multi(q, k, v, z, d["A"], beta, st)
+    K.kda_decode_multi(q, k, v, z, d["A"], beta, st, update_state=True, want_outputs=False)
+    torch.cuda.synchronize()
+    assert relerr(to_np(st), to_np(st_steps)) <= 1e-6
+    for t in range(Tq):
+        assert relerr(to_np(ov[:, t]), to_np(outs[t])) <= 1e-2
