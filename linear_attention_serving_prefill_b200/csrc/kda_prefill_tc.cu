@@ -145,16 +145,25 @@ constexpr uint32_t kRawStage = 4 * kRawTile;       // k, q, v, z
 constexpr uint32_t kRawK = 0, kRawQ = kRawTile, kRawV = 2 * kRawTile, kRawZ = 3 * kRawTile;
 // Shared memory (offsets from a 1024-aligned base).
 constexpr uint32_t kIRaw = 0;                      // 2 raw stages
-constexpr uint32_t kIRbig = 2 * kRawStage;         // 2 x 160 rows x 128 B: A-operands R^(I)
-constexpr uint32_t kIKQ = kIRbig + 40960;          // [Kt_I; Qt_I] per sub-tile, then [bK e^G; bV]^T
+// A operands of the A/P products, R^(I) = k e^{m_I - G} scaled to sub-tile I's
+// reference, stacked in pairs for M = 128 products: pair p holds R^(2p+1) in rows
+// 0..63 and R^(2p) in rows 64..127, one 128-row x 128-byte sub-block per 64-wide
+// K half.  Rows that are never valid (R^(I) beyond row 16 I + 15) sit at the ends
+// of some sub-blocks, so the next buffer starts inside that tail: the product
+// reads whatever is there into rows it discards, and nobody writes them.
+constexpr uint32_t kIRbig = 2 * kRawStage;
+__host__ __device__ constexpr uint32_t r_sub(int p, int kb) {
+    return p == 0 ? (kb == 0 ? 0u : 10240u) : (kb == 0 ? 20480u : 34816u);
+}
+constexpr uint32_t kIKQ = kIRbig + 49152;          // [Kt_I; Qt_I] per sub-tile, then [bK e^G; bV]^T
 constexpr uint32_t kISmem = kIKQ + 32768;
 // Reused inside Rbig once the A/P products are read back:
 constexpr uint32_t kIAf = kIRbig;                  // fp32 A [64][65]
 constexpr uint32_t kITf = kIRbig + 16640;          // fp32 T [64][65]
 constexpr uint32_t kIXf = kIRbig + 33280;          // fp32 scratch [32][33]
 constexpr int kLd = 65;
-// First row of R^(I) in Rbig: 16 * (0 + 1 + ... + I) = 0, 16, 48, 96.
-__host__ __device__ constexpr int row_base(int I) { return 8 * I * (I + 1); }
+// Row block of sub-tile I inside its pair: 0 for the odd tile, 64 for the even one.
+__host__ __device__ constexpr int pair_slot_row(int I) { return (I & 1) ? 0 : 64; }
 
 struct IntraItem { int t0, len, g, h; };
 
@@ -246,6 +255,9 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         }
         cp_async_commit();
         if (lane == 0) {
+            // The stage's previous item staged W, U and Kd^T in it for bulk stores:
+            // all but the newest bulk group (this item's Kd^T) have finished reading.
+            bulk_wait_read<1>();
             info[sn] = IntraItem{t0, len, g, h};
             mbar_arrive_expect_tx(&full[sn], kRawStage);
             uint8_t *stn = sm + kIRaw + sn * kRawStage;
@@ -332,13 +344,16 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 const float2 e1 = make_float2(__expf(L[i].x), __expf(L[i].y));    // in [e^-80, 1]
                 const float2 e2 = make_float2(__expf(-L[i].x), __expf(-L[i].y));  // in [1, e^80]
                 const float br = sBeta[s][r];
-                *(uint32_t *)(sKQ + sw128_offset(32 * I + ri, c0, 128)) = pack_bf16(kv.x * e1.x, kv.y * e1.y);
-                *(uint32_t *)(sKQ + sw128_offset(32 * I + 16 + ri, c0, 128)) = pack_bf16(qv.x * e1.x, qv.y * e1.y);
+                // B rows of pair I / 2: [Kt_odd; Qt_odd; Kt_even; Qt_even], 16 rows each.
+                const int brow = 64 * (I >> 1) + ((I & 1) ? 0 : 32) + ri;
+                *(uint32_t *)(sKQ + sw128_offset(brow, c0, 128)) = pack_bf16(kv.x * e1.x, kv.y * e1.y);
+                *(uint32_t *)(sKQ + sw128_offset(brow + 16, c0, 128)) = pack_bf16(qv.x * e1.x, qv.y * e1.y);
                 const float2 kb = make_float2(kv.x * e2.x, kv.y * e2.y);
 #pragma unroll
                 for (int Ip = 0; Ip < 4; ++Ip)
                     if (Ip >= I)
-                        *(uint32_t *)(sR + sw128_offset(row_base(Ip) + r, c0, 160)) =
+                        *(uint32_t *)(sR + r_sub(Ip >> 1, c0 >> 6) +
+                                      sw128_offset(pair_slot_row(Ip) + r, c0 & 63, 128)) =
                             pack_bf16(kb.x * fac[Ip].x, kb.y * fac[Ip].y);
                 *(uint32_t *)(blk + kOffWQ + sw128_offset(64 + r, c0, 128)) =
                     pack_bf16(qv.x * e1.x * emI.x, qv.y * e1.y * emI.y);
@@ -354,8 +369,11 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                     kd0[i >> 1] |= hd0 << 16; kd1[i >> 1] |= hd1 << 16;
                 }
             }
-            *(uint4 *)(blk + kOffKd + sw128_offset(c0, 8 * q8, 128)) = make_uint4(kd0[0], kd0[1], kd0[2], kd0[3]);
-            *(uint4 *)(blk + kOffKd + sw128_offset(c0 + 1, 8 * q8, 128)) = make_uint4(kd1[0], kd1[1], kd1[2], kd1[3]);
+            // (K e^{G_C - G})^T is staged in the item's raw z tile (dead after pass 1)
+            // as the exact image of its block region, then bulk-stored.
+            uint8_t *stw = sm + kIRaw + s * kRawStage;
+            *(uint4 *)(stw + kRawZ + sw128_offset(c0, 8 * q8, 128)) = make_uint4(kd0[0], kd0[1], kd0[2], kd0[3]);
+            *(uint4 *)(stw + kRawZ + sw128_offset(c0 + 1, 8 * q8, 128)) = make_uint4(kd1[0], kd1[1], kd1[2], kd1[3]);
             if (q8 == 0) {
                 ((float *)(blk + kOffDecay))[c0] = __expf(GC.x);
                 ((float *)(blk + kOffDecay))[c0 + 1] = __expf(GC.y);
@@ -367,15 +385,20 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             compute_sync();
             tc_fence_after_sync();
             if (tid == 0) {
-                const uint32_t id = idesc_bf16_f32(64, 32);
+                bulk_s2g(blk + kOffKd, stw + kRawZ, 16384);
+                bulk_commit();
+                // Pair p: D[:, 64p .. 64p+63] = [R^(2p+1); R^(2p)] [B_(2p+1); B_(2p)]^T
+                // (M = 128, N = 64); the wanted blocks are rows 0..63 x columns 0..31
+                // and rows 64..127 x columns 32..63.
+                const uint32_t id = idesc_bf16_f32(128, 64);
 #pragma unroll
-                for (int I = 0; I < 4; ++I)
+                for (int pp = 0; pp < 2; ++pp)
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t kb2 = ks >> 2, kin = ks & 3;
-                        const uint32_t a = smem_u32(sR) + kb2 * 160 * 128 + row_base(I) * 128 + kin * 32;
-                        const uint32_t b = smem_u32(sKQ) + kb2 * 128 * 128 + 32 * I * 128 + kin * 32;
-                        mma_ss(tmem_addr(tb, 0, 32 * I), desc_kmajor_sw128(a), desc_kmajor_sw128(b), id, ks > 0);
+                        const uint32_t a = smem_u32(sR) + r_sub(pp, kb2) + kin * 32;
+                        const uint32_t b = smem_u32(sKQ) + kb2 * 128 * 128 + 64 * pp * 128 + kin * 32;
+                        mma_ss(tmem_addr(tb, 0, 64 * pp), desc_kmajor_sw128(a), desc_kmajor_sw128(b), id, ks > 0);
                     }
                 mma_commit(&mma_bar);
             }
@@ -395,13 +418,15 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
 
             float *Af = (float *)(sm + kIAf), *Tf = (float *)(sm + kITf), *Xf = (float *)(sm + kIXf);
             {
-                // M = 64 layout: warp (w % 4) lanes 0-15 hold rows s = 16 (w % 4) + lane;
-                // warp w reads sub-tile w / 4.
-                uint32_t rr[32];
-                const int wq = warp & 3, sidx = 16 * wq + lane, Ia = warp >> 2;
-                tmem_ld32(tmem_addr(tb, 32 * wq, 32 * Ia), rr);
-                tmem_ld_wait();
-                if (lane < 16) {
+                // M = 128 layout: TMEM lane = A row.  Warps 0-7: pair p = warp / 4,
+                // lane quarter q = warp % 4; quarters 0-1 hold R^(2p+1) rows (wanted
+                // columns 0..31 of the pair), quarters 2-3 hold R^(2p) rows (32..63).
+                if (warp < 8) {
+                    uint32_t rr[32];
+                    const int q = warp & 3, pp = warp >> 2, slot = q >> 1;
+                    const int sidx = 32 * (q & 1) + lane, Ia = slot ? 2 * pp : 2 * pp + 1;
+                    tmem_ld32(tmem_addr(tb, 32 * q, 64 * pp + 32 * slot), rr);
+                    tmem_ld_wait();
 #pragma unroll
                     for (int jr = 0; jr < 16; ++jr) {
                         const int r = 16 * Ia + jr;
@@ -420,8 +445,8 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             compute_sync();
 
             // T, rounded to bf16, is also the A operand of the W/U product
-            // (64 rows x 64 K), written into the item's raw z tile as it is formed.
-            uint8_t *sT = sm + kIRaw + s * kRawStage + kRawZ;
+            // (64 rows x 64 K), written into the item's raw k tile as it is formed.
+            uint8_t *sT = stw + kRawK;
             // T = (I + A)^-1 by blocks of 16: diagonal blocks by forward
             // substitution, then T_ij = -T_ii A_ij T_jj doubled from 16 to 32 to 64.
             // Only the lower triangle is used; the two upper blocks that the
@@ -461,14 +486,21 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 // Level 1, blocks (1,0) and (3,2): X = A_ij T_jj, one output per thread.
                 const int p = tid >> 8, r = (tid >> 4) & 15, sb = tid & 15;
                 const int oi = 32 * p + 16, oj = 32 * p;
-                float x0 = 0.f;
+                float x0 = 0.f, x1 = 0.f;
 #pragma unroll
-                for (int t = 0; t < 16; ++t) x0 = fmaf(Af[(oi + r) * kLd + oj + t], Tf[(oj + t) * kLd + oj + sb], x0);
-                Xf[(16 * p + r) * 33 + sb] = x0;
+                for (int t = 0; t < 16; t += 2) {
+                    x0 = fmaf(Af[(oi + r) * kLd + oj + t], Tf[(oj + t) * kLd + oj + sb], x0);
+                    x1 = fmaf(Af[(oi + r) * kLd + oj + t + 1], Tf[(oj + t + 1) * kLd + oj + sb], x1);
+                }
+                Xf[(16 * p + r) * 33 + sb] = x0 + x1;
                 compute_sync();
-                float y0 = 0.f;
+                float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-                for (int t = 0; t < 16; ++t) y0 = fmaf(Tf[(oi + r) * kLd + oi + t], Xf[(16 * p + t) * 33 + sb], y0);
+                for (int t = 0; t < 16; t += 2) {
+                    y0 = fmaf(Tf[(oi + r) * kLd + oi + t], Xf[(16 * p + t) * 33 + sb], y0);
+                    y1 = fmaf(Tf[(oi + r) * kLd + oi + t + 1], Xf[(16 * p + t + 1) * 33 + sb], y1);
+                }
+                y0 += y1;
                 Tf[(oi + r) * kLd + oj + sb] = -y0;
                 *(__nv_bfloat16 *)(sT + sw128_offset(oi + r, oj + sb, 64)) = __float2bfloat16_rn(-y0);
             }
@@ -476,23 +508,30 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             {
                 // Level 2, block rows 32..63 x columns 0..31: two outputs per thread.
                 const int r = tid >> 4, sb = tid & 15;
-                float x[2] = {0.f, 0.f};
-#pragma unroll 8
-                for (int t = 0; t < 32; ++t) {
-                    const float a = Af[(32 + r) * kLd + t];
+                float x[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) x[jj] = fmaf(a, Tf[t * kLd + sb + 16 * jj], x[jj]);
+                for (int t = 0; t < 32; t += 2) {
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const float a = Af[(32 + r) * kLd + t + u];
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) x[u][jj] = fmaf(a, Tf[(t + u) * kLd + sb + 16 * jj], x[u][jj]);
+                    }
                 }
 #pragma unroll
-                for (int jj = 0; jj < 2; ++jj) Xf[r * 33 + sb + 16 * jj] = x[jj];
+                for (int jj = 0; jj < 2; ++jj) Xf[r * 33 + sb + 16 * jj] = x[0][jj] + x[1][jj];
                 compute_sync();
-                float y[2] = {0.f, 0.f};
-#pragma unroll 8
-                for (int t = 0; t < 32; ++t) {
-                    const float tt = Tf[(32 + r) * kLd + 32 + t];
+                float yy[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) y[jj] = fmaf(tt, Xf[t * 33 + sb + 16 * jj], y[jj]);
+                for (int t = 0; t < 32; t += 2) {
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const float tt = Tf[(32 + r) * kLd + 32 + t + u];
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) yy[u][jj] = fmaf(tt, Xf[(t + u) * 33 + sb + 16 * jj], yy[u][jj]);
+                    }
                 }
+                const float y[2] = {yy[0][0] + yy[1][0], yy[0][1] + yy[1][1]};
 #pragma unroll
                 for (int jj = 0; jj < 2; ++jj)
                     *(__nv_bfloat16 *)(sT + sw128_offset(32 + r, sb + 16 * jj, 64)) = __float2bfloat16_rn(-y[jj]);
@@ -521,11 +560,17 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 // Warp w: lane quadrant w % 4, columns 64 (w / 4) .. + 63.
                 uint32_t rr[32];
                 const int wq = warp & 3, r = 16 * wq + lane, cg = warp >> 2;
+                uint32_t rr2[32];
+                tmem_ld32(tmem_addr(tb, 32 * wq, 64 * cg), rr);
+                tmem_ld32(tmem_addr(tb, 32 * wq, 64 * cg + 32), rr2);
+                tmem_ld_wait();
 #pragma unroll
                 for (int q4 = 0; q4 < 2; ++q4) {
                     const int colbase = 64 * cg + 32 * q4;
-                    tmem_ld32(tmem_addr(tb, 32 * wq, colbase), rr);
-                    tmem_ld_wait();
+                    if (q4 == 1) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) rr[i] = rr2[i];
+                    }
                     if (lane < 16) {
 #pragma unroll
                         for (int cc = 0; cc < 32; cc += 8) {
@@ -535,17 +580,27 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                                 pack_bf16(__uint_as_float(rr[cc + 4]), __uint_as_float(rr[cc + 5])),
                                 pack_bf16(__uint_as_float(rr[cc + 6]), __uint_as_float(rr[cc + 7])));
                             const int col = colbase + cc;
+                            // Staged as block images: W (two 64-wide K halves of rows
+                            // 0..63 of [W; Qt]) in the v tile, U (row-major) in the q tile.
                             if (col < 128)
-                                *(uint4 *)(blk + kOffWQ + sw128_offset(r, col, 128)) = w4;
+                                *(uint4 *)(stw + kRawV + (col >> 6) * 8192 + sw128_offset(r, col & 63, 64)) = w4;
                             else
-                                *(uint4 *)(blk + kOffU + (size_t)(r * 128 + col - 128) * 2) = w4;
+                                *(uint4 *)(stw + kRawQ + (r * 128 + col - 128) * 2) = w4;
                         }
                     }
                 }
             }
+            fence_proxy_async_smem();
             tc_fence_before_sync();
             compute_sync();
+            if (tid == 0) {
+                bulk_s2g(blk + kOffWQ, stw + kRawV, 8192);
+                bulk_s2g(blk + kOffWQ + 16384, stw + kRawV + 8192, 8192);
+                bulk_s2g(blk + kOffU, stw + kRawQ, 16384);
+                bulk_commit();
+            }
         }
+        if (tid == 0) bulk_wait<0>();  // every staged block region has reached memory
         // Drain: every requested copy has landed before the CTA may exit.
         if (warp == 0) {
             cp_async_wait_all();
