@@ -46,6 +46,18 @@ KERNELS = {
 FALLBACK_BF16_TFLOPS = 1590.0
 
 
+def split_kernels(G: int):
+    """Kernels of a call split into G segments per sequence, with their
+    algorithmic bytes per token-head when a fraction f = (G - 1) / G of the
+    chunks lies in segments >= 1: the state kernel reads the blocks of those
+    chunks twice (local and transition chains) and writes an E image (256 B/th)
+    for them besides o; the correction reads E and reads and writes o there.
+    The segment composition moves O(N H G) states, nothing per token."""
+    f = (G - 1) / G
+    return (["plan_kernel", "intra_kernel", "state_kernel", "compose_kernel", "correct_kernel"],
+            [0, 1028 + 1160, 1160 * (1 + f) + 256 + 256 * f, 0, 768 * f], "kda_prefill_tc.cu")
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -206,13 +218,66 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def split_leg(K, rank_seed, rank, world, dev, stream, args, max_over_ranks, barrier):
+    """The single-sequence 4,096-token, 32-head prefill (32 state chains for 148
+    SMs), whole and split into segments by the affine scan.  L2 is flushed
+    (a 256 MiB write) before every timed call; each call is timed alone."""
+    from dataclasses import replace
+
+    from linear_attention_serving_prefill_b200.workloads import CONFIGS, config_inputs
+    cfg = CONFIGS["prefill_4k"]
+    x = config_inputs(replace(cfg, seed=rank_seed(cfg.seed, rank)), device=dev)
+    T, H = x["q"].shape[0], cfg.H
+    o = torch.empty(T, H, cfg.dv, dtype=torch.bfloat16, device=dev)
+    S = torch.empty(1, H, cfg.dk, cfg.dv, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out = {"workload": cfg.name, "tokens": T, "heads": H, "l2": "flushed before every call"}
+    reps = 30
+    for algo in ("tensor_core", "auto"):
+        G = K.kda_prefill_segments(T, 1, H, cfg.dk, cfg.dv, torch.bfloat16, algo)
+        nk = K.kda_prefill_kernel_count(T, 1, H, cfg.dk, cfg.dv, torch.bfloat16, algo)
+        names = KERNELS[nk][0] if nk != 5 else split_kernels(G)[0]
+        ws = torch.empty(max(K.kda_prefill_workspace_size(T, 1, H, cfg.dk, cfg.dv, torch.bfloat16,
+                                                          algo), 1), dtype=torch.uint8, device=dev)
+
+        def call(ev=None):
+            K.kda_prefill(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"], x["cu_seqlens"],
+                          x["cu_seqlens_host"], None, final_state=S, o=o, workspace=ws, algo=algo,
+                          stream=stream, stage_events=ev)
+
+        for _ in range(args.warmup):
+            call()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(reps)]
+        for row in evs:
+            for e in row:
+                e.record(stream)   # creates the CUDA event
+        torch.cuda.synchronize()
+        barrier()
+        for i in range(reps):
+            flush.fill_(i & 0xFF)
+            call(evs[i])
+        torch.cuda.synchronize()
+        per = [statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(reps))
+               for j in range(nk)]
+        ms = max_over_ranks(sum(per), world, dev)
+        out["split" if G > 1 else "whole"] = {
+            "algo": algo, "segments": G, "ms": ms, "tokens_per_s": T / (ms / 1e3),
+            "kernels_ms": dict(zip(names, per))}
+        del ws
+    if "split" in out and "whole" in out:
+        out["speedup"] = out["whole"]["ms"] / out["split"]["ms"]
+    del x, o, S, flush
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--algo", default="auto", choices=["auto", "cuda_core", "tensor_core"])
+    ap.add_argument("--algo", default="auto",
+                    choices=["auto", "cuda_core", "tensor_core", "tensor_core_split"])
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -256,8 +321,10 @@ def main():
     ws_bytes = K.kda_prefill_workspace_size(T, 1, H, dk, dv, torch.bfloat16, args.algo)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
 
-    nk = K.kda_prefill_kernel_count(dk, dv, torch.bfloat16, args.algo)
-    kernel_names, kernel_bytes_per_th, kernel_file = KERNELS[nk]
+    nk = K.kda_prefill_kernel_count(T, 1, H, dk, dv, torch.bfloat16, args.algo)
+    n_seg = K.kda_prefill_segments(T, 1, H, dk, dv, torch.bfloat16, args.algo)
+    kernel_names, kernel_bytes_per_th, kernel_file = (KERNELS[nk] if nk != 5 else
+                                                      split_kernels(n_seg))
 
     def step(events=None):
         K.kda_prefill(inp["q"], inp["k"], inp["v"], inp["z"], inp["A"], inp["beta"],
@@ -312,8 +379,10 @@ def main():
             "roofline_ms": th * BYTES_PER_TOKEN_HEAD / hbm_peak / 1e6}
     launches = args.steps * nk
 
-    decode = e2e = cpu = ckpt = None
+    decode = e2e = cpu = ckpt = split = None
     if not args.prefill_only:
+        split = split_leg(K, rank_seed, rank, world, dev, stream, args, max_over_ranks, barrier)
+
         # Prefix-cache checkpoints every 512 tokens (the pages' hash block) on the same
         # workload: the cost of writing 64 KiB per (checkpoint, head) from the state pass.
         every = 512
@@ -453,6 +522,7 @@ def main():
             "path_roofline": path,
             "decode": decode,
             "checkpoints": ckpt,
+            "sequence_split": split,
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clocks,

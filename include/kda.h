@@ -50,7 +50,7 @@
 extern "C" {
 #endif
 
-#define KDA_ABI_VERSION 1
+#define KDA_ABI_VERSION 2
 
 typedef enum {
     KDA_OK = 0,
@@ -67,9 +67,13 @@ typedef enum {
 } kda_dtype;
 
 typedef enum {
-    KDA_ALGO_AUTO = 0,         /* tensor-core path for bf16, CUDA-core fp32 path for fp32 */
+    KDA_ALGO_AUTO = 0,         /* tensor-core path for bf16 (split when it pays, see
+                                  kda_prefill_segments), CUDA-core fp32 path for fp32 */
     KDA_ALGO_CUDA_CORE = 1,    /* chunked prefill in fp32 FMA on CUDA cores (check mode) */
-    KDA_ALGO_TENSOR_CORE = 2   /* chunked prefill on tcgen05 tensor cores (bf16 only) */
+    KDA_ALGO_TENSOR_CORE = 2,  /* chunked prefill on tcgen05 tensor cores (bf16 only),
+                                  every sequence one chain of chunks */
+    KDA_ALGO_TENSOR_CORE_SPLIT = 3  /* tensor cores with every sequence split into
+                                  segments composed by an affine scan (bf16 only) */
 } kda_algo;
 
 /* Version of this ABI (KDA_ABI_VERSION of the build). */
@@ -106,8 +110,9 @@ size_t kda_prefill_workspace_size(int32_t total_tokens, int32_t num_seqs, int32_
  *   workspace       device buffer of at least
  *                   kda_prefill_workspace_size(T, N, H, dk, dv, dt, algo) bytes
  *                   (may be NULL when that size is 0); contents are scratch.
- *   algo            KDA_ALGO_AUTO, or a forced path; KDA_ALGO_TENSOR_CORE with
- *                   dt = KDA_DTYPE_F32 or dk, dv != 128 returns KDA_ERR_UNSUPPORTED.
+ *   algo            KDA_ALGO_AUTO, or a forced path; KDA_ALGO_TENSOR_CORE(_SPLIT)
+ *                   with dt = KDA_DTYPE_F32 or dk, dv != 128 returns
+ *                   KDA_ERR_UNSUPPORTED.
  *   stage_events    optional instrumentation (NULL = none): an array of
  *                   num_stage_events cudaEvent_t handles (as void*), owned by
  *                   the caller.  events[0] is recorded on `stream` before the
@@ -170,10 +175,38 @@ int64_t kda_checkpoint_count(const int32_t *cu_seqlens_host, int32_t num_seqs,
                              int32_t checkpoint_every);
 
 /*
- * Number of kernels one kda_prefill_ex call launches for these sizes and
- * algorithm (for a non-empty batch); 0 for invalid arguments.
+ * Number of kernels one kda_prefill_ex call (no checkpoints) launches for these
+ * sizes and algorithm, for a non-empty batch: 1 on CUDA cores, 3 on tensor cores
+ * (plan, intra-chunk, state), 5 when the call splits its sequences (plus the
+ * segment composition and the output correction).  0 for invalid arguments.
  */
-int32_t kda_prefill_kernel_count(int32_t dk, int32_t dv, kda_dtype dt, kda_algo algo);
+int32_t kda_prefill_kernel_count(int32_t total_tokens, int32_t num_seqs, int32_t H, int32_t dk,
+                                 int32_t dv, kda_dtype dt, kda_algo algo);
+
+/*
+ * Segments per sequence that a kda_prefill_ex call without checkpoints uses
+ * for these sizes: 1 = no split; 0 for invalid arguments.
+ *
+ * Sequence split by affine composition ("Kimi K3 Under the Hood", section
+ * "Infrastructure for a 3T-class MoE", on KDA context parallelism: a sequence
+ * segment is summarised by the map it applies to the
+ * state, a cumulative dk x dk transition plus the state it produces from zero,
+ * and these maps compose associatively).  Here the segments of one sequence run
+ * on different SMs of one GPU: segment s >= 1 computes, from its chunk blocks,
+ * its state from zero S_loc(s), its transition M_s and, per chunk, the matrix E
+ * that maps the segment's true entry state to the missing part of the chunk's
+ * outputs; then S_in(s + 1) = M_s S_in(s) + S_loc(s) in fp32 and o += E S_in(s)
+ * on the tensor cores.  Results equal the unsplit path's up to rounding.
+ * The count: each (sequence, head) takes 2 G - 1 concurrent state chains, so G
+ * is the largest value with N H (2 G - 1) <= 148 (the B200's SMs), at most 16;
+ * KDA_ALGO_AUTO additionally requires T / (64 N) >= 16 G (long sequences) and
+ * KDA_ALGO_TENSOR_CORE_SPLIT at least 2.  A sequence with fewer chunks than G
+ * uses one segment per chunk.  kda_prefill_checkpointed with checkpoints never
+ * splits under AUTO and returns KDA_ERR_UNSUPPORTED under
+ * KDA_ALGO_TENSOR_CORE_SPLIT.
+ */
+int32_t kda_prefill_segments(int32_t total_tokens, int32_t num_seqs, int32_t H, int32_t dk,
+                             int32_t dv, kda_dtype dt, kda_algo algo);
 
 /*
  * kda_prefill without a workspace argument, for callers that cannot allocate

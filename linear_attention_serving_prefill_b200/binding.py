@@ -18,7 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libkda_b200.so")
 
 KDA_DTYPE = {torch.bfloat16: 0, torch.float32: 1}
-KDA_ALGO = {"auto": 0, "cuda_core": 1, "tensor_core": 2}
+KDA_ALGO = {"auto": 0, "cuda_core": 1, "tensor_core": 2, "tensor_core_split": 3}
 STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
                 3: "KDA_ERR_WORKSPACE", 4: "KDA_ERR_CUDA", 5: "KDA_ERR_TIMEOUT"}
 
@@ -30,7 +30,8 @@ SIGNATURES = {
     "kda_prefill_workspace_size": ([_I32, _I32, _I32, _I32, _I32, _I32, _I32], _SZ),
     "kda_prefill": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _P], _I32),
     "kda_prefill_ex": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _I32, _P, _P, _I32], _I32),
-    "kda_prefill_kernel_count": ([_I32, _I32, _I32, _I32], _I32),
+    "kda_prefill_kernel_count": ([_I32] * 7, _I32),
+    "kda_prefill_segments": ([_I32] * 7, _I32),
     "kda_prefill_checkpointed": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _I32, _P, _P, _I32, _I32, _P],
                                  _I32),
     "kda_checkpoint_count": ([_P, _I32, _I32], ctypes.c_int64),
@@ -219,8 +220,15 @@ def kda_prefill_noalloc(q, k, v, z, A, beta, cu_seqlens, cu_seqlens_host=None,
     return o, final_state
 
 
-def kda_prefill_kernel_count(dk: int, dv: int, dtype=torch.bfloat16, algo: str = "auto") -> int:
-    return int(_lib.kda_prefill_kernel_count(dk, dv, KDA_DTYPE[dtype], KDA_ALGO[algo]))
+def kda_prefill_kernel_count(T: int, N: int, H: int, dk: int, dv: int, dtype=torch.bfloat16,
+                             algo: str = "auto") -> int:
+    return int(_lib.kda_prefill_kernel_count(T, N, H, dk, dv, KDA_DTYPE[dtype], KDA_ALGO[algo]))
+
+
+def kda_prefill_segments(T: int, N: int, H: int, dk: int, dv: int, dtype=torch.bfloat16,
+                         algo: str = "auto") -> int:
+    """Segments per sequence the call uses (1 = no split, 0 = invalid arguments)."""
+    return int(_lib.kda_prefill_segments(T, N, H, dk, dv, KDA_DTYPE[dtype], KDA_ALGO[algo]))
 
 
 def kda_decode_step(q, k, v, z, A, beta, state, slots=None, o=None, stream=None):

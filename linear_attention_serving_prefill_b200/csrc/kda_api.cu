@@ -42,11 +42,13 @@ kda_status check_prefill_sizes(int32_t total_tokens, int32_t num_seqs, int32_t H
 {
     if (total_tokens < 0 || num_seqs < 0 || H <= 0) return KDA_ERR_INVALID_ARG;
     if (dt != KDA_DTYPE_BF16 && dt != KDA_DTYPE_F32) return KDA_ERR_INVALID_ARG;
-    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_CUDA_CORE && algo != KDA_ALGO_TENSOR_CORE)
+    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_CUDA_CORE && algo != KDA_ALGO_TENSOR_CORE &&
+        algo != KDA_ALGO_TENSOR_CORE_SPLIT)
         return KDA_ERR_INVALID_ARG;
     if (dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
-    if (algo == KDA_ALGO_TENSOR_CORE && (dt != KDA_DTYPE_BF16 || dk != 128 || dv != 128))
+    if ((algo == KDA_ALGO_TENSOR_CORE || algo == KDA_ALGO_TENSOR_CORE_SPLIT) &&
+        (dt != KDA_DTYPE_BF16 || dk != 128 || dv != 128))
         return KDA_ERR_UNSUPPORTED;
     return KDA_OK;
 }
@@ -55,9 +57,19 @@ kda_status check_prefill_sizes(int32_t total_tokens, int32_t num_seqs, int32_t H
 // CUDA-core path is forced; the fp32 CUDA-core path otherwise.
 bool use_tensor_core(int32_t dk, int32_t dv, kda_dtype dt, kda_algo algo)
 {
-    if (algo == KDA_ALGO_TENSOR_CORE) return true;
+    if (algo == KDA_ALGO_TENSOR_CORE || algo == KDA_ALGO_TENSOR_CORE_SPLIT) return true;
     if (algo == KDA_ALGO_CUDA_CORE) return false;
     return dt == KDA_DTYPE_BF16 && dk == 128 && dv == 128;
+}
+
+// Segments per sequence on the tensor-core path: AUTO splits when few
+// (sequence, head) chains would leave most SMs idle, SPLIT always does,
+// TENSOR_CORE never.  (Valid arguments assumed.)
+int32_t segments_for(int32_t total_tokens, int32_t num_seqs, int32_t H, int32_t dk, int32_t dv,
+                     kda_dtype dt, kda_algo algo)
+{
+    if (!use_tensor_core(dk, dv, dt, algo) || algo == KDA_ALGO_TENSOR_CORE) return 1;
+    return kda::tc_split_segments(total_tokens, num_seqs, H, algo == KDA_ALGO_TENSOR_CORE_SPLIT);
 }
 
 }  // namespace
@@ -81,8 +93,17 @@ extern "C" size_t kda_prefill_workspace_size(int32_t total_tokens, int32_t num_s
                                              int32_t dk, int32_t dv, kda_dtype dt, kda_algo algo)
 {
     if (check_prefill_sizes(total_tokens, num_seqs, H, dk, dv, dt, algo) != KDA_OK) return 0;
-    if (use_tensor_core(dk, dv, dt, algo)) return kda::tc_workspace_bytes(total_tokens, num_seqs, H);
+    if (use_tensor_core(dk, dv, dt, algo))
+        return kda::tc_workspace_bytes(total_tokens, num_seqs, H,
+                                       segments_for(total_tokens, num_seqs, H, dk, dv, dt, algo));
     return 0;  // the CUDA-core path keeps everything on chip
+}
+
+extern "C" int32_t kda_prefill_segments(int32_t total_tokens, int32_t num_seqs, int32_t H,
+                                        int32_t dk, int32_t dv, kda_dtype dt, kda_algo algo)
+{
+    if (check_prefill_sizes(total_tokens, num_seqs, H, dk, dv, dt, algo) != KDA_OK) return 0;
+    return segments_for(total_tokens, num_seqs, H, dk, dv, dt, algo);
 }
 
 extern "C" int64_t kda_checkpoint_count(const int32_t *cu_seqlens_host, int32_t num_seqs,
@@ -111,6 +132,7 @@ extern "C" kda_status kda_prefill_checkpointed(
     if (st != KDA_OK) return st;
     if (checkpoint_every < 0 || checkpoint_every % 64 != 0) return KDA_ERR_INVALID_ARG;
     if (checkpoint_every > 0 && (!checkpoints || !aligned(checkpoints, 16))) return KDA_ERR_INVALID_ARG;
+    if (checkpoint_every > 0 && algo == KDA_ALGO_TENSOR_CORE_SPLIT) return KDA_ERR_UNSUPPORTED;
     if (num_seqs > 0 && !cu_seqlens_dev) return KDA_ERR_INVALID_ARG;
     if (total_tokens > 0 && (!q || !k || !v || !z || !A || !beta || !o)) return KDA_ERR_INVALID_ARG;
     for (const void *p : {q, k, v, z, (const void *)o, (const void *)initial_state,
@@ -141,6 +163,9 @@ extern "C" kda_status kda_prefill_checkpointed(
     a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.status = status;
     a.events = stage_events; a.num_events = stage_events ? num_stage_events : 0;
     a.ckpt_every = checkpoint_every; a.checkpoints = checkpoint_every > 0 ? checkpoints : nullptr;
+    // Checkpoints come from the unsplit state chain; AUTO then keeps every
+    // sequence whole (its workspace, sized for a split, is large enough).
+    a.segments = checkpoint_every > 0 ? 1 : segments_for(total_tokens, num_seqs, H, dk, dv, dt, algo);
 
     cudaError_t err = use_tensor_core(dk, dv, dt, algo)
                           ? kda::launch_prefill_tensor_core(a, (cudaStream_t)stream)
@@ -177,10 +202,12 @@ extern "C" kda_status kda_prefill(const void *q, const void *k, const void *v, c
                           workspace_bytes, KDA_ALGO_AUTO, stream, nullptr, 0);
 }
 
-extern "C" int32_t kda_prefill_kernel_count(int32_t dk, int32_t dv, kda_dtype dt, kda_algo algo)
+extern "C" int32_t kda_prefill_kernel_count(int32_t total_tokens, int32_t num_seqs, int32_t H,
+                                            int32_t dk, int32_t dv, kda_dtype dt, kda_algo algo)
 {
-    if (check_prefill_sizes(0, 0, 1, dk, dv, dt, algo) != KDA_OK) return 0;
-    return use_tensor_core(dk, dv, dt, algo) ? 3 : 1;
+    if (check_prefill_sizes(total_tokens, num_seqs, H, dk, dv, dt, algo) != KDA_OK) return 0;
+    if (!use_tensor_core(dk, dv, dt, algo)) return 1;
+    return segments_for(total_tokens, num_seqs, H, dk, dv, dt, algo) > 1 ? 5 : 3;
 }
 
 extern "C" kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *z,

@@ -23,6 +23,7 @@ struct PrefillArgs {
     int32_t *status;                // device status word
     int32_t ckpt_every;             // 0 = no checkpoints, else a multiple of 64
     float *checkpoints;             // [count, H, dk, dv] or nullptr
+    int32_t segments;               // tensor-core path: segments per sequence (1 = no split)
     void *const *events;            // optional cudaEvent_t per kernel boundary
     int32_t num_events;
     // Records boundary i (0 = before the first kernel) when the caller asked for it.

@@ -630,12 +630,31 @@ struct StateBars {
 };
 constexpr uint32_t kEpi = 256;  // epilogue threads: two warpgroups
 
+// Segments: with G > 1 every sequence of nch chunks is cut into Gn = min(G, nch)
+// runs of chunks, [s nch / Gn, (s + 1) nch / Gn), and each (sequence, head) gets
+// 2 G - 1 CTAs ("slots"):
+//   slot 0          segment 0 from the true initial state; outputs -> o;
+//   slot 2 s - 1    segment s from a zero state (S_loc); outputs -> o (partial);
+//   slot 2 s        segment s on the transition X, X_0 = I and U = 0; its state
+//                   after the segment is the dk x dk map M_s, its outputs are
+//                   E = (Qt - P W) X per chunk, written as MMA A-operand images.
+// Segment ends: slot 0 -> Sx[n][0][h], slot 2s-1 -> Sx[n][s][h], slot 2s ->
+// Mx[n][s][h]; compose_kernel and correct_kernel finish the job.  With G == 1
+// the single slot writes the final state and checkpoints directly.
+__device__ __forceinline__ int seg_begin(int s, int nch, int Gn) {
+    return (int)(((int64_t)s * nch) / Gn);
+}
+constexpr uint32_t kEImg = kChunk * kDK * 2;    // E image of one (chunk, head): 16 KiB
+constexpr uint32_t kSinImg = kDV * kDK * 2;     // S_in image of one (segment, head): 32 KiB
+constexpr size_t kStateF32 = (size_t)kDK * kDV;  // one fp32 state, in floats
+
 __global__ void __launch_bounds__(kStateThreads, 1)
 state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_off,
              const int32_t *__restrict__ order, int N, int H,
              const uint8_t *__restrict__ blocks, int64_t max_chunks,
-             const float *S0, float *Sf, __nv_bfloat16 *__restrict__ o, int32_t *status,
-             int ckpt_every, const int32_t *__restrict__ ckpt_off, float *__restrict__ ckpts)
+             const float *S0user, float *Sfuser, __nv_bfloat16 *__restrict__ o, int32_t *status,
+             int ckpt_every, const int32_t *__restrict__ ckpt_off, float *__restrict__ ckpts,
+             int G, float *__restrict__ Sx, float *__restrict__ Mx, uint8_t *__restrict__ Eimg)
 {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
@@ -644,16 +663,30 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
     __shared__ volatile int sAbort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n = order[blockIdx.x / H], h = blockIdx.x % H;
-    const int tbeg = cu[n], tend = cu[n + 1];
-    const int nch = chunk_off[n + 1] - chunk_off[n];
+    const int slots = 2 * G - 1;
+    const int slot = blockIdx.x % slots;
+    const int n = order[(blockIdx.x / slots) / H], h = (blockIdx.x / slots) % H;
+    const int nch_seq = chunk_off[n + 1] - chunk_off[n];
+    const int Gn = min(G, nch_seq);
     const size_t sbase = ((size_t)n * H + h) * kDK * kDV;
 
-    if (nch == 0) {  // empty sequence: the state passes through
-        if (Sf)
-            for (int e = tid; e < kDK * kDV; e += kStateThreads) Sf[sbase + e] = S0 ? S0[sbase + e] : 0.f;
+    if (nch_seq == 0) {  // empty sequence: the state passes through
+        if (Sfuser && slot == 0)
+            for (int e = tid; e < kDK * kDV; e += kStateThreads)
+                Sfuser[sbase + e] = S0user ? S0user[sbase + e] : 0.f;
         return;
     }
+    if (slot >= 2 * Gn - 1) return;  // a segment this short sequence does not have
+    const int seg = (slot + 1) >> 1;
+    const bool xmode = slot > 0 && (slot & 1) == 0;  // transition X of segment seg
+    const int cbeg = seg_begin(seg, nch_seq, Gn);
+    const int nch = seg_begin(seg + 1, nch_seq, Gn) - cbeg;
+    const int tbeg = cu[n] + cbeg * kChunk, tend = cu[n + 1];
+    const float *S0 = slot == 0 ? S0user : nullptr;
+    const size_t xbase = (((size_t)n * G + seg) * H + h) * kStateF32;
+    float *Sf = Gn == 1 ? Sfuser : (xmode ? Mx + xbase : Sx + xbase);
+    const size_t fbase = Gn == 1 ? sbase : 0;  // Sf offset of this (sequence, head)
+    uint8_t *eimg = xmode ? Eimg + ((size_t)h * max_chunks + chunk_off[n] + cbeg) * kEImg : nullptr;
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) { mbar_init(&bars.full[s], 1); mbar_init(&bars.empty[s], kEpi + 1); }
         mbar_init(&bars.mma1, 1);
@@ -673,7 +706,7 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tb = tbase;
-    const uint8_t *blk0 = blocks + ((size_t)h * max_chunks + chunk_off[n]) * kBlockBytes;
+    const uint8_t *blk0 = blocks + ((size_t)h * max_chunks + chunk_off[n] + cbeg) * kBlockBytes;
 
     if (warp == 8) {
         // ---- loader: one bulk copy per chunk block into the stage ring ----
@@ -742,9 +775,11 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
         uint32_t ra[32], rb[32];
         // Initial state: S^T row j = column j of S0 (this half's 64 key channels):
         // fp32 master pre-multiplied by the first chunk's decay, and the bf16 copy.
+        // The transition X starts from the identity: X^T row j = e_j.
         bool ok = true;
         const float *dec0 = nullptr;
-        if (S0) {
+        const bool nonzero0 = S0 || xmode;
+        if (nonzero0) {
             ok = mbar_wait(&bars.full[0], 0, globaltimer_ns() + kWaitNs);
             if (!ok) { record_timeout(status); sAbort = 1; }
             dec0 = (const float *)(sm + kOffDecay);
@@ -753,9 +788,10 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
             const int c0 = 64 * hh + 32 * q2;
             float sv[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sv[i] = S0 ? S0[sbase + (size_t)(c0 + i) * kDV + j] : 0.f;
+            for (int i = 0; i < 32; ++i)
+                sv[i] = S0 ? S0[sbase + (size_t)(c0 + i) * kDV + j] : (xmode && c0 + i == j ? 1.f : 0.f);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ra[i] = __float_as_uint(S0 ? sv[i] * dec0[c0 + i] : 0.f);
+            for (int i = 0; i < 32; ++i) ra[i] = __float_as_uint(nonzero0 ? sv[i] * dec0[c0 + i] : 0.f);
             tmem_st32(tmem_addr(tb, lq, kTS + c0), ra);
             uint32_t sb[16];
 #pragma unroll
@@ -788,8 +824,16 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
                 return;
             }
             const int r = tid >> 2, part = tid & 3;
-            if (r < len) {
-                const uint4 *src = (const uint4 *)(ost + r * kDV + 32 * part);
+            const uint4 *src = (const uint4 *)(ost + r * kDV + 32 * part);
+            if (eimg) {
+                // E rows as the K-major, 128-byte-swizzled A operand of the
+                // correction product (two 64-wide K halves of 64 rows each).
+                uint8_t *dst = eimg + (size_t)cc * kEImg;
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    *(uint4 *)(dst + ((32 * part + 8 * m) >> 6) * 8192 +
+                               sw128_offset(r, (32 * part + 8 * m) & 63, 64)) = src[m];
+            } else if (r < len) {
                 uint4 *dst = (uint4 *)(o + ((size_t)(t0 + r) * H + h) * kDV + 32 * part);
 #pragma unroll
                 for (int m = 0; m < 4; ++m) dst[m] = src[m];
@@ -804,18 +848,25 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
                 record_timeout(status); sAbort = 1; break;
             }
             tc_fence_after_sync();
-            // Dl^T[j][r] = U[r][j] - D1[j][r] for this half's 32 rows -> bf16 pairs into TMEM.
+            // Dl^T[j][r] = U[r][j] - D1[j][r] for this half's 32 rows -> bf16 pairs into TMEM
+            // (U = 0 on the transition).
             {
                 const __nv_bfloat16 *U = (const __nv_bfloat16 *)(st + kOffU);
                 tmem_ld32(tmem_addr(tb, lq, kTD1 + 128 * b + 32 * hh), ra);
                 tmem_ld_wait();
                 uint32_t dl[16];
+                if (xmode) {
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const int r = 32 * hh + i;
-                    const float d0 = __bfloat162float(U[r * kDV + j]) - __uint_as_float(ra[i]);
-                    const float d1v = __bfloat162float(U[(r + 1) * kDV + j]) - __uint_as_float(ra[i + 1]);
-                    dl[i >> 1] = pack_bf16(d0, d1v);
+                    for (int i = 0; i < 32; i += 2)
+                        dl[i >> 1] = pack_bf16(-__uint_as_float(ra[i]), -__uint_as_float(ra[i + 1]));
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const int r = 32 * hh + i;
+                        const float d0 = __bfloat162float(U[r * kDV + j]) - __uint_as_float(ra[i]);
+                        const float d1v = __bfloat162float(U[(r + 1) * kDV + j]) - __uint_as_float(ra[i + 1]);
+                        dl[i >> 1] = pack_bf16(d0, d1v);
+                    }
                 }
                 tmem_st16(tmem_addr(tb, lq, kTDl + 16 * hh), dl);
                 tmem_st_wait();
@@ -850,8 +901,8 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
                 if (Sf) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        Sf[sbase + (size_t)(64 * hh + i) * kDV + j] = __uint_as_float(ra[i]);
-                        Sf[sbase + (size_t)(64 * hh + 32 + i) * kDV + j] = __uint_as_float(rb[i]);
+                        Sf[fbase + (size_t)(64 * hh + i) * kDV + j] = __uint_as_float(ra[i]);
+                        Sf[fbase + (size_t)(64 * hh + 32 + i) * kDV + j] = __uint_as_float(rb[i]);
                     }
                 }
             } else {
@@ -892,6 +943,170 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
     if (warp == 0) tmem_dealloc(tb, 512);
 }
 
+// ---------------------------------------------------------------- compose --
+
+// Affine composition of the segments of one (sequence, head), for 32 value
+// channels per CTA (columns of S never mix):
+//   S_in(1) = S after segment 0,   S_in(s + 1) = M_s S_in(s) + S_loc(s),
+// the final state being S_in(Gn).  The whole scan is in fp32; each S_in(s) is
+// also written as the bf16 B-operand image (row = value channel, K = key
+// channel, 128-byte swizzled) that the correction product reads.
+constexpr int kComposeThreads = 256;
+constexpr int kComposeCols = 32;
+constexpr int kMsLd = kDK + 1;
+constexpr uint32_t kComposeSmem = (kDK * kMsLd + kDK * kComposeCols) * 4;
+
+__global__ void __launch_bounds__(kComposeThreads)
+compose_kernel(const int32_t *__restrict__ chunk_off, int H, int G, const float *__restrict__ Sx,
+               const float *__restrict__ Mx, uint8_t *__restrict__ Simg, float *Sf)
+{
+    extern __shared__ float csm[];
+    float *Ms = csm;                 // M_s [128][129]
+    float *Ss = csm + kDK * kMsLd;   // S_in(s), this CTA's columns [128][32]
+    constexpr int nvb = kDV / kComposeCols;
+    const int vb = blockIdx.x % nvb, h = (blockIdx.x / nvb) % H, n = blockIdx.x / (nvb * H);
+    const int Gn = min(G, chunk_off[n + 1] - chunk_off[n]);
+    if (Gn <= 1) return;             // the state kernel wrote this final state itself
+    const int tid = threadIdx.x;
+    const int m = tid >> 1, cb = (tid & 1) * 16, v0 = vb * kComposeCols;
+    auto xoff = [&](int s) { return (((size_t)n * G + s) * H + h) * kStateF32; };
+
+    for (int e = tid; e < kDK * kComposeCols; e += kComposeThreads)
+        Ss[e] = Sx[xoff(0) + (size_t)(e / kComposeCols) * kDV + v0 + e % kComposeCols];
+    __syncthreads();
+    for (int s = 1; s < Gn; ++s) {
+        uint8_t *img = Simg + (((size_t)n * G + s) * H + h) * kSinImg;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            *(__nv_bfloat16 *)(img + sw128_offset(v0 + cb + i, m, kDV)) =
+                __float2bfloat16_rn(Ss[m * kComposeCols + cb + i]);
+        const float4 *Mg = (const float4 *)(Mx + xoff(s));
+        for (int e = tid; e < kDK * kDK / 4; e += kComposeThreads) {
+            const float4 x = Mg[e];
+            float *d = Ms + (e >> 5) * kMsLd + 4 * (e & 31);
+            d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
+        }
+        __syncthreads();
+        float acc[16];
+        const float *Sl = Sx + xoff(s) + (size_t)m * kDV + v0 + cb;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] = Sl[i];
+        for (int c = 0; c < kDK; ++c) {
+            const float a = Ms[m * kMsLd + c];
+            const float4 *sr = (const float4 *)(Ss + c * kComposeCols + cb);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 x = sr[q];
+                acc[4 * q + 0] = fmaf(a, x.x, acc[4 * q + 0]);
+                acc[4 * q + 1] = fmaf(a, x.y, acc[4 * q + 1]);
+                acc[4 * q + 2] = fmaf(a, x.z, acc[4 * q + 2]);
+                acc[4 * q + 3] = fmaf(a, x.w, acc[4 * q + 3]);
+            }
+        }
+        __syncthreads();             // every read of Ss and Ms is done
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Ss[m * kComposeCols + cb + i] = acc[i];
+        __syncthreads();
+    }
+    if (Sf) {
+        float *d = Sf + ((size_t)n * H + h) * kStateF32 + (size_t)m * kDV + v0 + cb;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) d[i] = Ss[m * kComposeCols + cb + i];
+    }
+}
+
+// ---------------------------------------------------------------- correct --
+
+// Outputs of a chunk in segment s >= 1: o += E S_in(s), one tcgen05 product
+// (M = 64 tokens, N = 128 value channels, K = 128 key channels) per
+// (chunk, head), fp32 in TMEM, added to the bf16 partial output in place.
+constexpr int kCorrThreads = 128;
+constexpr uint32_t kCorrSmem = kEImg + kSinImg + 1024;
+
+__global__ void __launch_bounds__(kCorrThreads)
+correct_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_off, int N, int H,
+               int G, int64_t max_chunks, const uint8_t *__restrict__ Eimg,
+               const uint8_t *__restrict__ Simg, __nv_bfloat16 *__restrict__ o, int32_t *status)
+{
+    const int h = blockIdx.x % H;
+    const int g = blockIdx.x / H;    // global chunk index
+    if (g >= chunk_off[N]) return;
+    const int n = find_seq(chunk_off, N, g);
+    const int nch = chunk_off[n + 1] - chunk_off[n];
+    const int Gn = min(G, nch), c = g - chunk_off[n];
+    if (Gn <= 1) return;
+    int s = 0;
+    while (s + 1 < Gn && seg_begin(s + 1, nch, Gn) <= c) ++s;
+    if (s == 0) return;              // segment 0 started from the true state
+
+    extern __shared__ uint8_t smraw[];
+    uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    __shared__ uint64_t bar_ld, bar_mma;
+    __shared__ uint32_t tbase;
+    __shared__ int sOk;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        mbar_init(&bar_ld, 1);
+        mbar_init(&bar_mma, 1);
+        fence_mbar_init();
+        sOk = 0;
+    }
+    if (warp == 0) { tmem_alloc(&tbase, 128); tmem_relinquish(); }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tb = tbase;
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&bar_ld, kEImg + kSinImg);
+        bulk_g2s(sm, Eimg + ((size_t)h * max_chunks + g) * kEImg, kEImg, &bar_ld);
+        bulk_g2s(sm + kEImg, Simg + (((size_t)n * G + s) * H + h) * kSinImg, kSinImg, &bar_ld);
+        if (mbar_wait(&bar_ld, 0, globaltimer_ns() + kWaitNs)) {
+            tc_fence_after_sync();
+            const uint32_t id = idesc_bf16_f32(64, 128), ea = smem_u32(sm), sa = smem_u32(sm + kEImg);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_ss(tmem_addr(tb, 0, 0), desc_kmajor_sw128(ea + (ks >> 2) * 8192 + (ks & 3) * 32),
+                       desc_kmajor_sw128(sa + (ks >> 2) * 16384 + (ks & 3) * 32), id, ks > 0);
+            mma_commit(&bar_mma);
+            sOk = mbar_wait(&bar_mma, 0, globaltimer_ns() + kWaitNs) ? 1 : 0;
+        } else {
+            // Drain: the copies must land before the CTA's shared memory is released.
+            mbar_wait(&bar_ld, 0, globaltimer_ns() + kWaitNs);
+        }
+        if (!sOk) record_timeout(status);
+    }
+    __syncthreads();
+    if (sOk) {
+        tc_fence_after_sync();
+        const int t0 = cu[n] + c * kChunk, len = min(kChunk, cu[n + 1] - t0);
+        const int r = 16 * warp + lane;  // M = 64: TMEM lane 32 w + i holds row 16 w + i
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+            uint32_t ra[32];
+            tmem_ld32(tmem_addr(tb, 32 * warp, 32 * q), ra);
+            tmem_ld_wait();
+            if (lane < 16 && r < len) {
+                uint4 *d4 = (uint4 *)(o + ((size_t)(t0 + r) * H + h) * kDV + 32 * q);
+#pragma unroll
+                for (int m4 = 0; m4 < 4; ++m4) {
+                    uint4 x = d4[m4];
+                    uint32_t *w = &x.x;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(*(const __nv_bfloat162 *)&w[e]);
+                        w[e] = pack_bf16(f.x + __uint_as_float(ra[8 * m4 + 2 * e]),
+                                         f.y + __uint_as_float(ra[8 * m4 + 2 * e + 1]));
+                    }
+                    d4[m4] = x;
+                }
+            }
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tb, 128);
+}
+
 // cuTensorMapEncodeTiled, fetched from the driver through the runtime (no
 // link-time dependency on libcuda).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
@@ -925,23 +1140,79 @@ bool encode_rows_map(CUtensorMap *map, const void *base, int32_t T, int32_t H)
 
 }  // namespace
 
-size_t tc_workspace_bytes(int32_t total_tokens, int32_t num_seqs, int32_t H)
+namespace {
+
+// SMs the split plan targets: the 148 of a B200.
+constexpr int64_t kSplitSms = 148;
+constexpr int64_t kMaxSegments = 16;
+
+// Workspace layout: plan region, per-(chunk, head) blocks, then (split only)
+// Sx and Mx [N][G][H] fp32 states, S_in images [N][G][H] and E images [H][chunks].
+struct WsLayout {
+    size_t plan, blocks, sx, mx, simg, eimg, total;
+};
+
+WsLayout ws_layout(int32_t total_tokens, int32_t num_seqs, int32_t H, int G)
 {
-    if (num_seqs <= 0) return 0;
+    WsLayout w{};
+    if (num_seqs <= 0) return w;
     const int64_t max_chunks = ((int64_t)total_tokens + 63LL * num_seqs) / kChunk;
-    const size_t plan = (((size_t)(3 * num_seqs + 3) * sizeof(int32_t)) + 1023) & ~(size_t)1023;
-    return plan + (size_t)H * max_chunks * kBlockBytes;
+    auto up = [](size_t x) { return (x + 1023) & ~(size_t)1023; };
+    w.plan = 0;
+    w.blocks = up((size_t)(3 * num_seqs + 3) * sizeof(int32_t));
+    size_t end = w.blocks + (size_t)H * max_chunks * kBlockBytes;
+    if (G > 1) {
+        const size_t states = (size_t)num_seqs * G * H;
+        w.sx = up(end);
+        w.mx = w.sx + states * kStateF32 * sizeof(float);
+        w.simg = w.mx + states * kStateF32 * sizeof(float);
+        w.eimg = w.simg + states * kSinImg;
+        end = w.eimg + (size_t)H * max_chunks * kEImg;
+    }
+    w.total = end;
+    return w;
+}
+
+}  // namespace
+
+int tc_split_segments(int32_t total_tokens, int32_t num_seqs, int32_t H, bool forced)
+{
+    if (num_seqs <= 0 || H <= 0) return 1;
+    const int64_t chains = (int64_t)num_seqs * H;
+    // 2 G - 1 CTAs per (sequence, head) should fit on the SMs at once.
+    int64_t G = (kSplitSms / chains + 1) / 2;
+    if (G > kMaxSegments) G = kMaxSegments;
+    if (!forced) {
+        // Only worth it when every segment keeps at least 16 chunks on average.
+        const int64_t avg_chunks = (int64_t)total_tokens / ((int64_t)kChunk * num_seqs);
+        if (G > avg_chunks / 16) G = avg_chunks / 16;
+    } else if (G < 2) {
+        G = 2;
+    }
+    return G < 2 ? 1 : (int)G;
+}
+
+size_t tc_workspace_bytes(int32_t total_tokens, int32_t num_seqs, int32_t H, int segments)
+{
+    return ws_layout(total_tokens, num_seqs, H, segments).total;
 }
 
 cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream)
 {
     if (a.dk != kDK || a.dv != kDV || !a.bf16) return cudaErrorInvalidValue;
+    const int G = a.segments > 1 ? a.segments : 1;
+    if (G > 1 && a.ckpt_every > 0) return cudaErrorInvalidValue;
     const int64_t max_chunks = ((int64_t)a.total_tokens + 63LL * a.num_seqs) / kChunk;
-    int32_t *chunk_off = (int32_t *)a.workspace;
+    const WsLayout w = ws_layout(a.total_tokens, a.num_seqs, a.H, G);
+    uint8_t *ws = (uint8_t *)a.workspace;
+    int32_t *chunk_off = (int32_t *)ws;
     int32_t *ckpt_off = chunk_off + a.num_seqs + 1;
     int32_t *order = ckpt_off + a.num_seqs + 1;
-    const size_t plan = (((size_t)(3 * a.num_seqs + 3) * sizeof(int32_t)) + 1023) & ~(size_t)1023;
-    uint8_t *blocks = (uint8_t *)a.workspace + plan;
+    uint8_t *blocks = ws + w.blocks;
+    float *Sx = G > 1 ? (float *)(ws + w.sx) : nullptr;
+    float *Mx = G > 1 ? (float *)(ws + w.mx) : nullptr;
+    uint8_t *Simg = G > 1 ? ws + w.simg : nullptr;
+    uint8_t *Eimg = G > 1 ? ws + w.eimg : nullptr;
     cudaError_t err;
 
     err = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -950,6 +1221,14 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
     err = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kStateSmem);
     if (err != cudaSuccess) return err;
+    if (G > 1) {
+        err = cudaFuncSetAttribute(compose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)kComposeSmem);
+        if (err != cudaSuccess) return err;
+        err = cudaFuncSetAttribute(correct_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)kCorrSmem);
+        if (err != cudaSuccess) return err;
+    }
 
     a.mark(0, stream);
     plan_kernel<<<1, kPlanThreads, 0, stream>>>(a.cu_seqlens, a.num_seqs, a.ckpt_every, chunk_off,
@@ -975,10 +1254,25 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
         if (err != cudaSuccess) return err;
     }
     a.mark(2, stream);
-    state_kernel<<<(unsigned)(a.num_seqs * a.H), kStateThreads, kStateSmem, stream>>>(
+    state_kernel<<<(unsigned)((int64_t)a.num_seqs * a.H * (2 * G - 1)), kStateThreads, kStateSmem,
+                   stream>>>(
         a.cu_seqlens, chunk_off, order, a.num_seqs, a.H, blocks, max_chunks, a.initial_state,
-        a.final_state, (__nv_bfloat16 *)a.o, a.status, a.ckpt_every, ckpt_off, a.checkpoints);
+        a.final_state, (__nv_bfloat16 *)a.o, a.status, a.ckpt_every, ckpt_off, a.checkpoints,
+        G, Sx, Mx, Eimg);
     a.mark(3, stream);
+    err = cudaGetLastError();
+    if (err != cudaSuccess || G == 1) return err;
+
+    compose_kernel<<<(unsigned)((int64_t)a.num_seqs * a.H * (kDV / kComposeCols)), kComposeThreads,
+                     kComposeSmem, stream>>>(chunk_off, a.H, G, Sx, Mx, Simg, a.final_state);
+    a.mark(4, stream);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    if (max_chunks > 0)
+        correct_kernel<<<(unsigned)(max_chunks * a.H), kCorrThreads, kCorrSmem, stream>>>(
+            a.cu_seqlens, chunk_off, a.num_seqs, a.H, G, max_chunks, Eimg, Simg,
+            (__nv_bfloat16 *)a.o, a.status);
+    a.mark(5, stream);
     return cudaGetLastError();
 }
 

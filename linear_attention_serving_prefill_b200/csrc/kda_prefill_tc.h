@@ -12,12 +12,19 @@
 
 namespace kda {
 
+// Segments per sequence of the split plan (1 = no split): 2 G - 1 state CTAs
+// per (sequence, head) must fit on the 148 SMs, and, unless `forced`, every
+// segment must keep 16 chunks of 64 tokens on average.  `forced` gives G >= 2.
+int tc_split_segments(int32_t total_tokens, int32_t num_seqs, int32_t H, bool forced);
+
 // Workspace bytes of the tensor-core path: the chunk plan plus one 74,240-byte
 // block of MMA-ready tiles per (chunk, head), for the worst case of
-// floor((T + 63 N) / 64) chunks.
-size_t tc_workspace_bytes(int32_t total_tokens, int32_t num_seqs, int32_t H);
+// floor((T + 63 N) / 64) chunks; with segments > 1 also the segment states,
+// transitions, S_in images (N G H of each) and 16 KiB E images per (chunk, head).
+size_t tc_workspace_bytes(int32_t total_tokens, int32_t num_seqs, int32_t H, int segments);
 
-// Launches plan, intra-chunk and state kernels on `stream`.
+// Launches plan, intra-chunk and state kernels on `stream`, then, when
+// a.segments > 1, the segment composition and the output correction.
 cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream);
 
 }  // namespace kda

@@ -18,7 +18,7 @@ HEADER = os.path.join(ROOT, "include", "kda.h")
 
 OK, INVALID, UNSUPPORTED, WORKSPACE, CUDA = 0, 1, 2, 3, 4
 BF16, F32 = 0, 1
-AUTO, CORE, TC = 0, 1, 2
+AUTO, CORE, TC, SPLIT = 0, 1, 2, 3
 
 
 def declared_functions():
@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_abi_version_and_status_strings():
-    assert B._lib.kda_abi_version() == 1
+    assert B._lib.kda_abi_version() == 2
     for code in range(6):
         s = B.kda_status_string(code)
         assert s.startswith(B.STATUS_NAMES[code])
@@ -78,11 +78,48 @@ def test_prefill_rejects_bad_sizes():
 
 
 def test_kernel_count():
-    assert B._lib.kda_prefill_kernel_count(128, 128, BF16, AUTO) == 3
-    assert B._lib.kda_prefill_kernel_count(128, 128, BF16, CORE) == 1
-    assert B._lib.kda_prefill_kernel_count(64, 64, BF16, AUTO) == 1
-    assert B._lib.kda_prefill_kernel_count(128, 128, F32, AUTO) == 1
-    assert B._lib.kda_prefill_kernel_count(96, 128, BF16, AUTO) == 0
+    kc = B._lib.kda_prefill_kernel_count
+    assert kc(32768, 1, 96, 128, 128, BF16, AUTO) == 3
+    assert kc(4096, 1, 32, 128, 128, BF16, AUTO) == 5      # split: + compose + correct
+    assert kc(4096, 1, 32, 128, 128, BF16, TC) == 3
+    assert kc(4096, 1, 32, 128, 128, BF16, CORE) == 1
+    assert kc(4096, 1, 32, 64, 64, BF16, AUTO) == 1
+    assert kc(4096, 1, 32, 128, 128, F32, AUTO) == 1
+    assert kc(4096, 1, 32, 96, 128, BF16, AUTO) == 0
+    assert kc(4096, 1, 32, 128, 128, F32, SPLIT) == 0
+
+
+def test_split_segment_count():
+    """The split plan: N H (2 G - 1) <= 148 concurrent state chains, G <= 16;
+    AUTO also keeps >= 16 chunks per segment; SPLIT forces G >= 2; other
+    paths never split."""
+    seg = B._lib.kda_prefill_segments
+    assert seg(32768, 1, 96, 128, 128, BF16, AUTO) == 1     # 96 chains already fill the GPU
+    assert seg(4096, 1, 32, 128, 128, BF16, AUTO) == 2      # 3 x 32 = 96 <= 148
+    assert seg(1 << 20, 1, 16, 128, 128, BF16, AUTO) == 5   # 9 x 16 = 144 <= 148
+    assert seg(1 << 20, 1, 1, 128, 128, BF16, AUTO) == 16   # capped
+    assert seg(2048, 1, 1, 128, 128, BF16, AUTO) == 2       # 32 chunks: 2 segments of 16
+    assert seg(1024, 1, 32, 128, 128, BF16, AUTO) == 1      # too short to pay
+    assert seg(1024, 1, 32, 128, 128, BF16, SPLIT) == 2
+    assert seg(32768, 16, 96, 128, 128, BF16, SPLIT) == 2   # forced even when the GPU is full
+    assert seg(4096, 1, 32, 128, 128, BF16, TC) == 1
+    assert seg(4096, 1, 32, 128, 128, F32, AUTO) == 1
+    assert seg(4096, 1, 32, 128, 128, BF16, CORE) == 1
+    assert seg(4096, 1, 32, 64, 64, BF16, SPLIT) == 0       # invalid: split is tensor-core only
+    for G in range(2, 17):
+        assert seg(1 << 24, 1, 148 // (2 * G - 1), 128, 128, BF16, AUTO) >= G
+
+
+def test_split_workspace_holds_the_segment_buffers():
+    ws = B._lib.kda_prefill_workspace_size
+    T, N, H = 4096, 1, 32
+    whole = ws(T, N, H, 128, 128, BF16, TC)
+    split = ws(T, N, H, 128, 128, BF16, SPLIT)
+    # Sx, Mx (fp32 64 KiB), S_in images (32 KiB) per (sequence, segment, head),
+    # E images (16 KiB) per (chunk, head), the first region 1 KiB aligned.
+    extra = N * 2 * H * (2 * 65536 + 32768) + H * (T // 64) * 16384
+    assert split - whole >= extra and split - whole < extra + 1024
+    assert ws(T, N, H, 128, 128, BF16, AUTO) == split
 
 
 def test_prefill_rejects_null_and_misaligned_pointers():
@@ -187,6 +224,10 @@ def test_checkpoint_count_and_validation():
     assert B._lib.kda_prefill_checkpointed(*common, 96, _fake()) == INVALID   # not a multiple of 64
     assert B._lib.kda_prefill_checkpointed(*common, 64, None) == INVALID      # no buffer
     assert B._lib.kda_prefill_checkpointed(*common, 64, _fake(0x10008)) == INVALID  # misaligned
+    split = list(common)
+    split[10:12] = [128, 128]          # dk, dv
+    split[-4] = SPLIT
+    assert B._lib.kda_prefill_checkpointed(*split, 64, _fake()) == UNSUPPORTED
 
 
 def test_decode_multi_rejects_bad_arguments():

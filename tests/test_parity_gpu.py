@@ -17,11 +17,13 @@ from tests.kda_testutil import (TOL_BF16, TOL_F32, gpu_subset, oracle_subset, re
 
 pytestmark = pytest.mark.gpu
 
-PREFILL_ALGOS = ["cuda_core", "tensor_core"]
+# tensor_core_split forces the affine-scan split of every sequence into >= 2
+# segments (one segment per chunk for sequences shorter than that).
+PREFILL_ALGOS = ["cuda_core", "tensor_core", "tensor_core_split"]
 
 
 def _supported(algo, dtype="bf16", dk=128, dv=128):
-    if algo == "tensor_core" and (dtype != "bf16" or dk != 128 or dv != 128):
+    if algo.startswith("tensor_core") and (dtype != "bf16" or dk != 128 or dv != 128):
         pytest.skip("the tensor-core path covers bf16 with dk = dv = 128")
 
 
@@ -169,6 +171,76 @@ def test_outputs_stay_inside_their_buffers(algo):
     assert torch.all(obuf[:guard] == 7.0) and torch.all(obuf[-guard:] == 7.0)
     assert torch.all(sbuf[:guard] == 7.0) and torch.all(sbuf[-guard:] == 7.0)
     _check_all(inp, o, S, TOL_BF16)
+
+
+# ---------------------------------------------------------- sequence split ----
+
+def test_split_long_single_head_sequence_sixteen_segments():
+    """One head, one 3,109-token sequence (49 chunks) cut into 16 segments of 3
+    or 4 chunks with a ragged tail, from a nonzero initial state: outputs and
+    final state against the oracle, and against the unsplit tensor-core path."""
+    L, H = 3109, 1
+    x = _cuda(prefill_inputs([L], H, 128, 128, "bf16", seed=31, s0_std=0.02))
+    assert K.kda_prefill_segments(L, 1, H, 128, 128, torch.bfloat16, "tensor_core_split") == 16
+    assert K.kda_prefill_segments(L, 1, H, 128, 128, torch.bfloat16, "auto") == 3
+    o, S = _run(x, "tensor_core_split")
+    o1, S1 = _run(x, "tensor_core")
+    torch.cuda.synchronize()
+    _check_all(x, o, S, TOL_BF16)
+    assert relerr(to_np(o), to_np(o1)) <= TOL_BF16
+    assert relerr(to_np(S), to_np(S1)) <= TOL_BF16
+
+
+@pytest.mark.parametrize("lengths,H", [([64 * 33], 4), ([130, 64 * 20 + 5, 64], 3), ([63 * 64 + 1], 2)])
+def test_split_segment_boundaries(lengths, H):
+    """Segment edges on and off chunk boundaries, a one-chunk sequence next to
+    split ones, and a one-token last chunk."""
+    x = _cuda(prefill_inputs(lengths, H, 128, 128, "bf16", seed=sum(lengths) + H, s0_std=0.05))
+    o, S = _run(x, "tensor_core_split")
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    _check_all(x, o, S, TOL_BF16)
+
+
+def test_auto_splits_the_4k_single_sequence_and_records_five_kernels():
+    """AUTO picks 2 segments for 32 heads x 4,096 tokens, launches 5 kernels
+    (one event boundary each) and gives the forced split's result bit for bit."""
+    cfg = CONFIGS["prefill_4k"]
+    x = config_inputs(cfg, device="cuda")
+    T = x["q"].shape[0]
+    assert K.kda_prefill_segments(T, 1, cfg.H, 128, 128, torch.bfloat16, "auto") == 2
+    assert K.kda_prefill_kernel_count(T, 1, cfg.H, 128, 128, torch.bfloat16, "auto") == 5
+    assert K.kda_prefill_kernel_count(T, 1, cfg.H, 128, 128, torch.bfloat16, "tensor_core") == 3
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    for e in evs:
+        e.record()  # torch creates the CUDA event at its first record
+    o, S = _run(x, "auto", stage_events=evs)
+    o2, S2 = _run(x, "tensor_core_split")
+    torch.cuda.synchronize()
+    assert all(evs[i].elapsed_time(evs[i + 1]) >= 0 for i in range(5))
+    assert torch.equal(o, o2) and torch.equal(S, S2)
+
+
+def test_auto_with_checkpoints_keeps_sequences_whole():
+    """Checkpoints come from the unsplit chain: AUTO on a split-eligible shape
+    with checkpoints equals the forced unsplit path, and the oracle."""
+    L, H = 64 * 40, 8
+    x = _cuda(prefill_inputs([L], H, 128, 128, "bf16", seed=33, s0_std=0.02))
+    assert K.kda_prefill_segments(L, 1, H, 128, 128, torch.bfloat16, "auto") == 2
+    got = K.kda_prefill_checkpointed(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"],
+                                     x["cu_seqlens"], x["cu_seqlens_host"], 512,
+                                     initial_state=x["initial_state"], algo="auto")
+    ref = K.kda_prefill_checkpointed(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"],
+                                     x["cu_seqlens"], x["cu_seqlens_host"], 512,
+                                     initial_state=x["initial_state"], algo="tensor_core")
+    torch.cuda.synchronize()
+    for a, b in zip(got, ref):
+        assert torch.equal(a, b)
+    _, ref_S, ref_ck = oracle.prefill_checkpoints(
+        x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"], x["cu_seqlens_host"], 512,
+        x["initial_state"])
+    assert relerr(to_np(got[2]), ref_ck) <= TOL_BF16
+    assert relerr(to_np(got[1]), ref_S) <= TOL_BF16
 
 
 # ------------------------------------------------------------------ decode ----
