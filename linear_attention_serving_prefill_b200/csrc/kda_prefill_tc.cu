@@ -71,16 +71,26 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 // ------------------------------------------------------------------- plan --
 
+__device__ __forceinline__ int find_seq(const int32_t *chunk_off, int N, int g) {
+    int lo = 0, hi = N - 1;  // largest n with chunk_off[n] <= g
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (chunk_off[mid] <= g) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
 // chunk_off[n] = sum_{m<n} ceil(L_m / 64); chunk_off[N] = total chunks.
 // ckpt_off[n] = sum_{m<n} L_m / every (checkpoint rows), when every > 0.
 // order[i] = sequence index with the i-th largest length (ties by index)
 // when N <= kMaxSorted, else the identity.
+// chunk_loc[g] = (first token, length) of global chunk g.
 constexpr int kPlanThreads = 1024;
 constexpr int kMaxSorted = 4096;
 
 __global__ void __launch_bounds__(kPlanThreads)
 plan_kernel(const int32_t *__restrict__ cu, int N, int every, int32_t *__restrict__ chunk_off,
-            int32_t *__restrict__ ckpt_off, int32_t *__restrict__ order)
+            int32_t *__restrict__ ckpt_off, int32_t *__restrict__ order, int2 *__restrict__ chunk_loc)
 {
     __shared__ int32_t part[2][kPlanThreads];
     const int tid = threadIdx.x;
@@ -115,6 +125,13 @@ plan_kernel(const int32_t *__restrict__ cu, int N, int every, int32_t *__restric
         chunk_off[N] = part[0][tid];
         ckpt_off[N] = part[1][tid];
     }
+    __syncthreads();  // chunk_off is complete
+    const int total = part[0][kPlanThreads - 1];
+    for (int g = tid; g < total; g += kPlanThreads) {
+        const int n = find_seq(chunk_off, N, g);
+        const int t0 = cu[n] + (g - chunk_off[n]) * kChunk;
+        chunk_loc[g] = make_int2(t0, min(kChunk, cu[n + 1] - t0));
+    }
     for (int n = tid; n < N; n += kPlanThreads) {
         int rank = n;
         if (N <= kMaxSorted) {
@@ -131,50 +148,53 @@ plan_kernel(const int32_t *__restrict__ cu, int N, int every, int32_t *__restric
 
 // ------------------------------------------------------------------ intra --
 
-// Persistent: one CTA per SM walks (chunk, head) items b, b + gridDim.x, ...;
-// item w is chunk w / H of head w % H.  While an item is computed, warp 0
-// prefetches the next item's raw k, q, v, z rows (256 B each) into the other
-// stage of a two-stage ring with bulk copies, and its beta values with
-// cp.async.  Thread (cp, q8) owns channels 2 cp, 2 cp + 1 of the eight rows
-// 8 q8 .. 8 q8 + 7 (q8 = warp / 2), inside sub-tile I = q8 / 2, so the
-// sub-tile index is uniform across a warp.
-constexpr int kIntraCompute = 512;
-constexpr int kIntraThreads = kIntraCompute;
+// Persistent, two CTAs of 256 threads per SM, each walking (chunk, head) items
+// b, b + gridDim.x, ...; item w is chunk w / H of head w % H.  A CTA holds one
+// item at a time; the SM's other CTA overlaps its waits (loads, products,
+// barriers).  Thread (cp, I) owns channels 2 cp, 2 cp + 1 of the 16 rows of
+// sub-tile I = warp / 2, so the sub-tile index is uniform across a warp.
+constexpr int kIntraThreads = 256;
 constexpr uint32_t kRawTile = kChunk * kDK * 2;    // one [64][128] bf16 tile, 16 KiB
-constexpr uint32_t kRawStage = 4 * kRawTile;       // k, q, v, z
+// Shared memory (offsets from a 1024-aligned base).  The raw k, q, v, z tiles
+// arrive by two 128-byte-swizzled TMA boxes each, as K-major operand images
+// [K half][64 rows][128 B]: element (r, c) at sw128_offset(r, c, 64).
 constexpr uint32_t kRawK = 0, kRawQ = kRawTile, kRawV = 2 * kRawTile, kRawZ = 3 * kRawTile;
-// Shared memory (offsets from a 1024-aligned base).
-constexpr uint32_t kIRaw = 0;                      // 2 raw stages
 // A operands of the A/P products, R^(I) = k e^{m_I - G} scaled to sub-tile I's
-// reference, stacked in pairs for M = 128 products: pair p holds R^(2p+1) in rows
-// 0..63 and R^(2p) in rows 64..127, one 128-row x 128-byte sub-block per 64-wide
-// K half.  Rows that are never valid (R^(I) beyond row 16 I + 15) sit at the ends
-// of some sub-blocks, so the next buffer starts inside that tail: the product
-// reads whatever is there into rows it discards, and nobody writes them.
-constexpr uint32_t kIRbig = 2 * kRawStage;
-__host__ __device__ constexpr uint32_t r_sub(int p, int kb) {
-    return p == 0 ? (kb == 0 ? 0u : 10240u) : (kb == 0 ? 20480u : 34816u);
+// reference: one 64-row image per (sub-tile I, K half), of which only rows
+// 0 .. 16 I + 15 are valid.  Each region starts where the previous region's
+// valid rows end; a product reads the rows past them (the next regions, or the
+// end of the area) into outputs it discards.  Valid bytes of (I, kb): 2048 (I + 1).
+constexpr uint32_t kIR = 4 * kRawTile;
+__host__ __device__ constexpr uint32_t r_region(int I, int kb) {
+    return kIR + 2048u * (uint32_t)(I * (I + 1) + kb * (I + 1));
 }
-constexpr uint32_t kIKQ = kIRbig + 49152;          // [Kt_I; Qt_I] per sub-tile, then [bK e^G; bV]^T
-constexpr uint32_t kISmem = kIKQ + 32768;
-// Reused inside Rbig once the A/P products are read back:
-constexpr uint32_t kIAf = kIRbig;                  // fp32 A [64][65]
-constexpr uint32_t kITf = kIRbig + 16640;          // fp32 T [64][65]
-constexpr uint32_t kIXf = kIRbig + 33280;          // fp32 scratch [32][33]
-constexpr int kLd = 65;
-// Row block of sub-tile I inside its pair: 0 for the odd tile, 64 for the even one.
-__host__ __device__ constexpr int pair_slot_row(int I) { return (I & 1) ? 0 : 64; }
+constexpr uint32_t kISmem = kIR + 40960;           // 104 KiB
+// Reused inside the R area once the A/P products are read back:
+// (rows padded to 68 and 36 floats: 16-byte aligned for vector loads)
+constexpr int kLd = 68, kXLd = 36;
+constexpr uint32_t kIAf = kIR;                     // fp32 A [64][68]
+constexpr uint32_t kITf = kIR + 64 * kLd * 4;      // fp32 T [64][68]
+constexpr uint32_t kIXf = kIR + 128 * kLd * 4;     // fp32 scratch [32][36]
+static_assert(kIXf + 32 * kXLd * 4 <= kIR + 40960, "inverse scratch exceeds the R area");
+// Later uses of the raw tiles within an item:
+//   k tile: K e^{L} (in place) -> T as bf16 operand of the W/U product (first
+//           8 KiB) and the P staging for its bulk store (second 8 KiB);
+//   q tile: Q e^{L} (in place) -> (K e^{G_C - G})^T staging for its bulk store;
+//   v, z tiles: [beta K e^G ; beta V]^T, the B operand of the W/U product.
+// Once the W/U product completes no tile is read any more, so the next item's
+// loads are issued then and overlap the W/U readback (which writes W and U to
+// the block straight from registers).
 
 struct IntraItem { int t0, len, g, h; };
 
-// One 3-D tile load: the box {128 channels, 1 head, 64 tokens} at (0, h, t0)
-// of a [T][H][128] bf16 tensor; rows past T arrive as zeros.
-__device__ __forceinline__ void tma_rows(void *smem_dst, const CUtensorMap *map, int h, int t0,
-                                         uint64_t *bar) {
+// One 3-D tile load: the box {64 channels, 1 head, 64 tokens} at (x, h, t0) of a
+// [T][H][128] bf16 tensor, 128-byte swizzled; rows past T arrive as zeros.
+__device__ __forceinline__ void tma_rows(void *smem_dst, const CUtensorMap *map, int x, int h,
+                                         int t0, uint64_t *bar) {
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3, %4}], [%5];"
-        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(h), "r"(t0),
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(h), "r"(t0),
           "r"(smem_u32(bar))
         : "memory");
 }
@@ -185,17 +205,12 @@ __device__ __forceinline__ void cp_async_4(void *smem_dst, const void *gmem_src)
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
                  : "memory");
 }
+__device__ __forceinline__ void cp_async_8(void *smem_dst, const void *gmem_src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
-__device__ __forceinline__ int find_seq(const int32_t *chunk_off, int N, int g) {
-    int lo = 0, hi = N - 1;  // largest n with chunk_off[n] <= g
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (chunk_off[mid] <= g) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-}
 
 __device__ __forceinline__ float2 ld_bf16x2_smem(const uint8_t *base, uint32_t off) {
     return __bfloat1622float2(*(const __nv_bfloat162 *)(base + off));
@@ -212,28 +227,31 @@ __device__ __forceinline__ float gate_log_decay_fast(float expA, float z) {
     return __fdividef(kGMin, 1.0f + __expf(-expA * z));
 }
 
-__global__ void __launch_bounds__(kIntraThreads, 1)
+__global__ void __launch_bounds__(kIntraThreads, 2)
 intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_z,
              const float *__restrict__ A, const float *__restrict__ beta,
-             const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_off, int N, int H,
+             const int2 *__restrict__ chunk_loc, const int32_t *__restrict__ chunk_off, int N, int H,
              uint8_t *__restrict__ blocks, int64_t max_chunks, int32_t *status)
 {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t full[2], mma_bar;
+    __shared__ uint64_t full, mma_bar, ap_bar;
     __shared__ uint32_t tbase;
-    __shared__ IntraItem info[2];
-    __shared__ float sBeta[2][kChunk];
-    __shared__ float sTot[8][kDK];
+    __shared__ IntraItem info;
+    __shared__ int2 next_loc;
+    __shared__ float sBeta[kChunk];
+    __shared__ float sA[kDK];
+    __shared__ float sTot[4][kDK];
     __shared__ volatile int sAbort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int total_items = chunk_off[N] * H;
     if ((int)blockIdx.x >= total_items) return;
     if (tid == 0) {
-        for (int s = 0; s < 2; ++s) mbar_init(&full[s], 1);
+        mbar_init(&full, 1);
         mbar_init(&mma_bar, 1);
+        mbar_init(&ap_bar, 4);   // one commit per sub-tile's issuing warp
         fence_mbar_init();
         sAbort = 0;
     }
@@ -243,82 +261,84 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     tc_fence_after_sync();
     const uint32_t tb = tbase;
 
-    // Warp 0: request item wn into stage sn (raw rows by bulk copy, beta by cp.async).
-    auto issue = [&](int wn, int sn) {
+    // Where item wn lives (one load of the plan's chunk table).
+    auto locate = [&](int wn) {
         const int g = wn / H, h = wn % H;
-        const int n = find_seq(chunk_off, N, g);
-        const int t0 = cu[n] + (g - chunk_off[n]) * kChunk;
-        const int len = min(kChunk, cu[n + 1] - t0);
+        const int2 loc = chunk_loc[g];
+        return IntraItem{loc.x, loc.y, g, h};
+    };
+    // Warp 0: request item `nx` (raw rows by eight TMA boxes, beta and A by
+    // cp.async).  Called once the previous item reads no raw tile, beta or A.
+    auto issue = [&](const IntraItem &nx) {
         for (int r = lane; r < kChunk; r += 32) {
-            if (r < len) cp_async_4(&sBeta[sn][r], beta + (size_t)(t0 + r) * H + h);
-            else sBeta[sn][r] = 0.f;
+            if (r < nx.len) cp_async_4(&sBeta[r], beta + (size_t)(nx.t0 + r) * H + nx.h);
+            else sBeta[r] = 0.f;
         }
+        for (int c = lane; c < kDK; c += 32) cp_async_4(&sA[c], A + (size_t)nx.h * kDK + c);
         cp_async_commit();
         if (lane == 0) {
-            // The stage's previous item staged W, U and Kd^T in it for bulk stores:
-            // all but the newest bulk group (this item's Kd^T) have finished reading.
-            bulk_wait_read<1>();
-            info[sn] = IntraItem{t0, len, g, h};
-            mbar_arrive_expect_tx(&full[sn], kRawStage);
-            uint8_t *stn = sm + kIRaw + sn * kRawStage;
-            tma_rows(stn + kRawK, &tm_k, h, t0, &full[sn]);
-            tma_rows(stn + kRawQ, &tm_q, h, t0, &full[sn]);
-            tma_rows(stn + kRawV, &tm_v, h, t0, &full[sn]);
-            tma_rows(stn + kRawZ, &tm_z, h, t0, &full[sn]);
+            info = nx;
+            mbar_arrive_expect_tx(&full, 4 * kRawTile);
+            const CUtensorMap *maps[4] = {&tm_k, &tm_q, &tm_v, &tm_z};
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                tma_rows(sm + m * kRawTile, maps[m], 0, nx.h, nx.t0, &full);
+                tma_rows(sm + m * kRawTile + 8192, maps[m], 64, nx.h, nx.t0, &full);
+            }
         }
         __syncwarp();
     };
-    if (warp == 0) issue(blockIdx.x, 0);
+    if (warp == 0) issue(locate(blockIdx.x));
     int issued = 1;  // items requested so far (meaningful in warp 0)
 
     {
-        // Thread (cp, q8): channels c0 = 2 cp and c0 + 1, rows 8 q8 .. 8 q8 + 7, sub-tile I.
-        const int cp = ((warp & 1) << 5) | lane, c0 = 2 * cp, q8 = warp >> 1, I = q8 >> 1;
+        const int cp = ((warp & 1) << 5) | lane, c0 = 2 * cp, I = warp >> 1;
+        float *Af = (float *)(sm + kIAf), *Tf = (float *)(sm + kITf), *Xf = (float *)(sm + kIXf);
         uint32_t mma_count = 0;
+        int mma_failed = -1, ap_failed = -1;  // parity of a product wait that gave up
         int it = 0;
         for (int w = blockIdx.x; w < total_items && !sAbort; w += gridDim.x, ++it) {
-            const int s = it & 1;
-            if (warp == 0) cp_async_wait_all();  // this item's beta values (issued one item ago)
-            if (!mbar_wait(&full[s], (it >> 1) & 1, globaltimer_ns() + kWaitNs)) {
+            if (warp == 0) cp_async_wait_all();  // this item's beta and A values
+            if (!mbar_wait(&full, it & 1, globaltimer_ns() + kWaitNs)) {
                 if (tid == 0) record_timeout(status);
                 sAbort = 1;
-                break;
             }
-            const IntraItem inf = info[s];
+            compute_sync();  // beta and A (landed by warp 0's cp.async) are visible
+            const IntraItem inf = info;
             const int len = inf.len, h = inf.h;
-            const uint8_t *st = sm + kIRaw + s * kRawStage;
             uint8_t *blk = blocks + ((size_t)h * max_chunks + inf.g) * kBlockBytes;
-            const float2 eA = make_float2(__expf(A[(size_t)h * kDK + c0]), __expf(A[(size_t)h * kDK + c0 + 1]));
+            const float2 eA = make_float2(__expf(sA[c0]), __expf(sA[c0 + 1]));
+            const bool has_next = w + (int)gridDim.x < total_items;
+            // The next item's chunk-table entry, fetched asynchronously for issue().
+            if (tid == 0 && has_next) {
+                cp_async_8(&next_loc, chunk_loc + (w + gridDim.x) / H);
+                cp_async_commit();
+            }
 
             // Pass 1: gate and cumulative log-decay of channels c0, c0 + 1 over the
-            // eight rows, then relative to the sub-tile start: L_r = G_r - m_I.
-            float2 L[8];
+            // sub-tile's 16 rows, relative to its start: L_r = G_r - m_I.
+            float2 L[16];
             float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int r = 8 * q8 + i;
+            for (int i = 0; i < 16; ++i) {
+                const int r = 16 * I + i;
                 if (r < len) {
-                    const float2 zz = ld_bf16x2_smem(st, kRawZ + r * 256 + 4 * cp);
+                    const float2 zz = ld_bf16x2_smem(sm, kRawZ + sw128_offset(r, c0, 64));
                     acc.x += gate_log_decay_fast(eA.x, zz.x);
                     acc.y += gate_log_decay_fast(eA.y, zz.y);
                 }
                 L[i] = acc;
             }
-            sTot[q8][c0] = acc.x;
-            sTot[q8][c0 + 1] = acc.y;
+            sTot[I][c0] = acc.x;
+            sTot[I][c0 + 1] = acc.y;
             compute_sync();
-            if (q8 & 1) {
-                const float ox = sTot[q8 - 1][c0], oy = sTot[q8 - 1][c0 + 1];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) { L[i].x += ox; L[i].y += oy; }
-            }
+            if (sAbort) break;
             // Sub-tile references m_J = G at the end of sub-tile J - 1 (m_0 = 0), G_C.
             float2 mref[5];
             mref[0] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int J = 0; J < 4; ++J)
-                mref[J + 1] = make_float2(mref[J].x + sTot[2 * J][c0] + sTot[2 * J + 1][c0],
-                                          mref[J].y + sTot[2 * J][c0 + 1] + sTot[2 * J + 1][c0 + 1]);
+                mref[J + 1] = make_float2(mref[J].x + sTot[J][c0], mref[J].y + sTot[J][c0 + 1]);
             const float2 mI = I == 0 ? mref[0] : I == 1 ? mref[1] : I == 2 ? mref[2] : mref[3];
             const float2 GC = mref[4];
             const float2 emI = make_float2(__expf(mI.x), __expf(mI.y));
@@ -331,29 +351,30 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 fac[Ip] = Ip > I ? make_float2(__expf(mref[Ip].x - mI.x), __expf(mref[Ip].y - mI.y))
                                  : make_float2(1.f, 1.f);
 
-            // Pass 2: scaled operands of channels c0, c0 + 1 for the eight rows.
-            uint8_t *sR = sm + kIRbig, *sKQ = sm + kIKQ;
-            uint32_t pk0[4], pk1[4], pv0[4], pv1[4], kd0[4], kd1[4];
+            // Pass 2: scaled operands of channels c0, c0 + 1 for the 16 rows.
+            // Kt = k e^{L} and Qt = q e^{L} replace k and q in place (same thread,
+            // same address); the rest goes to R, to the block, or into registers.
+            // beta K e^G, beta V and K e^{G_C - G} wait in registers until the tiles
+            // that receive them are no longer read.
+            uint32_t pk0[8], pk1[8], pv0[8], pv1[8], kd0[8], kd1[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int r = 8 * q8 + i, ri = r & 15;
+            for (int i = 0; i < 16; ++i) {
+                const int r = 16 * I + i;
                 const bool valid = r < len;
-                const float2 kv = valid ? ld_bf16x2_smem(st, kRawK + r * 256 + 4 * cp) : make_float2(0.f, 0.f);
-                const float2 qv = valid ? ld_bf16x2_smem(st, kRawQ + r * 256 + 4 * cp) : make_float2(0.f, 0.f);
-                const float2 vv = valid ? ld_bf16x2_smem(st, kRawV + r * 256 + 4 * cp) : make_float2(0.f, 0.f);
+                const uint32_t off = sw128_offset(r, c0, 64);
+                const float2 kv = valid ? ld_bf16x2_smem(sm, kRawK + off) : make_float2(0.f, 0.f);
+                const float2 qv = valid ? ld_bf16x2_smem(sm, kRawQ + off) : make_float2(0.f, 0.f);
+                const float2 vv = valid ? ld_bf16x2_smem(sm, kRawV + off) : make_float2(0.f, 0.f);
                 const float2 e1 = make_float2(__expf(L[i].x), __expf(L[i].y));    // in [e^-80, 1]
                 const float2 e2 = make_float2(__expf(-L[i].x), __expf(-L[i].y));  // in [1, e^80]
-                const float br = sBeta[s][r];
-                // B rows of pair I / 2: [Kt_odd; Qt_odd; Kt_even; Qt_even], 16 rows each.
-                const int brow = 64 * (I >> 1) + ((I & 1) ? 0 : 32) + ri;
-                *(uint32_t *)(sKQ + sw128_offset(brow, c0, 128)) = pack_bf16(kv.x * e1.x, kv.y * e1.y);
-                *(uint32_t *)(sKQ + sw128_offset(brow + 16, c0, 128)) = pack_bf16(qv.x * e1.x, qv.y * e1.y);
+                const float br = sBeta[r];
+                *(uint32_t *)(sm + kRawK + off) = pack_bf16(kv.x * e1.x, kv.y * e1.y);
+                *(uint32_t *)(sm + kRawQ + off) = pack_bf16(qv.x * e1.x, qv.y * e1.y);
                 const float2 kb = make_float2(kv.x * e2.x, kv.y * e2.y);
 #pragma unroll
                 for (int Ip = 0; Ip < 4; ++Ip)
                     if (Ip >= I)
-                        *(uint32_t *)(sR + r_sub(Ip >> 1, c0 >> 6) +
-                                      sw128_offset(pair_slot_row(Ip) + r, c0 & 63, 128)) =
+                        *(uint32_t *)(sm + r_region(Ip, c0 >> 6) + sw128_offset(r, c0 & 63, 64)) =
                             pack_bf16(kb.x * fac[Ip].x, kb.y * fac[Ip].y);
                 *(uint32_t *)(blk + kOffWQ + sw128_offset(64 + r, c0, 128)) =
                     pack_bf16(qv.x * e1.x * emI.x, qv.y * e1.y * emI.y);
@@ -369,88 +390,100 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                     kd0[i >> 1] |= hd0 << 16; kd1[i >> 1] |= hd1 << 16;
                 }
             }
-            // (K e^{G_C - G})^T is staged in the item's raw z tile (dead after pass 1)
-            // as the exact image of its block region, then bulk-stored.
-            uint8_t *stw = sm + kIRaw + s * kRawStage;
-            *(uint4 *)(stw + kRawZ + sw128_offset(c0, 8 * q8, 128)) = make_uint4(kd0[0], kd0[1], kd0[2], kd0[3]);
-            *(uint4 *)(stw + kRawZ + sw128_offset(c0 + 1, 8 * q8, 128)) = make_uint4(kd1[0], kd1[1], kd1[2], kd1[3]);
-            if (q8 == 0) {
+            if (I == 0) {
                 ((float *)(blk + kOffDecay))[c0] = __expf(GC.x);
                 ((float *)(blk + kOffDecay))[c0 + 1] = __expf(GC.y);
             }
 
-            // A/P products: D[s][32 I + j] = R^(I)_s . Kt_{16I+j} (j < 16) and . Qt (j >= 16).
+            // A/P products, per sub-tile I (M = 64 rows s of R^(I), N = 16 + 16):
+            // D[s][32 I + j] = R^(I)_s . Kt_{16 I + j},  D[s][32 I + 16 + j] = R^(I)_s . Qt_{16 I + j}.
             fence_proxy_async_smem();
             tc_fence_before_sync();
             compute_sync();
             tc_fence_after_sync();
-            if (tid == 0) {
-                bulk_s2g(blk + kOffKd, stw + kRawZ, 16384);
-                bulk_commit();
-                // Pair p: D[:, 64p .. 64p+63] = [R^(2p+1); R^(2p)] [B_(2p+1); B_(2p)]^T
-                // (M = 128, N = 64); the wanted blocks are rows 0..63 x columns 0..31
-                // and rows 64..127 x columns 32..63.
-                const uint32_t id = idesc_bf16_f32(128, 64);
+            if (warp < 4 && lane == 0) {
+                // Lane 0 of warp Ib issues sub-tile Ib's 16 products (the four warps
+                // sit on different schedulers), then commits them to ap_bar.
+                const int Ib = warp;
+                const uint32_t id = idesc_bf16_f32(64, 16), base = smem_u32(sm);
 #pragma unroll
-                for (int pp = 0; pp < 2; ++pp)
+                for (int part = 0; part < 2; ++part)
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t kb2 = ks >> 2, kin = ks & 3;
-                        const uint32_t a = smem_u32(sR) + r_sub(pp, kb2) + kin * 32;
-                        const uint32_t b = smem_u32(sKQ) + kb2 * 128 * 128 + 64 * pp * 128 + kin * 32;
-                        mma_ss(tmem_addr(tb, 0, 64 * pp), desc_kmajor_sw128(a), desc_kmajor_sw128(b), id, ks > 0);
+                        const uint32_t a = base + r_region(Ib, ks >> 2) + (ks & 3) * 32;
+                        const uint32_t b = base + (part ? kRawQ : kRawK) + (ks >> 2) * 8192 +
+                                           16 * Ib * 128 + (ks & 3) * 32;
+                        mma_ss(tmem_addr(tb, 0, 32 * Ib + 16 * part), desc_kmajor_sw128(a),
+                               desc_kmajor_sw128(b), id, ks > 0);
                     }
-                mma_commit(&mma_bar);
+                mma_commit(&ap_bar);
             }
-            // While the products run, warp 0 requests the next item into the other
-            // stage (free: its previous item finished with it).
-            if (warp == 0 && w + (int)gridDim.x < total_items) {
-                issue(w + gridDim.x, s ^ 1);
-                issued = it + 2;
+            // Meanwhile: [beta K e^G ; beta V]^T (rows = channels, K = tokens), the
+            // B operand of the W/U product, into the v and z tiles (no longer read).
+#pragma unroll
+            for (int hlf = 0; hlf < 2; ++hlf) {
+                const int kk = 16 * I + 8 * hlf;
+                *(uint4 *)(sm + kRawV + sw128_offset(c0, kk, 128)) =
+                    make_uint4(pk0[4 * hlf], pk0[4 * hlf + 1], pk0[4 * hlf + 2], pk0[4 * hlf + 3]);
+                *(uint4 *)(sm + kRawV + sw128_offset(c0 + 1, kk, 128)) =
+                    make_uint4(pk1[4 * hlf], pk1[4 * hlf + 1], pk1[4 * hlf + 2], pk1[4 * hlf + 3]);
+                *(uint4 *)(sm + kRawZ + sw128_offset(c0, kk, 128)) =
+                    make_uint4(pv0[4 * hlf], pv0[4 * hlf + 1], pv0[4 * hlf + 2], pv0[4 * hlf + 3]);
+                *(uint4 *)(sm + kRawZ + sw128_offset(c0 + 1, kk, 128)) =
+                    make_uint4(pv1[4 * hlf], pv1[4 * hlf + 1], pv1[4 * hlf + 2], pv1[4 * hlf + 3]);
             }
-            if (!mbar_wait(&mma_bar, mma_count & 1, globaltimer_ns() + kWaitNs)) {
+            if (!mbar_wait(&ap_bar, it & 1, globaltimer_ns() + kWaitNs)) {
                 if (tid == 0) record_timeout(status);
                 sAbort = 1;
-                break;
+                ap_failed = it & 1;
             }
-            ++mma_count;
             tc_fence_after_sync();
-
-            float *Af = (float *)(sm + kIAf), *Tf = (float *)(sm + kITf), *Xf = (float *)(sm + kIXf);
             {
-                // M = 128 layout: TMEM lane = A row.  Warps 0-7: pair p = warp / 4,
-                // lane quarter q = warp % 4; quarters 0-1 hold R^(2p+1) rows (wanted
-                // columns 0..31 of the pair), quarters 2-3 hold R^(2p) rows (32..63).
-                if (warp < 8) {
-                    uint32_t rr[32];
-                    const int q = warp & 3, pp = warp >> 2, slot = q >> 1;
-                    const int sidx = 32 * (q & 1) + lane, Ia = slot ? 2 * pp : 2 * pp + 1;
-                    tmem_ld32(tmem_addr(tb, 32 * q, 64 * pp + 32 * slot), rr);
-                    tmem_ld_wait();
+                // M = 64 layout: TMEM lane 32 q + i holds row 16 q + i (i < 16).  Warp w:
+                // lane quarter q = w % 4, sub-tiles 2 (w / 4) and 2 (w / 4) + 1.
+                const int q = warp & 3, hb = warp >> 2;
 #pragma unroll
-                    for (int jr = 0; jr < 16; ++jr) {
-                        const int r = 16 * Ia + jr;
-                        Af[r * kLd + sidx] = sidx < r ? sBeta[s][r] * __uint_as_float(rr[jr]) : 0.f;
-                        const float pvv = sidx <= r ? __uint_as_float(rr[16 + jr]) : 0.f;
-                        *(__nv_bfloat16 *)(blk + kOffP + sw128_offset(r, sidx, 64)) = __float2bfloat16_rn(pvv);
+                for (int u = 0; u < 2; ++u) {
+                    const int Ia = 2 * hb + u;
+                    uint32_t rr[32];
+                    tmem_ld32(tmem_addr(tb, 32 * q, 32 * Ia), rr);
+                    tmem_ld_wait();
+                    if (lane < 16) {
+                        const int sidx = 16 * q + lane;
+#pragma unroll
+                        for (int jr = 0; jr < 16; ++jr) {
+                            const int r = 16 * Ia + jr;
+                            Af[r * kLd + sidx] = sidx < r ? sBeta[r] * __uint_as_float(rr[jr]) : 0.f;
+                            const float pvv = sidx <= r ? __uint_as_float(rr[16 + jr]) : 0.f;
+                            *(__nv_bfloat16 *)(sm + kRawK + 8192 + sw128_offset(r, sidx, 64)) =
+                                __float2bfloat16_rn(pvv);
+                        }
                     }
                 }
             }
-            // [beta K e^G ; beta V]^T (256 rows x 64 tokens) into the freed [Kt; Qt] region.
-            *(uint4 *)(sKQ + sw128_offset(c0, 8 * q8, 256)) = make_uint4(pk0[0], pk0[1], pk0[2], pk0[3]);
-            *(uint4 *)(sKQ + sw128_offset(c0 + 1, 8 * q8, 256)) = make_uint4(pk1[0], pk1[1], pk1[2], pk1[3]);
-            *(uint4 *)(sKQ + sw128_offset(128 + c0, 8 * q8, 256)) = make_uint4(pv0[0], pv0[1], pv0[2], pv0[3]);
-            *(uint4 *)(sKQ + sw128_offset(128 + c0 + 1, 8 * q8, 256)) = make_uint4(pv1[0], pv1[1], pv1[2], pv1[3]);
+            // (K e^{G_C - G})^T staged in the q tile (Qt is no longer read) as the
+            // exact image of its block region, then bulk-stored with P.
+            *(uint4 *)(sm + kRawQ + sw128_offset(c0, 16 * I, 128)) = make_uint4(kd0[0], kd0[1], kd0[2], kd0[3]);
+            *(uint4 *)(sm + kRawQ + sw128_offset(c0, 16 * I + 8, 128)) = make_uint4(kd0[4], kd0[5], kd0[6], kd0[7]);
+            *(uint4 *)(sm + kRawQ + sw128_offset(c0 + 1, 16 * I, 128)) = make_uint4(kd1[0], kd1[1], kd1[2], kd1[3]);
+            *(uint4 *)(sm + kRawQ + sw128_offset(c0 + 1, 16 * I + 8, 128)) = make_uint4(kd1[4], kd1[5], kd1[6], kd1[7]);
+            fence_proxy_async_smem();
             tc_fence_before_sync();
             compute_sync();
+            if (sAbort) break;
+            if (tid == 0) {
+                bulk_s2g(blk + kOffKd, sm + kRawQ, 16384);
+                bulk_s2g(blk + kOffP, sm + kRawK + 8192, 8192);
+                bulk_commit();
+            }
 
-            // T, rounded to bf16, is also the A operand of the W/U product
-            // (64 rows x 64 K), written into the item's raw k tile as it is formed.
-            uint8_t *sT = stw + kRawK;
             // T = (I + A)^-1 by blocks of 16: diagonal blocks by forward
             // substitution, then T_ij = -T_ii A_ij T_jj doubled from 16 to 32 to 64.
             // Only the lower triangle is used; the two upper blocks that the
-            // doubling products read, (0,1) and (2,3), are set to zero.
+            // doubling products read, (0,1) and (2,3), are set to zero.  T, rounded
+            // to bf16, is also the A operand of the W/U product (64 rows x 64 K),
+            // written into the k tile as it is formed.
+            uint8_t *sT = sm + kRawK;
             if (tid < 64) {
                 const int Ib = tid >> 4, jc = tid & 15, o = 16 * Ib;
                 float col[16];
@@ -468,12 +501,12 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 }
             } else {
                 const int e = tid - 64;  // the other threads zero the upper blocks
-                for (int f = e; f < 512; f += kIntraCompute - 64) {
+                for (int f = e; f < 512; f += kIntraThreads - 64) {
                     const int blkz = f >> 8, r = (f >> 4) & 15, cz = f & 15;
                     const int ro = 32 * blkz, co = 32 * blkz + 16;
                     Tf[(ro + r) * kLd + co + cz] = 0.f;   // read by the doubling products
                 }
-                for (int f = e; f < 6 * 256; f += kIntraCompute - 64) {
+                for (int f = e; f < 6 * 256; f += kIntraThreads - 64) {
                     const int bz = f >> 8, r = (f >> 4) & 15, cz = f & 15;
                     // upper blocks (0,1) (0,2) (0,3) (1,2) (1,3) (2,3) of the bf16 operand
                     const int bi = bz < 3 ? 0 : bz < 5 ? 1 : 2;
@@ -483,94 +516,96 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             }
             compute_sync();
             {
-                // Level 1, blocks (1,0) and (3,2): X = A_ij T_jj, one output per thread.
-                const int p = tid >> 8, r = (tid >> 4) & 15, sb = tid & 15;
+                // Level 1, blocks (1,0) and (3,2): X = A_ij T_jj, columns 2 sb, 2 sb + 1.
+                const int p = tid >> 7, r = (tid >> 3) & 15, cb = 2 * (tid & 7);
                 const int oi = 32 * p + 16, oj = 32 * p;
-                float x0 = 0.f, x1 = 0.f;
+                float2 x = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int t = 0; t < 16; t += 2) {
-                    x0 = fmaf(Af[(oi + r) * kLd + oj + t], Tf[(oj + t) * kLd + oj + sb], x0);
-                    x1 = fmaf(Af[(oi + r) * kLd + oj + t + 1], Tf[(oj + t + 1) * kLd + oj + sb], x1);
+                for (int t = 0; t < 16; ++t) {
+                    const float a = Af[(oi + r) * kLd + oj + t];
+                    const float2 tv = *(const float2 *)&Tf[(oj + t) * kLd + oj + cb];
+                    x.x = fmaf(a, tv.x, x.x);
+                    x.y = fmaf(a, tv.y, x.y);
                 }
-                Xf[(16 * p + r) * 33 + sb] = x0 + x1;
+                *(float2 *)&Xf[(16 * p + r) * kXLd + cb] = x;
                 compute_sync();
-                float y0 = 0.f, y1 = 0.f;
+                float2 y = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int t = 0; t < 16; t += 2) {
-                    y0 = fmaf(Tf[(oi + r) * kLd + oi + t], Xf[(16 * p + t) * 33 + sb], y0);
-                    y1 = fmaf(Tf[(oi + r) * kLd + oi + t + 1], Xf[(16 * p + t + 1) * 33 + sb], y1);
+                for (int t = 0; t < 16; ++t) {
+                    const float tt = Tf[(oi + r) * kLd + oi + t];
+                    const float2 xv = *(const float2 *)&Xf[(16 * p + t) * kXLd + cb];
+                    y.x = fmaf(tt, xv.x, y.x);
+                    y.y = fmaf(tt, xv.y, y.y);
                 }
-                y0 += y1;
-                Tf[(oi + r) * kLd + oj + sb] = -y0;
-                *(__nv_bfloat16 *)(sT + sw128_offset(oi + r, oj + sb, 64)) = __float2bfloat16_rn(-y0);
+                *(float2 *)&Tf[(oi + r) * kLd + oj + cb] = make_float2(-y.x, -y.y);
+                *(uint32_t *)(sT + sw128_offset(oi + r, oj + cb, 64)) = pack_bf16(-y.x, -y.y);
             }
             compute_sync();
             {
-                // Level 2, block rows 32..63 x columns 0..31: two outputs per thread.
-                const int r = tid >> 4, sb = tid & 15;
-                float x[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+                // Level 2, block rows 32..63 x columns 0..31: columns 4 sb .. 4 sb + 3.
+                const int r = tid >> 3, cb = 4 * (tid & 7);
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int t = 0; t < 32; t += 2) {
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const float a = Af[(32 + r) * kLd + t + u];
-#pragma unroll
-                        for (int jj = 0; jj < 2; ++jj) x[u][jj] = fmaf(a, Tf[(t + u) * kLd + sb + 16 * jj], x[u][jj]);
-                    }
+                for (int t = 0; t < 32; ++t) {
+                    const float a = Af[(32 + r) * kLd + t];
+                    const float4 tv = *(const float4 *)&Tf[t * kLd + cb];
+                    x.x = fmaf(a, tv.x, x.x); x.y = fmaf(a, tv.y, x.y);
+                    x.z = fmaf(a, tv.z, x.z); x.w = fmaf(a, tv.w, x.w);
                 }
-#pragma unroll
-                for (int jj = 0; jj < 2; ++jj) Xf[r * 33 + sb + 16 * jj] = x[0][jj] + x[1][jj];
+                *(float4 *)&Xf[r * kXLd + cb] = x;
                 compute_sync();
-                float yy[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+                float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int t = 0; t < 32; t += 2) {
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const float tt = Tf[(32 + r) * kLd + 32 + t + u];
-#pragma unroll
-                        for (int jj = 0; jj < 2; ++jj) yy[u][jj] = fmaf(tt, Xf[(t + u) * 33 + sb + 16 * jj], yy[u][jj]);
-                    }
+                for (int t = 0; t < 32; ++t) {
+                    const float tt = Tf[(32 + r) * kLd + 32 + t];
+                    const float4 xv = *(const float4 *)&Xf[t * kXLd + cb];
+                    y.x = fmaf(tt, xv.x, y.x); y.y = fmaf(tt, xv.y, y.y);
+                    y.z = fmaf(tt, xv.z, y.z); y.w = fmaf(tt, xv.w, y.w);
                 }
-                const float y[2] = {yy[0][0] + yy[1][0], yy[0][1] + yy[1][1]};
-#pragma unroll
-                for (int jj = 0; jj < 2; ++jj)
-                    *(__nv_bfloat16 *)(sT + sw128_offset(32 + r, sb + 16 * jj, 64)) = __float2bfloat16_rn(-y[jj]);
+                *(uint2 *)(sT + sw128_offset(32 + r, cb, 64)) =
+                    make_uint2(pack_bf16(-y.x, -y.y), pack_bf16(-y.z, -y.w));
             }
+            // The Kd^T and P staging is read out before the next item's loads land on it.
+            if (tid == 0) bulk_wait_read<0>();
             fence_proxy_async_smem();
             tc_fence_before_sync();
             compute_sync();
             tc_fence_after_sync();
             if (tid == 0) {
+                // [W | U] = T [beta K e^G | beta V]  (M = 64, N = 256, K = 64)
                 const uint32_t id = idesc_bf16_f32(64, 256);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma_ss(tmem_addr(tb, 0, 0), desc_kmajor_sw128(smem_u32(sT) + ks * 32),
-                           desc_kmajor_sw128(smem_u32(sKQ) + ks * 32), id, ks > 0);
+                           desc_kmajor_sw128(smem_u32(sm + kRawV) + ks * 32), id, ks > 0);
                 mma_commit(&mma_bar);
             }
             if (!mbar_wait(&mma_bar, mma_count & 1, globaltimer_ns() + kWaitNs)) {
                 if (tid == 0) record_timeout(status);
                 sAbort = 1;
-                break;
+                mma_failed = (int)(mma_count & 1);
             }
             ++mma_count;
             tc_fence_after_sync();
+            // No raw tile is read any more: the next item's loads overlap the readback.
+            if (warp == 0 && has_next && !sAbort) {
+                cp_async_wait_all();
+                __syncwarp();
+                const int wn = w + gridDim.x;
+                const int2 loc = next_loc;
+                issue(IntraItem{loc.x, loc.y, wn / H, wn % H});
+                issued = it + 2;
+            }
             {
-                // W (columns 0..127) -> rows 0..63 of [W; Qt]; U (columns 128..255).
-                // Warp w: lane quadrant w % 4, columns 64 (w / 4) .. + 63.
-                uint32_t rr[32];
-                const int wq = warp & 3, r = 16 * wq + lane, cg = warp >> 2;
-                uint32_t rr2[32];
-                tmem_ld32(tmem_addr(tb, 32 * wq, 64 * cg), rr);
-                tmem_ld32(tmem_addr(tb, 32 * wq, 64 * cg + 32), rr2);
-                tmem_ld_wait();
+                // Rows r = 16 q + i (i < 16) of lane quarter q = w % 4; warps 0-3 read W
+                // (columns 0..127) into rows 0..63 of the block's [W; Qt] image, warps
+                // 4-7 read U (columns 128..255) into its row-major block region.
+                const int q = warp & 3, hb = warp >> 2, r = 16 * q + lane;
 #pragma unroll
-                for (int q4 = 0; q4 < 2; ++q4) {
-                    const int colbase = 64 * cg + 32 * q4;
-                    if (q4 == 1) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) rr[i] = rr2[i];
-                    }
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t rr[32];
+                    tmem_ld32(tmem_addr(tb, 32 * q, 128 * hb + 32 * q4), rr);
+                    tmem_ld_wait();
                     if (lane < 16) {
 #pragma unroll
                         for (int cc = 0; cc < 32; cc += 8) {
@@ -579,34 +614,28 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                                 pack_bf16(__uint_as_float(rr[cc + 2]), __uint_as_float(rr[cc + 3])),
                                 pack_bf16(__uint_as_float(rr[cc + 4]), __uint_as_float(rr[cc + 5])),
                                 pack_bf16(__uint_as_float(rr[cc + 6]), __uint_as_float(rr[cc + 7])));
-                            const int col = colbase + cc;
-                            // Staged as block images: W (two 64-wide K halves of rows
-                            // 0..63 of [W; Qt]) in the v tile, U (row-major) in the q tile.
-                            if (col < 128)
-                                *(uint4 *)(stw + kRawV + (col >> 6) * 8192 + sw128_offset(r, col & 63, 64)) = w4;
+                            const int col = 32 * q4 + cc;
+                            if (hb == 0)
+                                *(uint4 *)(blk + kOffWQ + sw128_offset(r, col, 128)) = w4;
                             else
-                                *(uint4 *)(stw + kRawQ + (r * 128 + col - 128) * 2) = w4;
+                                *(uint4 *)(blk + kOffU + (r * 128 + col) * 2) = w4;
                         }
                     }
                 }
             }
-            fence_proxy_async_smem();
             tc_fence_before_sync();
-            compute_sync();
-            if (tid == 0) {
-                bulk_s2g(blk + kOffWQ, stw + kRawV, 8192);
-                bulk_s2g(blk + kOffWQ + 16384, stw + kRawV + 8192, 8192);
-                bulk_s2g(blk + kOffU, stw + kRawQ, 16384);
-                bulk_commit();
-            }
+            compute_sync();  // TMEM is read out before the next item's products
+            if (sAbort) break;
         }
         if (tid == 0) bulk_wait<0>();  // every staged block region has reached memory
-        // Drain: every requested copy has landed before the CTA may exit.
+        // Drain: every requested copy and product has finished before the CTA exits.
         if (warp == 0) {
             cp_async_wait_all();
-            for (int d = it; d < issued; ++d)
-                mbar_wait(&full[d & 1], (d >> 1) & 1, globaltimer_ns() + kWaitNs);
+            if (lane == 0)
+                for (int d = it; d < issued; ++d) mbar_wait(&full, d & 1, globaltimer_ns() + kWaitNs);
         }
+        if (tid == 0 && mma_failed >= 0) mbar_wait(&mma_bar, (uint32_t)mma_failed, globaltimer_ns() + kWaitNs);
+        if (tid == 0 && ap_failed >= 0) mbar_wait(&ap_bar, (uint32_t)ap_failed, globaltimer_ns() + kWaitNs);
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -945,14 +974,16 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
 
 // ---------------------------------------------------------------- compose --
 
-// Affine composition of the segments of one (sequence, head), for 32 value
+// Affine composition of the segments of one (sequence, head), for 16 value
 // channels per CTA (columns of S never mix):
 //   S_in(1) = S after segment 0,   S_in(s + 1) = M_s S_in(s) + S_loc(s),
 // the final state being S_in(Gn).  The whole scan is in fp32; each S_in(s) is
 // also written as the bf16 B-operand image (row = value channel, K = key
-// channel, 128-byte swizzled) that the correction product reads.
+// channel, 128-byte swizzled) that the correction product reads.  Thread
+// (m, half) owns row m and 8 of the CTA's columns.
 constexpr int kComposeThreads = 256;
-constexpr int kComposeCols = 32;
+constexpr int kComposeCols = 16;
+constexpr int kCpt = kComposeCols / 2;           // columns per thread
 constexpr int kMsLd = kDK + 1;
 constexpr uint32_t kComposeSmem = (kDK * kMsLd + kDK * kComposeCols) * 4;
 
@@ -962,40 +993,59 @@ compose_kernel(const int32_t *__restrict__ chunk_off, int H, int G, const float 
 {
     extern __shared__ float csm[];
     float *Ms = csm;                 // M_s [128][129]
-    float *Ss = csm + kDK * kMsLd;   // S_in(s), this CTA's columns [128][32]
+    float *Ss = csm + kDK * kMsLd;   // S_in(s), this CTA's columns [128][16]
     constexpr int nvb = kDV / kComposeCols;
     const int vb = blockIdx.x % nvb, h = (blockIdx.x / nvb) % H, n = blockIdx.x / (nvb * H);
     const int Gn = min(G, chunk_off[n + 1] - chunk_off[n]);
     if (Gn <= 1) return;             // the state kernel wrote this final state itself
     const int tid = threadIdx.x;
-    const int m = tid >> 1, cb = (tid & 1) * 16, v0 = vb * kComposeCols;
+    const int m = tid >> 1, cb = (tid & 1) * kCpt, v0 = vb * kComposeCols;
     auto xoff = [&](int s) { return (((size_t)n * G + s) * H + h) * kStateF32; };
 
-    for (int e = tid; e < kDK * kComposeCols; e += kComposeThreads)
-        Ss[e] = Sx[xoff(0) + (size_t)(e / kComposeCols) * kDV + v0 + e % kComposeCols];
+    {   // S_in(1) = state after segment 0: 128 rows x 4 float4 of this CTA's columns
+        float4 x[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int e = tid + k * kComposeThreads;
+            x[k] = *(const float4 *)(Sx + xoff(0) + (size_t)(e >> 2) * kDV + v0 + 4 * (e & 3));
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) *(float4 *)(Ss + 4 * (tid + k * kComposeThreads)) = x[k];
+    }
     __syncthreads();
     for (int s = 1; s < Gn; ++s) {
+        // Issue every global load of the step first (one memory latency, not 20).
+        float4 mr[16], sl[2];
+        const float4 *Mg = (const float4 *)(Mx + xoff(s));
+#pragma unroll
+        for (int k = 0; k < 16; ++k) mr[k] = Mg[tid + k * kComposeThreads];
+        const float4 *Sl = (const float4 *)(Sx + xoff(s) + (size_t)m * kDV + v0 + cb);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) sl[k] = Sl[k];
         uint8_t *img = Simg + (((size_t)n * G + s) * H + h) * kSinImg;
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
+        for (int i = 0; i < kCpt; ++i)
             *(__nv_bfloat16 *)(img + sw128_offset(v0 + cb + i, m, kDV)) =
                 __float2bfloat16_rn(Ss[m * kComposeCols + cb + i]);
-        const float4 *Mg = (const float4 *)(Mx + xoff(s));
-        for (int e = tid; e < kDK * kDK / 4; e += kComposeThreads) {
-            const float4 x = Mg[e];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int e = tid + k * kComposeThreads;   // float4 index: row e / 32
             float *d = Ms + (e >> 5) * kMsLd + 4 * (e & 31);
-            d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
+            d[0] = mr[k].x; d[1] = mr[k].y; d[2] = mr[k].z; d[3] = mr[k].w;
         }
         __syncthreads();
-        float acc[16];
-        const float *Sl = Sx + xoff(s) + (size_t)m * kDV + v0 + cb;
+        float acc[kCpt];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = Sl[i];
+        for (int k = 0; k < 2; ++k) {
+            acc[4 * k + 0] = sl[k].x; acc[4 * k + 1] = sl[k].y;
+            acc[4 * k + 2] = sl[k].z; acc[4 * k + 3] = sl[k].w;
+        }
+#pragma unroll 8
         for (int c = 0; c < kDK; ++c) {
             const float a = Ms[m * kMsLd + c];
             const float4 *sr = (const float4 *)(Ss + c * kComposeCols + cb);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
                 const float4 x = sr[q];
                 acc[4 * q + 0] = fmaf(a, x.x, acc[4 * q + 0]);
                 acc[4 * q + 1] = fmaf(a, x.y, acc[4 * q + 1]);
@@ -1005,13 +1055,16 @@ compose_kernel(const int32_t *__restrict__ chunk_off, int H, int G, const float 
         }
         __syncthreads();             // every read of Ss and Ms is done
 #pragma unroll
-        for (int i = 0; i < 16; ++i) Ss[m * kComposeCols + cb + i] = acc[i];
+        for (int q = 0; q < 2; ++q)
+            *(float4 *)(Ss + m * kComposeCols + cb + 4 * q) =
+                make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
         __syncthreads();
     }
     if (Sf) {
-        float *d = Sf + ((size_t)n * H + h) * kStateF32 + (size_t)m * kDV + v0 + cb;
+        float4 *d = (float4 *)(Sf + ((size_t)n * H + h) * kStateF32 + (size_t)m * kDV + v0 + cb);
+        const float4 *src = (const float4 *)(Ss + m * kComposeCols + cb);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) d[i] = Ss[m * kComposeCols + cb + i];
+        for (int q = 0; q < 2; ++q) d[q] = src[q];
     }
 }
 
@@ -1060,6 +1113,19 @@ correct_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk
         mbar_arrive_expect_tx(&bar_ld, kEImg + kSinImg);
         bulk_g2s(sm, Eimg + ((size_t)h * max_chunks + g) * kEImg, kEImg, &bar_ld);
         bulk_g2s(sm + kEImg, Simg + (((size_t)n * G + s) * H + h) * kSinImg, kSinImg, &bar_ld);
+    }
+    // While the operands arrive, every epilogue thread fetches its partial output
+    // row (M = 64: TMEM lane 32 w + i holds row 16 w + i; lanes 16..31 have none).
+    const int t0 = cu[n] + c * kChunk, len = min(kChunk, cu[n + 1] - t0);
+    const int r = 16 * warp + lane;
+    const bool has_row = lane < 16 && r < len;
+    uint4 *orow = (uint4 *)(o + ((size_t)(t0 + (has_row ? r : 0)) * H + h) * kDV);
+    uint4 ov[16];
+    if (has_row) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) ov[i] = orow[i];
+    }
+    if (tid == 0) {
         if (mbar_wait(&bar_ld, 0, globaltimer_ns() + kWaitNs)) {
             tc_fence_after_sync();
             const uint32_t id = idesc_bf16_f32(64, 128), ea = smem_u32(sm), sa = smem_u32(sm + kEImg);
@@ -1078,28 +1144,29 @@ correct_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk
     __syncthreads();
     if (sOk) {
         tc_fence_after_sync();
-        const int t0 = cu[n] + c * kChunk, len = min(kChunk, cu[n + 1] - t0);
-        const int r = 16 * warp + lane;  // M = 64: TMEM lane 32 w + i holds row 16 w + i
-#pragma unroll 1
+#pragma unroll
         for (int q = 0; q < 4; ++q) {
             uint32_t ra[32];
             tmem_ld32(tmem_addr(tb, 32 * warp, 32 * q), ra);
             tmem_ld_wait();
-            if (lane < 16 && r < len) {
-                uint4 *d4 = (uint4 *)(o + ((size_t)(t0 + r) * H + h) * kDV + 32 * q);
+            if (has_row) {
 #pragma unroll
-                for (int m4 = 0; m4 < 4; ++m4) {
-                    uint4 x = d4[m4];
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t *acc = ra + 8 * i;
+                    uint4 &x = ov[4 * q + i];
                     uint32_t *w = &x.x;
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 f = __bfloat1622float2(*(const __nv_bfloat162 *)&w[e]);
-                        w[e] = pack_bf16(f.x + __uint_as_float(ra[8 * m4 + 2 * e]),
-                                         f.y + __uint_as_float(ra[8 * m4 + 2 * e + 1]));
+                        w[e] = pack_bf16(f.x + __uint_as_float(acc[2 * e]),
+                                         f.y + __uint_as_float(acc[2 * e + 1]));
                     }
-                    d4[m4] = x;
                 }
             }
+        }
+        if (has_row) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) orow[i] = ov[i];
         }
     }
     tc_fence_before_sync();
@@ -1124,17 +1191,18 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 }
 
 // [T][H][128] bf16 rows viewed as a 3-D tensor (channel, head, token) with a
-// {128, 1, 64} box: one chunk of one head per load, no swizzle.
+// {64, 1, 64} box and the 128-byte swizzle: one K half of one chunk of one head
+// per load, landing as the K-major operand image of 64 rows x 128 bytes.
 bool encode_rows_map(CUtensorMap *map, const void *base, int32_t T, int32_t H)
 {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)kDK, (cuuint64_t)H, (cuuint64_t)(T > 0 ? T : 1)};
     const cuuint64_t strides[2] = {(cuuint64_t)kDK * 2, (cuuint64_t)H * kDK * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)kDK, 1, (cuuint32_t)kChunk};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)kChunk};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
-               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1146,10 +1214,11 @@ namespace {
 constexpr int64_t kSplitSms = 148;
 constexpr int64_t kMaxSegments = 16;
 
-// Workspace layout: plan region, per-(chunk, head) blocks, then (split only)
+// Workspace layout: plan region (offsets, order, chunk table), per-(chunk, head)
+// blocks, then (split only)
 // Sx and Mx [N][G][H] fp32 states, S_in images [N][G][H] and E images [H][chunks].
 struct WsLayout {
-    size_t plan, blocks, sx, mx, simg, eimg, total;
+    size_t plan, loc, blocks, sx, mx, simg, eimg, total;
 };
 
 WsLayout ws_layout(int32_t total_tokens, int32_t num_seqs, int32_t H, int G)
@@ -1159,7 +1228,8 @@ WsLayout ws_layout(int32_t total_tokens, int32_t num_seqs, int32_t H, int G)
     const int64_t max_chunks = ((int64_t)total_tokens + 63LL * num_seqs) / kChunk;
     auto up = [](size_t x) { return (x + 1023) & ~(size_t)1023; };
     w.plan = 0;
-    w.blocks = up((size_t)(3 * num_seqs + 3) * sizeof(int32_t));
+    w.loc = ((size_t)(3 * num_seqs + 3) * sizeof(int32_t) + 7) & ~(size_t)7;
+    w.blocks = up(w.loc + (size_t)max_chunks * sizeof(int2));
     size_t end = w.blocks + (size_t)H * max_chunks * kBlockBytes;
     if (G > 1) {
         const size_t states = (size_t)num_seqs * G * H;
@@ -1208,6 +1278,7 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
     int32_t *chunk_off = (int32_t *)ws;
     int32_t *ckpt_off = chunk_off + a.num_seqs + 1;
     int32_t *order = ckpt_off + a.num_seqs + 1;
+    int2 *chunk_loc = (int2 *)(ws + w.loc);
     uint8_t *blocks = ws + w.blocks;
     float *Sx = G > 1 ? (float *)(ws + w.sx) : nullptr;
     float *Mx = G > 1 ? (float *)(ws + w.mx) : nullptr;
@@ -1217,6 +1288,10 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
 
     err = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)(kISmem + 1024));
+    if (err != cudaSuccess) return err;
+    // Two intra CTAs share an SM: ask for the largest shared-memory carveout.
+    err = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
     if (err != cudaSuccess) return err;
     err = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kStateSmem);
@@ -1232,7 +1307,7 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
 
     a.mark(0, stream);
     plan_kernel<<<1, kPlanThreads, 0, stream>>>(a.cu_seqlens, a.num_seqs, a.ckpt_every, chunk_off,
-                                                ckpt_off, order);
+                                                ckpt_off, order, chunk_loc);
     a.mark(1, stream);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
@@ -1242,13 +1317,13 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
         if (cudaGetDevice(&dev) == cudaSuccess)
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         const int64_t items = max_chunks * a.H;
-        const unsigned grid = (unsigned)(items < sms ? items : sms);
+        const unsigned grid = (unsigned)(items < 2 * sms ? items : 2 * sms);
         CUtensorMap mk, mq, mv, mz;
         if (!encode_rows_map(&mk, a.k, a.total_tokens, a.H) || !encode_rows_map(&mq, a.q, a.total_tokens, a.H) ||
             !encode_rows_map(&mv, a.v, a.total_tokens, a.H) || !encode_rows_map(&mz, a.z, a.total_tokens, a.H))
             return cudaErrorInvalidValue;
         intra_kernel<<<grid, kIntraThreads, kISmem + 1024, stream>>>(
-            mk, mq, mv, mz, a.A, a.beta, a.cu_seqlens, chunk_off, a.num_seqs, a.H,
+            mk, mq, mv, mz, a.A, a.beta, chunk_loc, chunk_off, a.num_seqs, a.H,
             blocks, max_chunks, a.status);
         err = cudaGetLastError();
         if (err != cudaSuccess) return err;
