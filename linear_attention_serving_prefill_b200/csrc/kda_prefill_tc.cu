@@ -315,9 +315,9 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 cp_async_commit();
             }
 
-            // Pass 1: gate and cumulative log-decay of channels c0, c0 + 1 over the
-            // sub-tile's 16 rows, relative to its start: L_r = G_r - m_I.
-            float2 L[16];
+            // Pass 1: gate of channels c0, c0 + 1 summed over the sub-tile's 16 rows.
+            // (Pass 2 forms the running sums L_r = G_r - m_I again from z, in the
+            // same order, instead of holding them in registers.)
             float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -327,7 +327,6 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                     acc.x += gate_log_decay_fast(eA.x, zz.x);
                     acc.y += gate_log_decay_fast(eA.y, zz.y);
                 }
-                L[i] = acc;
             }
             sTot[I][c0] = acc.x;
             sTot[I][c0 + 1] = acc.y;
@@ -357,16 +356,22 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             // beta K e^G, beta V and K e^{G_C - G} wait in registers until the tiles
             // that receive them are no longer read.
             uint32_t pk0[8], pk1[8], pv0[8], pv1[8], kd0[8], kd1[8];
+            float2 Lr = make_float2(0.f, 0.f);  // L of the current row
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int r = 16 * I + i;
                 const bool valid = r < len;
                 const uint32_t off = sw128_offset(r, c0, 64);
+                if (valid) {
+                    const float2 zz = ld_bf16x2_smem(sm, kRawZ + off);
+                    Lr.x += gate_log_decay_fast(eA.x, zz.x);
+                    Lr.y += gate_log_decay_fast(eA.y, zz.y);
+                }
                 const float2 kv = valid ? ld_bf16x2_smem(sm, kRawK + off) : make_float2(0.f, 0.f);
                 const float2 qv = valid ? ld_bf16x2_smem(sm, kRawQ + off) : make_float2(0.f, 0.f);
                 const float2 vv = valid ? ld_bf16x2_smem(sm, kRawV + off) : make_float2(0.f, 0.f);
-                const float2 e1 = make_float2(__expf(L[i].x), __expf(L[i].y));    // in [e^-80, 1]
-                const float2 e2 = make_float2(__expf(-L[i].x), __expf(-L[i].y));  // in [1, e^80]
+                const float2 e1 = make_float2(__expf(Lr.x), __expf(Lr.y));    // in [e^-80, 1]
+                const float2 e2 = make_float2(__expf(-Lr.x), __expf(-Lr.y));  // in [1, e^80]
                 const float br = sBeta[r];
                 *(uint32_t *)(sm + kRawK + off) = pack_bf16(kv.x * e1.x, kv.y * e1.y);
                 *(uint32_t *)(sm + kRawQ + off) = pack_bf16(qv.x * e1.x, qv.y * e1.y);
