@@ -26,6 +26,13 @@ so with Kt = K*e^{G}, Kh = K*e^{-G}, Qt = Q*e^{G} (row r scaled by e^{G_r}):
 
 Library primitives used: matrix products and ``np.linalg.inv``.  In fp64 the
 e^{-G} factors stay finite for chunks up to about 140 tokens (G >= -5 per token).
+
+With an unbounded gate (the negative Softplus of the earlier Kimi Linear design,
+which the pages contrast with K3's lower bound) e^{-G} overflows inside a chunk.
+``chunk_step_pairwise`` is then the position-pair form: every A and P entry takes
+its decay e^{G_r - G_s} (s <= r, never above 1) as one exponent per pair and key
+channel, and every other factor (e^{G}, e^{G_C - G}) is at most 1 -- the same
+unrolled recurrence, with no reciprocal decay anywhere.
 """
 from __future__ import annotations
 
@@ -34,9 +41,36 @@ import numpy as np
 G_MIN = -5.0
 
 
-def _gate(z: np.ndarray, A: np.ndarray) -> np.ndarray:
-    """g = g_min * sigmoid(exp(A) * z), section 3.3 gate equation (one head)."""
-    return G_MIN / (1.0 + np.exp(-(np.exp(A) * z)))
+def _gate(z: np.ndarray, A: np.ndarray, kind: str = "bounded") -> np.ndarray:
+    """g = g_min * sigmoid(exp(A) * z), section 3.3 gate equation (one head);
+    kind="softplus": g = -log(1 + exp(exp(A) * z))."""
+    x = np.exp(A) * z
+    if kind == "softplus":
+        return -np.logaddexp(0.0, x)
+    return G_MIN / (1.0 + np.exp(-x))
+
+
+def chunk_step_pairwise(q, k, v, g, beta, S0):
+    """``chunk_step`` with the intra-chunk decays taken pair by pair.
+
+    A[r,s] = beta_r sum_c k_rc k_sc e^{G_rc - G_sc} (s < r) and
+    P[r,s] = sum_c q_rc k_sc e^{G_rc - G_sc} (s <= r); the rest as in chunk_step.
+    """
+    C = q.shape[0]
+    G = np.cumsum(g, axis=0)
+    lower = np.tril(np.ones((C, C), dtype=bool))          # s <= r
+    expo = np.where(lower[:, :, None], G[:, None, :] - G[None, :, :], -np.inf)
+    E = np.exp(expo)                                      # [r, s, c], entries in [0, 1]
+    A = np.tril(beta[:, None] * np.einsum("rc,sc,rsc->rs", k, k, E), -1)
+    P = np.einsum("rc,sc,rsc->rs", q, k, E)
+    Kt, Qt = k * np.exp(G), q * np.exp(G)
+    Tinv = np.linalg.inv(np.eye(C) + A)
+    W = Tinv @ (beta[:, None] * Kt)
+    U = Tinv @ (beta[:, None] * v)
+    D = U - W @ S0
+    O = Qt @ S0 + P @ D
+    S_out = np.exp(G[-1])[:, None] * S0 + (k * np.exp(G[-1] - G)).T @ D
+    return O, S_out
 
 
 def chunk_step(q, k, v, g, beta, S0):
@@ -57,11 +91,12 @@ def chunk_step(q, k, v, g, beta, S0):
     return O, S_out
 
 
-def prefill(q, k, v, z, A, beta, cu_seqlens, initial_state=None, chunk: int = 16):
+def prefill(q, k, v, z, A, beta, cu_seqlens, initial_state=None, chunk: int = 16,
+            gate: str = "bounded", pairwise: bool = False):
     """Chunkwise prefill with chunks aligned to each sequence start.
 
     Same shapes and result as ``oracle.prefill``; every argument is a float64
-    (or int for cu_seqlens) NumPy array.
+    (or int for cu_seqlens) NumPy array.  ``pairwise`` uses chunk_step_pairwise.
     """
     q, k, v, z, A, beta = (np.asarray(t, dtype=np.float64) for t in (q, k, v, z, A, beta))
     cu = np.asarray(cu_seqlens, dtype=np.int64)
@@ -76,9 +111,9 @@ def prefill(q, k, v, z, A, beta, cu_seqlens, initial_state=None, chunk: int = 16
                  else np.asarray(initial_state[i, h], dtype=np.float64).copy())
             for c0 in range(int(cu[i]), int(cu[i + 1]), chunk):
                 c1 = min(c0 + chunk, int(cu[i + 1]))
-                g = _gate(z[c0:c1, h], A[h])
-                O, S = chunk_step(q[c0:c1, h], k[c0:c1, h], v[c0:c1, h], g,
-                                  beta[c0:c1, h], S)
+                g = _gate(z[c0:c1, h], A[h], gate)
+                step = chunk_step_pairwise if pairwise else chunk_step
+                O, S = step(q[c0:c1, h], k[c0:c1, h], v[c0:c1, h], g, beta[c0:c1, h], S)
                 o[c0:c1, h] = O
             sf[i, h] = S
     return o, sf

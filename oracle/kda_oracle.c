@@ -25,6 +25,10 @@
  *       g_t = g_min * sigmoid(exp(A) * z_t),  alpha_t = exp(g_t),  g_min = -5
  *     read per head h and key channel c as
  *       g[t,h,c] = -5 * sigmoid(exp(A[h,c]) * z[t,h,c]).
+ *   - the same section and "Kimi K3 Under the Hood" section "Sequence mixing":
+ *     the earlier Kimi Linear gate was an unbounded negative Softplus.  Read
+ *     with the same pre-activation (gate kind 1):
+ *       g[t,h,c] = -softplus(exp(A[h,c]) * z[t,h,c]),  softplus(x) = log(1 + e^x).
  *
  * Layouts (row-major, all fp64 on this side):
  *   q, k, z : [T, H, dk]     v, o : [T, H, dv]     beta : [T, H]
@@ -43,18 +47,25 @@
 #endif
 
 #define KDA_ORACLE_GMIN (-5.0)
+#define KDA_ORACLE_GATE_BOUNDED 0   /* g_min * sigmoid(exp(A) z) */
+#define KDA_ORACLE_GATE_SOFTPLUS 1  /* -softplus(exp(A) z), unbounded below */
 
 /* sigmoid(x) = 1 / (1 + exp(-x)).  For x -> -inf exp(-x) overflows to +inf and
  * the result is exactly 0; for x -> +inf it is exactly 1. */
 static double oracle_sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
 
-/* Gate of one (token, head): g[c] = g_min * sigmoid(exp(A[c]) * z[c]).
- * "Kimi K3: Architecture, Training, and Million-Token Agentic RL", section 3.3
- * gate equation. */
-static void oracle_gate_row(const double *z, const double *A, int dk, double *g)
+/* softplus(x) = log(1 + e^x), written as max(x, 0) + log(1 + e^{-|x|}) so that
+ * neither branch overflows. */
+static double oracle_softplus(double x) { return (x > 0.0 ? x : 0.0) + log1p(exp(-fabs(x))); }
+
+/* Gate of one (token, head): g[c] = g_min * sigmoid(exp(A[c]) * z[c])
+ * ("Kimi K3: Architecture, Training, and Million-Token Agentic RL", section 3.3
+ * gate equation), or -softplus(exp(A[c]) * z[c]) for the unbounded kind. */
+static void oracle_gate_row(const double *z, const double *A, int dk, double *g, int kind)
 {
     for (int c = 0; c < dk; ++c)
-        g[c] = KDA_ORACLE_GMIN * oracle_sigmoid(exp(A[c]) * z[c]);
+        g[c] = kind == KDA_ORACLE_GATE_SOFTPLUS ? -oracle_softplus(exp(A[c]) * z[c])
+                                                : KDA_ORACLE_GMIN * oracle_sigmoid(exp(A[c]) * z[c]);
 }
 
 /* One token of the recurrence on a dk x dv state, in the section 3.2 edit order.
@@ -91,22 +102,40 @@ int kda_oracle_max_threads(void)
 #endif
 }
 
-/* Gate for a whole [T, H, dk] tensor. */
-void kda_oracle_gate(const double *z, const double *A, int64_t T, int H, int dk,
-                     double *g)
+/* Gate for a whole [T, H, dk] tensor, of the given kind. */
+void kda_oracle_gate_kind(const double *z, const double *A, int64_t T, int H, int dk,
+                          double *g, int kind)
 {
     for (int64_t t = 0; t < T; ++t)
         for (int h = 0; h < H; ++h)
             oracle_gate_row(z + ((size_t)t * H + h) * dk, A + (size_t)h * dk, dk,
-                            g + ((size_t)t * H + h) * dk);
+                            g + ((size_t)t * H + h) * dk, kind);
 }
+
+void kda_oracle_gate(const double *z, const double *A, int64_t T, int H, int dk,
+                     double *g)
+{
+    kda_oracle_gate_kind(z, A, T, H, dk, g, KDA_ORACLE_GATE_BOUNDED);
+}
+
+int kda_oracle_prefill_gate(const double *q, const double *k, const double *v,
+                            const double *z, const double *A, const double *beta,
+                            const int32_t *cu_seqlens, int num_seqs, int H, int dk,
+                            int dv, const double *initial_state, double *o,
+                            double *final_state, int every, double *checkpoints,
+                            int nthreads, int kind);
 
 int kda_oracle_prefill_ckpt(const double *q, const double *k, const double *v,
                             const double *z, const double *A, const double *beta,
                             const int32_t *cu_seqlens, int num_seqs, int H, int dk,
                             int dv, const double *initial_state, double *o,
                             double *final_state, int every, double *checkpoints,
-                            int nthreads);
+                            int nthreads)
+{
+    return kda_oracle_prefill_gate(q, k, v, z, A, beta, cu_seqlens, num_seqs, H, dk, dv,
+                                   initial_state, o, final_state, every, checkpoints, nthreads,
+                                   KDA_ORACLE_GATE_BOUNDED);
+}
 
 /*
  * Prefill over packed variable-length sequences: for every sequence n and head
@@ -134,12 +163,12 @@ int kda_oracle_prefill(const double *q, const double *k, const double *v,
  * tokens, stored at row (sum_{m<n} L_m / every) + j - 1 of checkpoints
  * [count, H, dk, dv].
  */
-int kda_oracle_prefill_ckpt(const double *q, const double *k, const double *v,
+int kda_oracle_prefill_gate(const double *q, const double *k, const double *v,
                             const double *z, const double *A, const double *beta,
                             const int32_t *cu_seqlens, int num_seqs, int H, int dk,
                             int dv, const double *initial_state, double *o,
                             double *final_state, int every, double *checkpoints,
-                            int nthreads)
+                            int nthreads, int kind)
 {
     int failed = 0;
 #ifdef _OPENMP
@@ -171,7 +200,7 @@ int kda_oracle_prefill_ckpt(const double *q, const double *k, const double *v,
                         ck_base += (cu_seqlens[m + 1] - cu_seqlens[m]) / every;
                 for (int64_t t = cu_seqlens[n]; t < cu_seqlens[n + 1]; ++t) {
                     const size_t th = (size_t)t * H + h;
-                    oracle_gate_row(z + th * dk, A + (size_t)h * dk, dk, g);
+                    oracle_gate_row(z + th * dk, A + (size_t)h * dk, dk, g, kind);
                     oracle_token_step(S, q + th * dk, k + th * dk, v + th * dv, g,
                                       beta[th], dk, dv, vhat, o + th * dv);
                     const int64_t done = t + 1 - cu_seqlens[n];
@@ -198,10 +227,10 @@ int kda_oracle_prefill_ckpt(const double *q, const double *k, const double *v,
  * the read after the write.  slots == NULL means slot[b] = b.  Section 3.2 of
  * the same note gives the decode interface (x_t, S_{t-1}) -> (y_t, S_t).
  */
-int kda_oracle_decode(const double *q, const double *k, const double *v,
-                      const double *z, const double *A, const double *beta,
-                      int B, int H, int dk, int dv, double *state,
-                      const int32_t *slots, double *o, int nthreads)
+int kda_oracle_decode_gate(const double *q, const double *k, const double *v,
+                           const double *z, const double *A, const double *beta,
+                           int B, int H, int dk, int dv, double *state,
+                           const int32_t *slots, double *o, int nthreads, int kind)
 {
     int failed = 0;
 #ifdef _OPENMP
@@ -224,7 +253,7 @@ int kda_oracle_decode(const double *q, const double *k, const double *v,
                 const int slot = slots ? slots[b] : b;
                 const size_t th = (size_t)b * H + h;
                 double *S = state + ((size_t)slot * H + h) * (size_t)dk * dv;
-                oracle_gate_row(z + th * dk, A + (size_t)h * dk, dk, g);
+                oracle_gate_row(z + th * dk, A + (size_t)h * dk, dk, g, kind);
                 oracle_token_step(S, q + th * dk, k + th * dk, v + th * dv, g,
                                   beta[th], dk, dv, vhat, o + th * dv);
             }
@@ -233,4 +262,13 @@ int kda_oracle_decode(const double *q, const double *k, const double *v,
         free(vhat);
     }
     return failed ? -1 : 0;
+}
+
+int kda_oracle_decode(const double *q, const double *k, const double *v,
+                      const double *z, const double *A, const double *beta,
+                      int B, int H, int dk, int dv, double *state,
+                      const int32_t *slots, double *o, int nthreads)
+{
+    return kda_oracle_decode_gate(q, k, v, z, A, beta, B, H, dk, dv, state, slots, o, nthreads,
+                                  KDA_ORACLE_GATE_BOUNDED);
 }

@@ -8,7 +8,9 @@ CUDA package never imports it.
 What it computes ("Kimi K3: Architecture, Training, and Million-Token Agentic
 RL", sections 3.1-3.3): per head, the state edit
 ``Sbar = Diag(alpha) S; vhat = Sbar^T k; S = Sbar + beta k (v - vhat)^T;
-o = S^T q`` with the gate ``g = -5 * sigmoid(exp(A) * z)``, ``alpha = exp(g)``.
+o = S^T q`` with the gate ``g = -5 * sigmoid(exp(A) * z)``, ``alpha = exp(g)``
+-- or, as the earlier unbounded gate the pages contrast it with, the negative
+Softplus ``g = -softplus(exp(A) * z)``.
 
 Every input is converted to float64 before the call, so the oracle consumes the
 exact values the GPU receives (bf16 or fp32 tensors upcast without rounding).
@@ -61,6 +63,14 @@ def _load():
         lib.kda_oracle_decode.restype = i32
         lib.kda_oracle_gate.argtypes = [d, d, i64, i32, i32, d]
         lib.kda_oracle_gate.restype = None
+        lib.kda_oracle_gate_kind.argtypes = [d, d, i64, i32, i32, d, i32]
+        lib.kda_oracle_gate_kind.restype = None
+        lib.kda_oracle_prefill_gate.argtypes = [d, d, d, d, d, d, d, i32, i32, i32, i32,
+                                                d, d, d, i32, d, i32, i32]
+        lib.kda_oracle_prefill_gate.restype = i32
+        lib.kda_oracle_decode_gate.argtypes = [d, d, d, d, d, d, i32, i32, i32, i32, d,
+                                               d, d, i32, i32]
+        lib.kda_oracle_decode_gate.restype = i32
         lib.kda_oracle_max_threads.argtypes = []
         lib.kda_oracle_max_threads.restype = i32
         _lib = lib
@@ -90,20 +100,28 @@ def max_threads() -> int:
     return int(_load().kda_oracle_max_threads())
 
 
-def gate(z, A) -> np.ndarray:
-    """g[t,h,c] = -5 * sigmoid(exp(A[h,c]) * z[t,h,c]) for z [T,H,dk], A [H,dk]."""
+# Gate kinds: the K3 lower-bounded gate (section 3.3 of the note) and the
+# unbounded negative Softplus of the earlier Kimi Linear design.
+GATES = {"bounded": 0, "softplus": 1}
+
+
+def gate(z, A, kind: str = "bounded") -> np.ndarray:
+    """g[t,h,c] = -5 * sigmoid(exp(A[h,c]) * z[t,h,c]) for z [T,H,dk], A [H,dk];
+    with kind="softplus", g = -softplus(exp(A[h,c]) * z[t,h,c])."""
     z, A = _f64(z), _f64(A)
     T, H, dk = z.shape
     g = np.empty_like(z)
-    _load().kda_oracle_gate(_ptr(z), _ptr(A), T, H, dk, _ptr(g))
+    _load().kda_oracle_gate_kind(_ptr(z), _ptr(A), T, H, dk, _ptr(g), GATES[kind])
     return g
 
 
-def prefill(q, k, v, z, A, beta, cu_seqlens, initial_state=None, nthreads: int = 0):
+def prefill(q, k, v, z, A, beta, cu_seqlens, initial_state=None, nthreads: int = 0,
+            gate: str = "bounded"):
     """Token-by-token fp64 recurrence over packed sequences.
 
     Shapes: q, k, z [T,H,dk]; v [T,H,dv]; beta [T,H]; A [H,dk];
     cu_seqlens [N+1]; initial_state [N,H,dk,dv] or None (zeros).
+    ``gate`` selects the gate kind (see ``gate``).
     Returns ``(o [T,H,dv], final_state [N,H,dk,dv])`` as float64 arrays.
     """
     q, k, v, z, A, beta = (_f64(t) for t in (q, k, v, z, A, beta))
@@ -114,9 +132,9 @@ def prefill(q, k, v, z, A, beta, cu_seqlens, initial_state=None, nthreads: int =
     s0 = None if initial_state is None else _f64(initial_state)
     o = np.zeros((T, H, dv), dtype=np.float64)
     sf = np.zeros((n, H, dk, dv), dtype=np.float64)
-    rc = _load().kda_oracle_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(A),
-                                    _ptr(beta), _ptr(cu), n, H, dk, dv, _ptr(s0),
-                                    _ptr(o), _ptr(sf), nthreads)
+    rc = _load().kda_oracle_prefill_gate(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(A),
+                                         _ptr(beta), _ptr(cu), n, H, dk, dv, _ptr(s0),
+                                         _ptr(o), _ptr(sf), 0, None, nthreads, GATES[gate])
     if rc != 0:
         raise MemoryError("kda oracle: allocation failed")
     return o, sf
@@ -155,7 +173,8 @@ def prefill_checkpoints(q, k, v, z, A, beta, cu_seqlens, every: int, initial_sta
     return o, sf, ck
 
 
-def decode_step(q, k, v, z, A, beta, state, slots=None, nthreads: int = 0):
+def decode_step(q, k, v, z, A, beta, state, slots=None, nthreads: int = 0,
+                gate: str = "bounded"):
     """One single-token step per batch row; returns ``(o [B,H,dv], new_state)``.
 
     ``state`` is the pool [P,H,dk,dv]; it is copied, never modified in place.
@@ -167,9 +186,9 @@ def decode_step(q, k, v, z, A, beta, state, slots=None, nthreads: int = 0):
     dv = v.shape[2]
     sl = None if slots is None else _i32(slots)
     o = np.zeros((B, H, dv), dtype=np.float64)
-    rc = _load().kda_oracle_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(A),
-                                   _ptr(beta), B, H, dk, dv, _ptr(st), _ptr(sl),
-                                   _ptr(o), nthreads)
+    rc = _load().kda_oracle_decode_gate(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(A),
+                                        _ptr(beta), B, H, dk, dv, _ptr(st), _ptr(sl),
+                                        _ptr(o), nthreads, GATES[gate])
     if rc != 0:
         raise MemoryError("kda oracle: allocation failed")
     return o, st

@@ -375,3 +375,86 @@ def test_checkpoints_are_prefix_final_states():
                 np.testing.assert_array_equal(ck[row], s_pref[0])
                 row += 1
         assert row == ck.shape[0]
+
+
+# ------------------------------------------- the unbounded (Softplus) gate ----
+# "Kimi K3: Architecture, Training, and Million-Token Agentic RL", section 3.3,
+# and "Kimi K3 Under the Hood", section "Sequence mixing": the earlier Kimi
+# Linear gate was an unbounded negative Softplus, whose 16-token cumulative decay
+# has no lower bound, so reciprocal decay overflows and diagonal tiles need a
+# position-pair path.  Read here as g = -softplus(exp(A) * z).
+
+def test_softplus_gate_closed_forms():
+    rs = np.random.RandomState(11)
+    A = rs.uniform(-1, 1, (3, 7))
+    # at z = 0: -log 2 exactly, whatever A is
+    np.testing.assert_allclose(oracle.gate(np.zeros((1, 3, 7)), A, "softplus"), -np.log(2.0),
+                               rtol=1e-15)
+    # A = 0 reduces to -log(1 + e^z), scipy's log-sum-exp of (0, z)
+    from scipy.special import logsumexp
+    zs = rs.randn(9, 1, 4) * 3
+    ref = -logsumexp(np.stack([np.zeros_like(zs), zs]), axis=0)
+    np.testing.assert_allclose(oracle.gate(zs, np.zeros((1, 4)), "softplus"), ref, rtol=1e-14)
+    # asymptotes: -x + e^{-x} terms for large x, -e^{x} for very negative x
+    big = np.full((1, 1, 1), 40.0)
+    assert abs(oracle.gate(big, np.zeros((1, 1)), "softplus")[0, 0, 0] + 40.0) < 1e-15
+    small = np.full((1, 1, 1), -40.0)
+    np.testing.assert_allclose(oracle.gate(small, np.zeros((1, 1)), "softplus"), -np.exp(-40.0),
+                               rtol=1e-12)
+    # unbounded below: g = -exp(A) z once exp(A) z is large
+    z = np.full((1, 3, 7), 1e4)
+    np.testing.assert_allclose(oracle.gate(z, A, "softplus"), -np.exp(A)[None] * 1e4, rtol=1e-12)
+    # strictly negative and decreasing in z
+    zz = np.linspace(-6, 6, 101)[:, None, None] * np.ones((1, 3, 7))
+    gg = oracle.gate(zz, A, "softplus")
+    assert np.all(gg < 0) and np.all(np.diff(gg, axis=0) < 0)
+
+
+def test_softplus_tile_decay_leaves_the_bound():
+    """With z = 60 the 16-token cumulative decay passes -80 (and -745, where
+    e^{-G} overflows even fp64): the separable chunk form breaks down, the
+    position-pair form stays finite and equals the token recurrence."""
+    x = _inputs([40], H=2, dk=6, dv=5, seed=12, z_mean=60.0)
+    g = oracle.gate(x["z"], x["A"], "softplus")
+    G16 = np.cumsum(g[:16], axis=0)
+    assert G16[-1].min() < -745.0
+    o, sf = oracle.prefill(**x, gate="softplus")
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(sf))
+    with np.errstate(all="ignore"):
+        o_sep, _ = chunkwise.prefill(**x, chunk=16, gate="softplus")
+    assert not np.all(np.isfinite(o_sep))
+    o_pw, sf_pw = chunkwise.prefill(**x, chunk=16, gate="softplus", pairwise=True)
+    assert _relerr(o_pw, o) < 1e-12 and _relerr(sf_pw, sf) < 1e-12
+
+
+@pytest.mark.parametrize("gate", ["bounded", "softplus"])
+@pytest.mark.parametrize("chunk", [1, 3, 16])
+def test_pairwise_chunk_form_equals_recurrence(gate, chunk):
+    x = _inputs([37, 16, 5], H=2, dk=6, dv=4, seed=13 + chunk, z_mean=1.0)
+    o, sf = oracle.prefill(**x, gate=gate)
+    o_pw, sf_pw = chunkwise.prefill(**x, chunk=chunk, gate=gate, pairwise=True)
+    assert _relerr(o_pw, o) < 1e-11 and _relerr(sf_pw, sf) < 1e-11
+
+
+def test_softplus_recurrence_matches_brute_force_product():
+    x = _inputs([6], H=1, dk=4, dv=3, seed=14, z_mean=2.0)
+    o, sf = oracle.prefill(**x, gate="softplus")
+    g = oracle.gate(x["z"], x["A"], "softplus")
+    S = x["initial_state"][0, 0].copy()
+    for t in range(6):
+        kk, b = x["k"][t, 0], x["beta"][t, 0]
+        S = (np.eye(4) - b * np.outer(kk, kk)) @ np.diag(np.exp(g[t, 0])) @ S + b * np.outer(kk, x["v"][t, 0])
+        np.testing.assert_allclose(o[t, 0], S.T @ x["q"][t, 0], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(sf[0, 0], S, rtol=1e-12, atol=1e-14)
+
+
+def test_softplus_decode_continues_prefill():
+    x = _inputs([9], H=2, dk=5, dv=4, seed=15, z_mean=3.0)
+    o, sf = oracle.prefill(**x, gate="softplus")
+    head = {key: x[key][:8] for key in ("q", "k", "v", "z", "beta")}
+    _, s8 = oracle.prefill(**head, A=x["A"], cu_seqlens=np.array([0, 8], np.int32),
+                           initial_state=x["initial_state"], gate="softplus")
+    od, sd = oracle.decode_step(*(x[key][8:9] for key in ("q", "k", "v", "z")), x["A"],
+                                x["beta"][8:9], s8, gate="softplus")
+    np.testing.assert_allclose(od[0], o[8], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(sd, sf, rtol=1e-12, atol=1e-14)

@@ -32,6 +32,9 @@ MUTANTS = {
     "gmin_wrong": ("#define KDA_ORACLE_GMIN (-5.0)", "#define KDA_ORACLE_GMIN (-4.0)"),
     "gate_without_exp_A": ("oracle_sigmoid(exp(A[c]) * z[c])", "oracle_sigmoid(A[c] * z[c])"),
     "no_decay": ("const double alpha = exp(g[c]);", "const double alpha = 1.0 + 0.0 * g[c];"),
+    "softplus_argument_negated": ("-oracle_softplus(exp(A[c]) * z[c])", "-oracle_softplus(-exp(A[c]) * z[c])"),
+    "softplus_without_exp_A": ("-oracle_softplus(exp(A[c]) * z[c])", "-oracle_softplus(A[c] * z[c])"),
+    "softplus_without_log": ("+ log1p(exp(-fabs(x)))", "+ exp(-fabs(x))"),
     "vhat_from_old_state": (
         "    /* vhat = Sbar^T k. */",
         "    for (int c = 0; c < dk; ++c) { const double a = exp(g[c]);"
@@ -47,6 +50,7 @@ PIN_TESTS = [
     pins.test_decay_scales_rows_scalar_channel_via_lfilter,
     pins.test_per_step_write_identity,
     lambda: pins.test_chunkwise_form_equals_recurrence(16),
+    pins.test_softplus_gate_closed_forms,
 ]
 
 
@@ -66,7 +70,9 @@ def _build_mutant(tmp_path, name):
 def test_pins_catch_mutant(tmp_path, name):
     real = ormod._load()
     lib = ctypes.CDLL(_build_mutant(tmp_path, name))
-    for fn in ("kda_oracle_prefill", "kda_oracle_decode", "kda_oracle_gate", "kda_oracle_max_threads"):
+    for fn in ("kda_oracle_prefill", "kda_oracle_decode", "kda_oracle_gate", "kda_oracle_max_threads",
+               "kda_oracle_prefill_gate", "kda_oracle_decode_gate", "kda_oracle_gate_kind",
+               "kda_oracle_prefill_ckpt"):
         getattr(lib, fn).argtypes = getattr(real, fn).argtypes
         getattr(lib, fn).restype = getattr(real, fn).restype
     caught = []
