@@ -270,6 +270,55 @@ def split_leg(K, rank_seed, rank, world, dev, stream, args, max_over_ranks, barr
     return out
 
 
+def gate_leg(K, rank_seed, rank, world, dev, stream, args, max_over_ranks, barrier):
+    """The cost the lower bound removes: the 4,096-token, 32-head prefill on the
+    fp32 CUDA-core path with the K3 gate (dense 16-token tiles, separable
+    e^{+-G}) and with the unbounded Softplus gate (position-pair tiles, one
+    exponent per pair and key channel), next to the tensor-core path, which the
+    bound makes possible.  L2 is flushed before every call."""
+    from dataclasses import replace
+
+    from linear_attention_serving_prefill_b200.workloads import CONFIGS, config_inputs
+    cfg = CONFIGS["prefill_4k"]
+    x = config_inputs(replace(cfg, seed=rank_seed(cfg.seed, rank)), device=dev)
+    T, H = x["q"].shape[0], cfg.H
+    o = torch.empty(T, H, cfg.dv, dtype=torch.bfloat16, device=dev)
+    S = torch.empty(1, H, cfg.dk, cfg.dv, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(K.kda_prefill_workspace_size(T, 1, H, cfg.dk, cfg.dv, torch.bfloat16,
+                                                      "tensor_core"), 1),
+                     dtype=torch.uint8, device=dev)
+    out = {"workload": cfg.name, "l2": "flushed before every call"}
+    reps = 5
+    for name, algo, gate in (("tensor_core_bounded", "tensor_core", "bounded"),
+                             ("cuda_core_bounded", "cuda_core", "bounded"),
+                             ("cuda_core_softplus", "cuda_core", "softplus")):
+        def call():
+            K.kda_prefill(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"], x["cu_seqlens"],
+                          x["cu_seqlens_host"], None, final_state=S, o=o, workspace=ws, algo=algo,
+                          stream=stream, gate=gate)
+
+        for _ in range(2):
+            call()
+        torch.cuda.synchronize()
+        barrier()
+        ts = []
+        for i in range(reps):
+            flush.fill_(i & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            call()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ms = max_over_ranks(statistics.median(ts), world, dev)
+        out[name] = {"ms": ms, "tokens_per_s": T / (ms / 1e3)}
+    out["pair_path_cost"] = out["cuda_core_softplus"]["ms"] / out["cuda_core_bounded"]["ms"]
+    out["softplus_vs_tensor_core_bounded"] = out["cuda_core_softplus"]["ms"] / out["tensor_core_bounded"]["ms"]
+    del x, o, S, flush, ws
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -379,9 +428,10 @@ def main():
             "roofline_ms": th * BYTES_PER_TOKEN_HEAD / hbm_peak / 1e6}
     launches = args.steps * nk
 
-    decode = e2e = cpu = ckpt = split = None
+    decode = e2e = cpu = ckpt = split = gate_cost = None
     if not args.prefill_only:
         split = split_leg(K, rank_seed, rank, world, dev, stream, args, max_over_ranks, barrier)
+        gate_cost = gate_leg(K, rank_seed, rank, world, dev, stream, args, max_over_ranks, barrier)
 
         # Prefix-cache checkpoints every 512 tokens (the pages' hash block) on the same
         # workload: the cost of writing 64 KiB per (checkpoint, head) from the state pass.
@@ -523,6 +573,7 @@ def main():
             "decode": decode,
             "checkpoints": ckpt,
             "sequence_split": split,
+            "unbounded_gate": gate_cost,
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clocks,

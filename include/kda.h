@@ -76,6 +76,11 @@ typedef enum {
                                   segments composed by an affine scan (bf16 only) */
 } kda_algo;
 
+typedef enum {
+    KDA_GATE_LOWER_BOUNDED = 0,  /* K3: g = -5 sigmoid(exp(A) z), in [-5, 0] */
+    KDA_GATE_SOFTPLUS = 1        /* earlier Kimi Linear: g = -softplus(exp(A) z), unbounded */
+} kda_gate;
+
 /* Version of this ABI (KDA_ABI_VERSION of the build). */
 int32_t kda_abi_version(void);
 
@@ -164,6 +169,32 @@ kda_status kda_prefill_checkpointed(const void *q, const void *k, const void *v,
                                     size_t workspace_bytes, kda_algo algo, void *stream,
                                     void *const *stage_events, int32_t num_stage_events,
                                     int32_t checkpoint_every, float *checkpoints);
+
+/*
+ * kda_prefill_ex with a choice of gate, without events.  KDA_GATE_LOWER_BOUNDED is
+ * kda_prefill_ex itself.  KDA_GATE_SOFTPLUS is the earlier Kimi Linear gate, which
+ * the pages contrast with K3's bound ("Kimi K3: Architecture, Training, and
+ * Million-Token Agentic RL", section 3.3; "Kimi K3 Under the Hood", section
+ * "Sequence mixing": an unbounded negative Softplus, read with K3's pre-activation
+ * as g = -softplus(exp(A[h,c]) z[t,h,c])).  Its cumulative decay inside a 16-token
+ * tile is unbounded, so the reciprocal factors of the dense tile form overflow and
+ * every diagonal tile needs the position-pair path: the fp32 CUDA-core path
+ * computes each intra-chunk decay e^{G_r - G_s} as one exponent per pair and key
+ * channel.  With KDA_GATE_SOFTPLUS, algo AUTO or CUDA_CORE runs that path;
+ * TENSOR_CORE(_SPLIT), whose dense diagonal tiles rest on the bound, returns
+ * KDA_ERR_UNSUPPORTED.  The per-token log-decay is clamped at -110 (e^{-110} is
+ * 0 in fp32), which changes no result and keeps a chunk's cumulative decay
+ * small enough for fp32 differences.  That path needs no workspace (workspace may
+ * be NULL with workspace_bytes = 0).  A gate value outside the enum is
+ * KDA_ERR_INVALID_ARG.
+ */
+kda_status kda_prefill_gated(const void *q, const void *k, const void *v, const void *z,
+                             const float *A, const float *beta,
+                             const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                             int32_t num_seqs, int32_t total_tokens, int32_t H, int32_t dk,
+                             int32_t dv, kda_dtype dt, const float *initial_state,
+                             float *final_state, void *o, void *workspace,
+                             size_t workspace_bytes, kda_algo algo, kda_gate gate, void *stream);
 
 /*
  * Rows of the checkpoint tensor for these HOST offsets: sum over sequences of
@@ -256,6 +287,17 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
                            int32_t dk, int32_t dv, kda_dtype dt, float *state,
                            int32_t pool_size, const int32_t *slots, void *o,
                            void *stream);
+
+/*
+ * kda_decode_step with a choice of gate (kda_gate, as for kda_prefill_gated; the
+ * decode step needs no special path for the unbounded gate: alpha = e^{g} is
+ * applied directly).  A gate value outside the enum is KDA_ERR_INVALID_ARG.
+ */
+kda_status kda_decode_step_gated(const void *q, const void *k, const void *v, const void *z,
+                                 const float *A, const float *beta, int32_t B, int32_t H,
+                                 int32_t dk, int32_t dv, kda_dtype dt, float *state,
+                                 int32_t pool_size, const int32_t *slots, void *o,
+                                 kda_gate gate, void *stream);
 
 /*
  * Speculative-decoding verify and replay ("Kimi K3 Under the Hood", section

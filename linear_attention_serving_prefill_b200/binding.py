@@ -19,6 +19,7 @@ _LIB_PATH = os.path.join(_PKG, "libkda_b200.so")
 
 KDA_DTYPE = {torch.bfloat16: 0, torch.float32: 1}
 KDA_ALGO = {"auto": 0, "cuda_core": 1, "tensor_core": 2, "tensor_core_split": 3}
+KDA_GATE = {"bounded": 0, "softplus": 1}
 STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
                 3: "KDA_ERR_WORKSPACE", 4: "KDA_ERR_CUDA", 5: "KDA_ERR_TIMEOUT"}
 
@@ -37,6 +38,8 @@ SIGNATURES = {
     "kda_checkpoint_count": ([_P, _I32, _I32], ctypes.c_int64),
     "kda_prefill_noalloc": ([_P] * 8 + [_I32] * 6 + [_P] * 4, _I32),
     "kda_decode_step": ([_P] * 6 + [_I32] * 5 + [_P, _I32, _P, _P, _P], _I32),
+    "kda_decode_step_gated": ([_P] * 6 + [_I32] * 5 + [_P, _I32, _P, _P, _I32, _P], _I32),
+    "kda_prefill_gated": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _I32, _I32, _P], _I32),
     "kda_device_status": ([_P, _P], _I32),
     "kda_decode_multi": ([_P] * 6 + [_I32] * 6 + [_P, _I32, _P, _P, _I32, _P, _P], _I32),
     "kda_selftest_wait_timeout": ([ctypes.c_int64, _P], _I32),
@@ -102,7 +105,7 @@ def kda_prefill_workspace_size(total_tokens: int, num_seqs: int, H: int, dk: int
 
 def kda_prefill(q, k, v, z, A, beta, cu_seqlens, cu_seqlens_host=None, initial_state=None,
                 output_final_state: bool = True, final_state=None, o=None, workspace=None,
-                algo: str = "auto", stream=None, stage_events=None):
+                algo: str = "auto", stream=None, stage_events=None, gate: str = "bounded"):
     """Chunked KDA prefill over packed sequences; returns ``(o, final_state)``.
 
     q, k, z [T,H,dk], v [T,H,dv] (bf16 or fp32, one dtype); A [H,dk] fp32;
@@ -111,6 +114,7 @@ def kda_prefill(q, k, v, z, A, beta, cu_seqlens, cu_seqlens_host=None, initial_s
     may be passed (e.g. ``initial_state`` itself, for in-place resume);
     otherwise it is allocated when ``output_final_state``.  ``stage_events``
     (a list of recorded ``torch.cuda.Event``) receives the kernel boundaries.
+    ``gate="softplus"`` selects the unbounded gate (kda_prefill_gated; no events).
     """
     T, H, dk = q.shape
     dv = v.shape[2]
@@ -130,6 +134,19 @@ def kda_prefill(q, k, v, z, A, beta, cu_seqlens, cu_seqlens_host=None, initial_s
         ch = cu_seqlens_host.to(torch.int32).contiguous()
         host = ctypes.c_void_p(ch.data_ptr())
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if gate != "bounded":
+        if stage_events:
+            raise ValueError("stage events are recorded for the lower-bounded gate only")
+        code = _lib.kda_prefill_gated(
+            _dev(q, "q", dt), _dev(k, "k", dt), _dev(v, "v", dt), _dev(z, "z", dt),
+            _dev(A, "A", torch.float32), _dev(beta, "beta", torch.float32),
+            _dev(cu_seqlens, "cu_seqlens", torch.int32), host, N, T, H, dk, dv, KDA_DTYPE[dt],
+            _dev(initial_state, "initial_state", torch.float32),
+            _dev(final_state, "final_state", torch.float32), _dev(o, "o", dt),
+            _dev(workspace, "workspace"), ws_bytes, KDA_ALGO[algo], KDA_GATE[gate],
+            _stream_ptr(stream))
+        _check(code, "kda_prefill_gated")
+        return o, final_state
     ev_arr, n_ev = None, 0
     if stage_events:
         ev_arr = (ctypes.c_void_p * len(stage_events))(*[e.cuda_event for e in stage_events])
@@ -231,18 +248,19 @@ def kda_prefill_segments(T: int, N: int, H: int, dk: int, dv: int, dtype=torch.b
     return int(_lib.kda_prefill_segments(T, N, H, dk, dv, KDA_DTYPE[dtype], KDA_ALGO[algo]))
 
 
-def kda_decode_step(q, k, v, z, A, beta, state, slots=None, o=None, stream=None):
+def kda_decode_step(q, k, v, z, A, beta, state, slots=None, o=None, stream=None,
+                    gate: str = "bounded"):
     """One decode step; ``state`` [P,H,dk,dv] fp32 is updated in place; returns o."""
     B, H, dk = q.shape
     dv = v.shape[2]
     dt = q.dtype
     if o is None:
         o = torch.empty(B, H, dv, dtype=dt, device=q.device)
-    code = _lib.kda_decode_step(
+    code = _lib.kda_decode_step_gated(
         _dev(q, "q", dt), _dev(k, "k", dt), _dev(v, "v", dt), _dev(z, "z", dt),
         _dev(A, "A", torch.float32), _dev(beta, "beta", torch.float32), B, H, dk, dv,
         KDA_DTYPE[dt], _dev(state, "state", torch.float32), state.shape[0],
-        _dev(slots, "slots", torch.int32), _dev(o, "o", dt), _stream_ptr(stream))
+        _dev(slots, "slots", torch.int32), _dev(o, "o", dt), KDA_GATE[gate], _stream_ptr(stream))
     _check(code, "kda_decode_step")
     return o
 

@@ -120,16 +120,27 @@ extern "C" int64_t kda_checkpoint_count(const int32_t *cu_seqlens_host, int32_t 
     return total;
 }
 
-extern "C" kda_status kda_prefill_checkpointed(
-    const void *q, const void *k, const void *v, const void *z, const float *A, const float *beta,
-    const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host, int32_t num_seqs,
-    int32_t total_tokens, int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
-    const float *initial_state, float *final_state, void *o, void *workspace,
-    size_t workspace_bytes, kda_algo algo, void *stream, void *const *stage_events,
-    int32_t num_stage_events, int32_t checkpoint_every, float *checkpoints)
+namespace {
+
+// Every prefill entry point lands here.
+kda_status prefill_impl(const void *q, const void *k, const void *v, const void *z, const float *A,
+                        const float *beta, const int32_t *cu_seqlens_dev,
+                        const int32_t *cu_seqlens_host, int32_t num_seqs, int32_t total_tokens,
+                        int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+                        const float *initial_state, float *final_state, void *o, void *workspace,
+                        size_t workspace_bytes, kda_algo algo, void *stream,
+                        void *const *stage_events, int32_t num_stage_events,
+                        int32_t checkpoint_every, float *checkpoints, kda_gate gate)
 {
     kda_status st = check_prefill_sizes(total_tokens, num_seqs, H, dk, dv, dt, algo);
     if (st != KDA_OK) return st;
+    if (gate != KDA_GATE_LOWER_BOUNDED && gate != KDA_GATE_SOFTPLUS) return KDA_ERR_INVALID_ARG;
+    if (gate == KDA_GATE_SOFTPLUS) {
+        // The tensor-core path relies on the lower bound; the unbounded gate runs
+        // on the CUDA-core path with its position-pair diagonal tiles.
+        if (algo == KDA_ALGO_TENSOR_CORE || algo == KDA_ALGO_TENSOR_CORE_SPLIT) return KDA_ERR_UNSUPPORTED;
+        algo = KDA_ALGO_CUDA_CORE;
+    }
     if (checkpoint_every < 0 || checkpoint_every % 64 != 0) return KDA_ERR_INVALID_ARG;
     if (checkpoint_every > 0 && (!checkpoints || !aligned(checkpoints, 16))) return KDA_ERR_INVALID_ARG;
     if (checkpoint_every > 0 && algo == KDA_ALGO_TENSOR_CORE_SPLIT) return KDA_ERR_UNSUPPORTED;
@@ -166,11 +177,43 @@ extern "C" kda_status kda_prefill_checkpointed(
     // Checkpoints come from the unsplit state chain; AUTO then keeps every
     // sequence whole (its workspace, sized for a split, is large enough).
     a.segments = checkpoint_every > 0 ? 1 : segments_for(total_tokens, num_seqs, H, dk, dv, dt, algo);
+    a.gate = gate == KDA_GATE_SOFTPLUS ? 1 : 0;
 
     cudaError_t err = use_tensor_core(dk, dv, dt, algo)
                           ? kda::launch_prefill_tensor_core(a, (cudaStream_t)stream)
                           : kda::launch_prefill_cuda_core(a, (cudaStream_t)stream);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" kda_status kda_prefill_checkpointed(
+    const void *q, const void *k, const void *v, const void *z, const float *A, const float *beta,
+    const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host, int32_t num_seqs,
+    int32_t total_tokens, int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+    const float *initial_state, float *final_state, void *o, void *workspace,
+    size_t workspace_bytes, kda_algo algo, void *stream, void *const *stage_events,
+    int32_t num_stage_events, int32_t checkpoint_every, float *checkpoints)
+{
+    return prefill_impl(q, k, v, z, A, beta, cu_seqlens_dev, cu_seqlens_host, num_seqs,
+                        total_tokens, H, dk, dv, dt, initial_state, final_state, o, workspace,
+                        workspace_bytes, algo, stream, stage_events, num_stage_events,
+                        checkpoint_every, checkpoints, KDA_GATE_LOWER_BOUNDED);
+}
+
+extern "C" kda_status kda_prefill_gated(const void *q, const void *k, const void *v, const void *z,
+                                        const float *A, const float *beta,
+                                        const int32_t *cu_seqlens_dev,
+                                        const int32_t *cu_seqlens_host, int32_t num_seqs,
+                                        int32_t total_tokens, int32_t H, int32_t dk, int32_t dv,
+                                        kda_dtype dt, const float *initial_state,
+                                        float *final_state, void *o, void *workspace,
+                                        size_t workspace_bytes, kda_algo algo, kda_gate gate,
+                                        void *stream)
+{
+    return prefill_impl(q, k, v, z, A, beta, cu_seqlens_dev, cu_seqlens_host, num_seqs,
+                        total_tokens, H, dk, dv, dt, initial_state, final_state, o, workspace,
+                        workspace_bytes, algo, stream, nullptr, 0, 0, nullptr, gate);
 }
 
 extern "C" kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const void *z,
@@ -216,7 +259,19 @@ extern "C" kda_status kda_decode_step(const void *q, const void *k, const void *
                                       int32_t pool_size, const int32_t *slots, void *o,
                                       void *stream)
 {
+    return kda_decode_step_gated(q, k, v, z, A, beta, B, H, dk, dv, dt, state, pool_size, slots, o,
+                                 KDA_GATE_LOWER_BOUNDED, stream);
+}
+
+extern "C" kda_status kda_decode_step_gated(const void *q, const void *k, const void *v,
+                                            const void *z, const float *A, const float *beta,
+                                            int32_t B, int32_t H, int32_t dk, int32_t dv,
+                                            kda_dtype dt, float *state, int32_t pool_size,
+                                            const int32_t *slots, void *o, kda_gate gate,
+                                            void *stream)
+{
     if (B < 0 || H <= 0 || pool_size < 0) return KDA_ERR_INVALID_ARG;
+    if (gate != KDA_GATE_LOWER_BOUNDED && gate != KDA_GATE_SOFTPLUS) return KDA_ERR_INVALID_ARG;
     if (dt != KDA_DTYPE_BF16 && dt != KDA_DTYPE_F32) return KDA_ERR_INVALID_ARG;
     if (dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
@@ -232,6 +287,7 @@ extern "C" kda_status kda_decode_step(const void *q, const void *k, const void *
     a.q = q; a.k = k; a.v = v; a.z = z; a.A = A; a.beta = beta;
     a.B = B; a.H = H; a.dk = dk; a.dv = dv; a.bf16 = (dt == KDA_DTYPE_BF16);
     a.state = state; a.slots = slots; a.o = o;
+    a.gate = gate == KDA_GATE_SOFTPLUS ? 1 : 0;
     cudaError_t err = kda::launch_decode_step(a, (cudaStream_t)stream);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

@@ -28,4 +28,24 @@ __device__ __forceinline__ float gate_log_decay(float expA, float z) {
     return kGMin / (1.0f + expf(-expA * z));
 }
 
+// The unbounded gate of the earlier Kimi Linear design, which the same section
+// contrasts with the bound: g = -softplus(exp(A) * z) = -log(1 + e^{exp(A) z}),
+// evaluated as -(max(x, 0) + log1p(e^{-|x|})).  The result is clamped at
+// kGClampSoftplus: below it e^{g} is already 0 in fp32, and the clamp keeps the
+// cumulative log-decay of a chunk small enough that differences of it do not
+// cancel catastrophically.
+constexpr float kGClampSoftplus = -110.0f;
+
+__device__ __forceinline__ float gate_log_decay_softplus(float expA, float z) {
+    const float x = expA * z;
+    return fmaxf(-(fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)))), kGClampSoftplus);
+}
+
+// Gate kinds of the C ABI (kda_gate).
+enum GateKind : int { kGateBounded = 0, kGateSoftplus = 1 };
+
+template <int GATE> __device__ __forceinline__ float gate_fn(float expA, float z) {
+    return GATE == kGateSoftplus ? gate_log_decay_softplus(expA, z) : gate_log_decay(expA, z);
+}
+
 }  // namespace kda

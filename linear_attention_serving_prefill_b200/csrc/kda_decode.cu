@@ -19,7 +19,7 @@ namespace {
 
 constexpr int kThreads = 256;
 
-template <int DK, int DV, typename TIn>
+template <int DK, int DV, typename TIn, int GATE>
 __global__ void __launch_bounds__(kThreads)
 decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                    const TIn *__restrict__ v, const TIn *__restrict__ z,
@@ -53,7 +53,7 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     if (tid < DK) {
         const float kc = to_f32(k[tok * DK + tid]);
         const float qc = to_f32(q[tok * DK + tid]);
-        const float g = gate_log_decay(expf(A[(size_t)h * DK + tid]), to_f32(z[tok * DK + tid]));
+        const float g = gate_fn<GATE>(expf(A[(size_t)h * DK + tid]), to_f32(z[tok * DK + tid]));
         sAlpha[tid] = expf(g);
         sK[tid] = kc;
         sQ[tid] = qc;
@@ -122,9 +122,14 @@ cudaError_t launch_typed(const DecodeArgs &a, cudaStream_t stream)
 {
     const long long blocks = (long long)a.B * a.H;
     if (blocks == 0) return cudaSuccess;
-    decode_step_kernel<DK, DV, TIn><<<(unsigned)blocks, kThreads, 0, stream>>>(
-        (const TIn *)a.q, (const TIn *)a.k, (const TIn *)a.v, (const TIn *)a.z, a.A, a.beta,
-        a.H, a.state, a.slots, (TIn *)a.o);
+    if (a.gate == kGateSoftplus)
+        decode_step_kernel<DK, DV, TIn, kGateSoftplus><<<(unsigned)blocks, kThreads, 0, stream>>>(
+            (const TIn *)a.q, (const TIn *)a.k, (const TIn *)a.v, (const TIn *)a.z, a.A, a.beta,
+            a.H, a.state, a.slots, (TIn *)a.o);
+    else
+        decode_step_kernel<DK, DV, TIn, kGateBounded><<<(unsigned)blocks, kThreads, 0, stream>>>(
+            (const TIn *)a.q, (const TIn *)a.k, (const TIn *)a.v, (const TIn *)a.z, a.A, a.beta,
+            a.H, a.state, a.slots, (TIn *)a.o);
     return cudaGetLastError();
 }
 

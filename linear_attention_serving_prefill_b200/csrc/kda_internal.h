@@ -24,6 +24,7 @@ struct PrefillArgs {
     int32_t ckpt_every;             // 0 = no checkpoints, else a multiple of 64
     float *checkpoints;             // [count, H, dk, dv] or nullptr
     int32_t segments;               // tensor-core path: segments per sequence (1 = no split)
+    int32_t gate = 0;               // 0 = K3 lower-bounded gate, 1 = unbounded -softplus
     void *const *events;            // optional cudaEvent_t per kernel boundary
     int32_t num_events;
     // Records boundary i (0 = before the first kernel) when the caller asked for it.
@@ -40,6 +41,7 @@ struct DecodeArgs {
     float *state;
     const int32_t *slots;
     void *o;
+    int32_t gate = 0;               // as PrefillArgs::gate
 };
 
 struct DecodeMultiArgs {

@@ -18,6 +18,12 @@
 // crosses only chunk boundaries (section 3.3 chunk I/O equation).  The e^{-G}
 // factor reaches at most e^{80}, finite in fp32 -- the bound section 3.3 gives
 // for a 16-token tile.
+//
+// With the unbounded negative-Softplus gate that section contrasts with the
+// bound, e^{-G} overflows and every chunk is a diagonal tile needing the
+// position-pair path: A and P take their decays pair by pair,
+//   A[r][s] = beta_r sum_c k_rc k_sc e^{G_rc - G_sc},   P[r][s] = sum_c q_rc k_sc e^{G_rc - G_sc},
+// each exponent <= 0, and nothing else uses a reciprocal decay.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -28,15 +34,17 @@ constexpr int kC = 16;      // chunk length
 constexpr int kDVS = 32;    // dv slice per CTA
 constexpr int kThreads = 256;
 
-template <int DK>
+template <int DK, int GATE>
 struct CudaCoreSmem {
     static constexpr int LD = DK + 1;  // padded row stride: conflict-free column walks
+    // the pair path keeps the raw q and the cumulative log-decay G besides
+    static constexpr int kPair = GATE == kGateSoftplus ? 2 * kC * LD : 0;
     static constexpr int kFloats = 4 * kC * LD + DK * kDVS + 2 * kC * kDVS +
-                                   2 * kC * (kC + 1) + 3 * DK + kC;
+                                   2 * kC * (kC + 1) + 3 * DK + kC + kPair;
     static constexpr size_t kBytes = sizeof(float) * kFloats;
 };
 
-template <int DK, typename TIn>
+template <int DK, typename TIn, int GATE>
 __global__ void __launch_bounds__(kThreads)
 prefill_cuda_core_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                          const TIn *__restrict__ v, const TIn *__restrict__ z,
@@ -45,7 +53,8 @@ prefill_cuda_core_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                          const float *S0, float *Sf, TIn *__restrict__ o, int ckpt_every,
                          float *__restrict__ ckpts)
 {
-    constexpr int LD = CudaCoreSmem<DK>::LD;
+    constexpr int LD = CudaCoreSmem<DK, GATE>::LD;
+    constexpr bool kPairPath = GATE == kGateSoftplus;
     extern __shared__ float sm[];
     float *sKt = sm;                  // [kC][LD]  K e^{G}
     float *sKh = sKt + kC * LD;       // [kC][LD]  K e^{-G}
@@ -60,6 +69,8 @@ prefill_cuda_core_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     float *sGL = sEA + DK;            // [DK] G at the chunk's last row
     float *sEGL = sGL + DK;           // [DK] exp(G_last)
     float *sB = sEGL + DK;            // [kC] beta
+    float *sQr = sB + kC;             // [kC][LD] raw q   (pair path only)
+    float *sG = sQr + kC * LD;        // [kC][LD] G       (pair path only)
 
     const int nslices = dv / kDVS;
     const int slice = blockIdx.x % nslices;
@@ -96,7 +107,7 @@ prefill_cuda_core_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                 const size_t idx = ((size_t)(tc + r) * H + h) * DK + c;
                 kv = to_f32(k[idx]);
                 qv = to_f32(q[idx]);
-                gv = gate_log_decay(sEA[c], to_f32(z[idx]));
+                gv = gate_fn<GATE>(sEA[c], to_f32(z[idx]));
             }
             sKt[r * LD + c] = kv;
             sQt[r * LD + c] = qv;
@@ -124,11 +135,17 @@ prefill_cuda_core_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         for (int e = tid; e < kC * DK; e += kThreads) {
             const int r = e / DK, c = e % DK;
             const float G = sKd[r * LD + c], kv = sKt[r * LD + c], qv = sQt[r * LD + c];
-            const float eg = expf(G), emg = expf(-G);
+            const float eg = expf(G);
             sKt[r * LD + c] = kv * eg;
-            sKh[r * LD + c] = kv * emg;
             sQt[r * LD + c] = qv * eg;
             sKd[r * LD + c] = kv * expf(sGL[c] - G);
+            if (kPairPath) {
+                sKh[r * LD + c] = kv;   // raw k, q and G for the pair decays
+                sQr[r * LD + c] = qv;
+                sG[r * LD + c] = G;
+            } else {
+                sKh[r * LD + c] = kv * expf(-G);
+            }
         }
         __syncthreads();
 
@@ -136,11 +153,23 @@ prefill_cuda_core_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         {
             const int r = tid / kC, s = tid % kC;
             float a = 0.f, p = 0.f;
+            if (kPairPath) {
+                if (s <= r) {
+#pragma unroll 4
+                    for (int c = 0; c < DK; ++c) {
+                        const float e = expf(sG[r * LD + c] - sG[s * LD + c]);  // <= 1
+                        const float ke = sKh[s * LD + c] * e;
+                        a = fmaf(sKh[r * LD + c], ke, a);
+                        p = fmaf(sQr[r * LD + c], ke, p);
+                    }
+                }
+            } else {
 #pragma unroll 8
-            for (int c = 0; c < DK; ++c) {
-                const float kh = sKh[s * LD + c];
-                a = fmaf(sKt[r * LD + c], kh, a);
-                p = fmaf(sQt[r * LD + c], kh, p);
+                for (int c = 0; c < DK; ++c) {
+                    const float kh = sKh[s * LD + c];
+                    a = fmaf(sKt[r * LD + c], kh, a);
+                    p = fmaf(sQt[r * LD + c], kh, p);
+                }
             }
             sA[r * (kC + 1) + s] = s < r ? sB[r] * a : 0.f;
             sP[r * (kC + 1) + s] = s <= r ? p : 0.f;
@@ -216,11 +245,11 @@ prefill_cuda_core_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     }
 }
 
-template <int DK, typename TIn>
-cudaError_t launch_typed(const PrefillArgs &a, cudaStream_t stream)
+template <int DK, typename TIn, int GATE>
+cudaError_t launch_gated(const PrefillArgs &a, cudaStream_t stream)
 {
-    const size_t smem = CudaCoreSmem<DK>::kBytes;
-    auto kern = prefill_cuda_core_kernel<DK, TIn>;
+    const size_t smem = CudaCoreSmem<DK, GATE>::kBytes;
+    auto kern = prefill_cuda_core_kernel<DK, TIn, GATE>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem);
     if (err != cudaSuccess) return err;
@@ -233,6 +262,13 @@ cudaError_t launch_typed(const PrefillArgs &a, cudaStream_t stream)
         a.checkpoints);
     a.mark(1, stream);
     return cudaGetLastError();
+}
+
+template <int DK, typename TIn>
+cudaError_t launch_typed(const PrefillArgs &a, cudaStream_t stream)
+{
+    return a.gate == kGateSoftplus ? launch_gated<DK, TIn, kGateSoftplus>(a, stream)
+                                   : launch_gated<DK, TIn, kGateBounded>(a, stream);
 }
 
 }  // namespace

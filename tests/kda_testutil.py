@@ -29,7 +29,7 @@ def token_index(cu_host, seqs):
     return torch.cat([torch.arange(cu[n], cu[n + 1]) for n in seqs]) if seqs else torch.zeros(0, dtype=torch.long)
 
 
-def oracle_subset(inp: dict, seqs, heads):
+def oracle_subset(inp: dict, seqs, heads, gate: str = "bounded"):
     """Oracle on every token of sequences ``seqs`` for heads ``heads``.
 
     Returns ``(o [T_sub, len(heads), dv], S [len(seqs), len(heads), dk, dv], tok)``
@@ -51,7 +51,7 @@ def oracle_subset(inp: dict, seqs, heads):
                                  .index_select(1, hs.to(dev)).cpu()
     o, S = oracle.prefill(pick(inp["q"]), pick(inp["k"]), pick(inp["v"]), pick(inp["z"]),
                           inp["A"].index_select(0, hs.to(dev)).cpu(), pick(inp["beta"]),
-                          sub_cu, s0)
+                          sub_cu, s0, gate=gate)
     return o, S, tok
 
 

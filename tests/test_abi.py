@@ -245,3 +245,20 @@ def test_decode_multi_rejects_bad_arguments():
     assert call(dk=48) == UNSUPPORTED
     assert call(nt=_fake(0x10002)) == INVALID
     assert call(Bn=0) == OK
+
+
+def test_gated_entry_points_validate_the_gate():
+    """The unbounded gate runs on the CUDA-core path only; a gate outside the
+    enum is rejected before anything is launched."""
+    def gated(algo, gate, dt=BF16, dk=128, dv=128):
+        return B._lib.kda_prefill_gated(_fake(), _fake(), _fake(), _fake(), _fake(), _fake(),
+                                        _fake(), None, 2, 10, 4, dk, dv, dt, None, None, _fake(),
+                                        None, 0, algo, gate, None)
+    assert gated(TC, 1) == UNSUPPORTED
+    assert gated(SPLIT, 1) == UNSUPPORTED
+    assert gated(AUTO, 7) == INVALID
+    assert gated(CORE, -1) == INVALID
+    assert gated(TC, 1, dt=F32) == UNSUPPORTED
+    dec = B._lib.kda_decode_step_gated(_fake(), _fake(), _fake(), _fake(), _fake(), _fake(), 2, 2,
+                                       128, 128, BF16, _fake(), 2, None, _fake(), 3, None)
+    assert dec == INVALID

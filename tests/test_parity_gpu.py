@@ -243,6 +243,81 @@ def test_auto_with_checkpoints_keeps_sequences_whole():
     assert relerr(to_np(got[1]), ref_S) <= TOL_BF16
 
 
+# ------------------------------------------------- unbounded (Softplus) gate ----
+
+@pytest.mark.parametrize("dtype,tol", [("f32", TOL_F32), ("bf16", TOL_BF16)])
+@pytest.mark.parametrize("z_mean", [0.0, 3.0])
+def test_softplus_gate_prefill_matches_oracle(dtype, tol, z_mean):
+    """The unbounded gate on the CUDA-core path (position-pair diagonal tiles).
+    At z_mean = 3 a 16-token cumulative log-decay reaches well below -88, where
+    the dense tile form's e^{-G} would overflow fp32."""
+    lengths = [1, 15, 16, 17, 100, 0, 257]
+    x = _cuda(prefill_inputs(lengths, 3, 128, 128, dtype, seed=70 + int(z_mean), s0_std=0.02,
+                             z_mean=z_mean))
+    if z_mean > 0:
+        from oracle import oracle as orc
+        g = orc.gate(x["z"], x["A"], "softplus")
+        # tokens 165..180: one 16-token chunk of the 257-token sequence (starts at 149)
+        assert np.cumsum(g[165:181], axis=0).min() < -88.0
+    o, S = K.kda_prefill(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"], x["cu_seqlens"],
+                         x["cu_seqlens_host"], initial_state=x["initial_state"], gate="softplus")
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    n, H = len(lengths), 3
+    ref_o, ref_S, tok = oracle_subset(x, list(range(n)), list(range(H)), gate="softplus")
+    got_o, got_S = gpu_subset(o, S, tok, list(range(n)), list(range(H)))
+    assert relerr(got_o, ref_o) <= tol and relerr(got_S, ref_S) <= tol
+
+
+def test_softplus_gate_saturated_decay():
+    """z = 60: per-token log-decay far below the -110 clamp, the state is wiped
+    at every step; both sides agree and nothing overflows."""
+    x = _cuda(prefill_inputs([70, 33], 2, 128, 128, "bf16", seed=72, s0_std=0.5, z_mean=60.0,
+                             z_std=0.0))
+    o, S = K.kda_prefill(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"], x["cu_seqlens"],
+                         x["cu_seqlens_host"], initial_state=x["initial_state"], gate="softplus",
+                         algo="cuda_core")
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    ref_o, ref_S, tok = oracle_subset(x, [0, 1], [0, 1], gate="softplus")
+    got_o, got_S = gpu_subset(o, S, tok, [0, 1], [0, 1])
+    assert relerr(got_o, ref_o) <= TOL_BF16 and relerr(got_S, ref_S) <= TOL_BF16
+
+
+def test_softplus_gate_bounded_inputs_differ_from_bounded_gate():
+    """The gate selector is live: the same inputs under the two gates differ,
+    and the bounded call through the gated entry point equals kda_prefill."""
+    x = _cuda(prefill_inputs([80], 2, 128, 128, "f32", seed=73))
+    o_b, S_b = K.kda_prefill(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"], x["cu_seqlens"],
+                             x["cu_seqlens_host"], algo="cuda_core")
+    o_s, _ = K.kda_prefill(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"], x["cu_seqlens"],
+                           x["cu_seqlens_host"], algo="cuda_core", gate="softplus")
+    ws = torch.empty(0, dtype=torch.uint8, device="cuda")
+    o_g = torch.empty_like(o_b)
+    S_g = torch.empty_like(S_b)
+    ch = x["cu_seqlens_host"].to(torch.int32).contiguous()
+    code = K._lib.kda_prefill_gated(
+        x["q"].data_ptr(), x["k"].data_ptr(), x["v"].data_ptr(), x["z"].data_ptr(), x["A"].data_ptr(),
+        x["beta"].data_ptr(), x["cu_seqlens"].data_ptr(), ch.data_ptr(), 1, 80, 2, 128, 128, 1,
+        None, S_g.data_ptr(), o_g.data_ptr(), None, 0, K.KDA_ALGO["cuda_core"], 0, None)
+    torch.cuda.synchronize()
+    assert code == 0
+    assert torch.equal(o_g, o_b) and torch.equal(S_g, S_b)
+    assert (o_s - o_b).abs().max().item() > 1e-3
+
+
+@pytest.mark.parametrize("dtype,tol", [("f32", TOL_F32), ("bf16", TOL_BF16)])
+def test_softplus_gate_decode_matches_oracle(dtype, tol):
+    d = decode_inputs(16, 4, 128, 128, dtype, seed=74, nsets=2, device="cuda")
+    st = d["state"].clone()
+    o = K.kda_decode_step(d["q"][0], d["k"][0], d["v"][0], d["z"][0], d["A"], d["beta"][0], st,
+                          gate="softplus")
+    torch.cuda.synchronize()
+    ref_o, ref_S = oracle.decode_step(d["q"][0], d["k"][0], d["v"][0], d["z"][0], d["A"],
+                                      d["beta"][0], d["state"], gate="softplus")
+    assert relerr(to_np(o), ref_o) <= tol and relerr(to_np(st), ref_S) <= tol
+
+
 # ------------------------------------------------------------------ decode ----
 
 @pytest.mark.parametrize("dtype,tol", [("bf16", TOL_BF16), ("f32", TOL_F32)])
