@@ -14,6 +14,9 @@
 //     which is written back in place once.
 // One CTA of 256 threads per (sequence, head); thread (rg, cg) holds rows
 // rg, rg + RG, ... of float4 column group cg, as in the single-token kernel.
+// The inputs of kGroup tokens at a time are fetched together into shared
+// memory (one memory latency per group, not one per token) before the group's
+// sequential token steps run on the register-resident state.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -21,6 +24,7 @@ namespace kda {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kGroup = 8;   // tokens whose inputs are fetched together
 
 template <int DK, int DV, typename TIn>
 __global__ void __launch_bounds__(kThreads)
@@ -36,7 +40,9 @@ decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     constexpr int RPT = DK / RG;
     static_assert(RPT >= 1 && RG * CG == kThreads, "bad decode tiling");
 
-    __shared__ float sAlpha[DK], sK[DK], sQ[DK];
+    __shared__ float sEA[DK];
+    __shared__ float sAlphaG[kGroup][DK], sKG[kGroup][DK], sQG[kGroup][DK], sVG[kGroup][DV];
+    __shared__ float sBetaG[kGroup];
     __shared__ float4 sRedV[RG][CG], sRedP[RG][CG];
     __shared__ float4 sDelta[CG];
     __shared__ float sKQ;
@@ -53,17 +59,30 @@ decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     float4 s[RPT];
 #pragma unroll
     for (int i = 0; i < RPT; ++i) s[i] = S4[(size_t)(rg + i * RG) * CG + cg];
-    const float eA = tid < DK ? expf(A[(size_t)h * DK + tid]) : 0.f;
+    for (int c = tid; c < DK; c += kThreads) sEA[c] = expf(A[(size_t)h * DK + c]);
 
     for (int t = 0; t < n_tok; ++t) {
+        const int tg = t % kGroup;
         const size_t tok = ((size_t)b * Tq + t) * H + h;   // [B, Tq, H, ...]
-        __syncthreads();  // the previous token's reads of sAlpha/sK/sQ/sDelta are done
-        if (tid < DK) {
-            sAlpha[tid] = expf(gate_log_decay(eA, to_f32(z[tok * DK + tid])));
-            sK[tid] = to_f32(k[tok * DK + tid]);
-            sQ[tid] = to_f32(q[tok * DK + tid]);
+        __syncthreads();  // the previous token's reads of the group buffers and sDelta are done
+        if (tg == 0) {
+            // Inputs of tokens t .. t + kGroup - 1 (those that exist), all loads in flight together.
+            const int ng = min(kGroup, n_tok - t);
+            for (int e = tid; e < ng * DK; e += kThreads) {
+                const int u = e / DK, c = e % DK;
+                const size_t tu = ((size_t)b * Tq + t + u) * H + h;
+                sAlphaG[u][c] = expf(gate_log_decay(sEA[c], to_f32(z[tu * DK + c])));
+                sKG[u][c] = to_f32(k[tu * DK + c]);
+                sQG[u][c] = to_f32(q[tu * DK + c]);
+            }
+            for (int e = tid; e < ng * DV; e += kThreads) {
+                const int u = e / DV, jv = e % DV;
+                sVG[u][jv] = to_f32(v[(((size_t)b * Tq + t + u) * H + h) * DV + jv]);
+            }
+            if (tid < ng) sBetaG[tid] = beta[((size_t)b * Tq + t + tid) * H + h];
+            __syncthreads();
         }
-        __syncthreads();
+        const float *sAlpha = sAlphaG[tg], *sK = sKG[tg], *sQ = sQG[tg];
         if (tid < 32) {
             float acc = 0.f;
             for (int c = tid; c < DK; c += 32) acc = fmaf(sK[c], sQ[c], acc);
@@ -92,13 +111,14 @@ decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                 tv.x += a.x; tv.y += a.y; tv.z += a.z; tv.w += a.w;
                 tp.x += c.x; tp.y += c.y; tp.z += c.z; tp.w += c.w;
             }
-            const float bt = beta[tok];
+            const float bt = sBetaG[tg];
             const size_t vo = tok * DV + (size_t)tid * 4;
+            const float4 vv = *(const float4 *)&sVG[tg][4 * tid];
             float4 d;
-            d.x = bt * (to_f32(v[vo + 0]) - tv.x);
-            d.y = bt * (to_f32(v[vo + 1]) - tv.y);
-            d.z = bt * (to_f32(v[vo + 2]) - tv.z);
-            d.w = bt * (to_f32(v[vo + 3]) - tv.w);
+            d.x = bt * (vv.x - tv.x);
+            d.y = bt * (vv.y - tv.y);
+            d.z = bt * (vv.z - tv.z);
+            d.w = bt * (vv.w - tv.w);
             sDelta[tid] = d;
             if (o) {
                 const float kq = sKQ;
