@@ -243,6 +243,44 @@ def test_auto_with_checkpoints_keeps_sequences_whole():
     assert relerr(to_np(got[1]), ref_S) <= TOL_BF16
 
 
+# ------------------------------------------------------- plan edge cases ----
+
+@pytest.mark.parametrize("algo", ["tensor_core", "tensor_core_split"])
+def test_more_sequences_than_the_sorted_plan(algo):
+    """4,200 sequences of 0-70 tokens: above the 4,096 sequences the plan sorts
+    longest-first, so launch order falls back to the identity; every output and
+    final state against the oracle."""
+    rs = np.random.RandomState(80)
+    lengths = [int(x) for x in rs.randint(0, 71, size=4200)]
+    x = _cuda(prefill_inputs(lengths, 2, 128, 128, "bf16", seed=81, s0_std=0.02))
+    o, S = _run(x, algo)
+    torch.cuda.synchronize()
+    _check_all(x, o, S, TOL_BF16)
+
+
+@pytest.mark.parametrize("algo", ["tensor_core", "tensor_core_split"])
+def test_one_long_sequence_two_heads(algo):
+    """65,537 tokens (1,025 chunks, a one-token last chunk), 2 heads: the whole
+    chain, and 16 segments of 64-65 chunks, against the oracle."""
+    L = 65537
+    x = _cuda(prefill_inputs([L], 2, 128, 128, "bf16", seed=82, s0_std=0.02))
+    if algo == "tensor_core_split":
+        assert K.kda_prefill_segments(L, 1, 2, 128, 128, torch.bfloat16, algo) == 16
+    o, S = _run(x, algo)
+    torch.cuda.synchronize()
+    _check_all(x, o, S, TOL_BF16)
+
+
+def test_split_with_empty_and_single_chunk_sequences_interleaved():
+    lengths = [0, 64 * 9 + 3, 0, 1, 64 * 5, 0]
+    x = _cuda(prefill_inputs(lengths, 3, 128, 128, "bf16", seed=83, s0_std=0.3))
+    o, S = _run(x, "tensor_core_split")
+    torch.cuda.synchronize()
+    for n in (0, 2, 5):
+        assert torch.equal(S[n], x["initial_state"][n])
+    _check_all(x, o, S, TOL_BF16)
+
+
 # ------------------------------------------------- unbounded (Softplus) gate ----
 
 @pytest.mark.parametrize("dtype,tol", [("f32", TOL_F32), ("bf16", TOL_BF16)])
