@@ -197,6 +197,35 @@ kda_status kda_prefill_gated(const void *q, const void *k, const void *v, const 
                              size_t workspace_bytes, kda_algo algo, kda_gate gate, void *stream);
 
 /*
+ * Debug run of the tensor-core prefill (bf16, dk = dv = 128; otherwise
+ * KDA_ERR_UNSUPPORTED): the same call as kda_prefill_ex with
+ * KDA_ALGO_TENSOR_CORE, which also writes the intermediates that its fused
+ * kernels keep on chip, per token, as fp32 [T, H, 128] (any pointer may be NULL;
+ * 16-byte aligned):
+ *   G_out      the cumulative log-decay of the token's 64-token chunk (chunks
+ *              start at each sequence start; "Kimi K3: Architecture, Training,
+ *              and Million-Token Agentic RL", section 3.3 gate equation and the
+ *              inclusive in-chunk sum), from a separate kernel with the fused
+ *              kernel's arithmetic;
+ *   W_out      W = (I + A)^-1 Diag(beta) K e^{G}, as stored for the state pass (bf16 values);
+ *   U_out      U = (I + A)^-1 Diag(beta) V, likewise;
+ *   delta_out  delta = U - W S_in, the chunk's state-independent correction, as
+ *              the state pass consumes it (bf16 values), S_in the state entering
+ *              the chunk.
+ * A debugging and test aid with no counterpart in the pages: it exposes the
+ * stages of the chunked form that section 3.3 describes, so that each can be
+ * compared with a plain chunkwise computation.  Sequences are never split.
+ */
+kda_status kda_prefill_debug(const void *q, const void *k, const void *v, const void *z,
+                             const float *A, const float *beta,
+                             const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                             int32_t num_seqs, int32_t total_tokens, int32_t H, int32_t dk,
+                             int32_t dv, kda_dtype dt, const float *initial_state,
+                             float *final_state, void *o, void *workspace,
+                             size_t workspace_bytes, float *G_out, float *W_out, float *U_out,
+                             float *delta_out, void *stream);
+
+/*
  * Rows of the checkpoint tensor for these HOST offsets: sum over sequences of
  * L_n / checkpoint_every.  Returns -1 for invalid arguments (NULL offsets with
  * num_seqs > 0, checkpoint_every not a positive multiple of 64, decreasing
@@ -287,6 +316,14 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
                            int32_t dk, int32_t dv, kda_dtype dt, float *state,
                            int32_t pool_size, const int32_t *slots, void *o,
                            void *stream);
+
+/*
+ * Optional host-side check of a decode batch's slots (a HOST copy): KDA_OK when
+ * every slot lies in [0, pool_size) and no two batch rows share one, else
+ * KDA_ERR_INVALID_ARG.  kda_decode_step does not make this check itself (it
+ * would need the slots on the host); two rows sharing a slot race on it.
+ */
+kda_status kda_decode_check_slots(const int32_t *slots_host, int32_t B, int32_t pool_size);
 
 /*
  * kda_decode_step with a choice of gate (kda_gate, as for kda_prefill_gated; the

@@ -10,7 +10,8 @@ from __future__ import annotations
 __all__ = ["kda_prefill", "kda_decode_step", "kda_prefill_workspace_size",
            "kda_status_string", "library_path", "KdaError", "kda_prefill_kernel_count",
            "kda_device_status", "kda_prefill_noalloc", "kda_prefill_checkpointed",
-           "kda_checkpoint_count", "kda_decode_multi", "kda_prefill_segments"]
+           "kda_checkpoint_count", "kda_decode_multi", "kda_prefill_segments",
+           "kda_prefill_debug", "kda_decode_check_slots"]
 
 
 def __getattr__(name):

@@ -40,6 +40,8 @@ SIGNATURES = {
     "kda_decode_step": ([_P] * 6 + [_I32] * 5 + [_P, _I32, _P, _P, _P], _I32),
     "kda_decode_step_gated": ([_P] * 6 + [_I32] * 5 + [_P, _I32, _P, _P, _I32, _P], _I32),
     "kda_prefill_gated": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _I32, _I32, _P], _I32),
+    "kda_prefill_debug": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ] + [_P] * 5, _I32),
+    "kda_decode_check_slots": ([_P, _I32, _I32], _I32),
     "kda_device_status": ([_P, _P], _I32),
     "kda_decode_multi": ([_P] * 6 + [_I32] * 6 + [_P, _I32, _P, _P, _I32, _P, _P], _I32),
     "kda_selftest_wait_timeout": ([ctypes.c_int64, _P], _I32),
@@ -299,3 +301,37 @@ def kda_device_status(stream=None) -> int:
     out = ctypes.c_int32(0)
     _check(_lib.kda_device_status(_stream_ptr(stream), ctypes.byref(out)), "kda_device_status")
     return int(out.value)
+
+
+def kda_prefill_debug(q, k, v, z, A, beta, cu_seqlens, cu_seqlens_host, initial_state=None,
+                      stream=None):
+    """Tensor-core prefill plus its stage intermediates; returns a dict with o,
+    final_state and G, W, U, delta (fp32 [T, H, 128], see include/kda.h)."""
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = cu_seqlens.shape[0] - 1
+    dt = q.dtype
+    dev = q.device
+    out = {"o": torch.empty(T, H, dv, dtype=dt, device=dev),
+           "final_state": torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)}
+    for name, d in (("G", dk), ("W", dk), ("U", dv), ("delta", dv)):
+        out[name] = torch.full((T, H, d), float("nan"), dtype=torch.float32, device=dev)
+    need = kda_prefill_workspace_size(T, N, H, dk, dv, dt, "tensor_core")
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    ch = cu_seqlens_host.to(torch.int32).contiguous()
+    code = _lib.kda_prefill_debug(
+        _dev(q, "q", dt), _dev(k, "k", dt), _dev(v, "v", dt), _dev(z, "z", dt),
+        _dev(A, "A", torch.float32), _dev(beta, "beta", torch.float32),
+        _dev(cu_seqlens, "cu_seqlens", torch.int32), ctypes.c_void_p(ch.data_ptr()), N, T, H, dk,
+        dv, KDA_DTYPE[dt], _dev(initial_state, "initial_state", torch.float32),
+        _dev(out["final_state"], "final_state", torch.float32), _dev(out["o"], "o", dt),
+        _dev(ws, "workspace"), need, _dev(out["G"], "G"), _dev(out["W"], "W"), _dev(out["U"], "U"),
+        _dev(out["delta"], "delta"), _stream_ptr(stream))
+    _check(code, "kda_prefill_debug")
+    return out
+
+
+def kda_decode_check_slots(slots_host, pool_size: int) -> bool:
+    """True when the host slots are in range and distinct (kda_decode_check_slots)."""
+    sl = torch.as_tensor(slots_host, dtype=torch.int32).contiguous()
+    return _lib.kda_decode_check_slots(ctypes.c_void_p(sl.data_ptr()), sl.numel(), pool_size) == 0

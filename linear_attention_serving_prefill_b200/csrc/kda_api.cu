@@ -2,6 +2,7 @@
 // dispatch to the kernels.  Nothing here allocates device memory; every call is
 // asynchronous on the caller's stream.
 #include <mutex>
+#include <vector>
 #include <stdint.h>
 #include <string.h>
 
@@ -130,7 +131,8 @@ kda_status prefill_impl(const void *q, const void *k, const void *v, const void 
                         const float *initial_state, float *final_state, void *o, void *workspace,
                         size_t workspace_bytes, kda_algo algo, void *stream,
                         void *const *stage_events, int32_t num_stage_events,
-                        int32_t checkpoint_every, float *checkpoints, kda_gate gate)
+                        int32_t checkpoint_every, float *checkpoints, kda_gate gate,
+                        float *const *dbg = nullptr)
 {
     kda_status st = check_prefill_sizes(total_tokens, num_seqs, H, dk, dv, dt, algo);
     if (st != KDA_OK) return st;
@@ -178,6 +180,9 @@ kda_status prefill_impl(const void *q, const void *k, const void *v, const void 
     // sequence whole (its workspace, sized for a split, is large enough).
     a.segments = checkpoint_every > 0 ? 1 : segments_for(total_tokens, num_seqs, H, dk, dv, dt, algo);
     a.gate = gate == KDA_GATE_SOFTPLUS ? 1 : 0;
+    if (dbg) {
+        a.dbg_G = dbg[0]; a.dbg_W = dbg[1]; a.dbg_U = dbg[2]; a.dbg_delta = dbg[3];
+    }
 
     cudaError_t err = use_tensor_core(dk, dv, dt, algo)
                           ? kda::launch_prefill_tensor_core(a, (cudaStream_t)stream)
@@ -199,6 +204,43 @@ extern "C" kda_status kda_prefill_checkpointed(
                         total_tokens, H, dk, dv, dt, initial_state, final_state, o, workspace,
                         workspace_bytes, algo, stream, stage_events, num_stage_events,
                         checkpoint_every, checkpoints, KDA_GATE_LOWER_BOUNDED);
+}
+
+extern "C" kda_status kda_prefill_debug(const void *q, const void *k, const void *v, const void *z,
+                                        const float *A, const float *beta,
+                                        const int32_t *cu_seqlens_dev,
+                                        const int32_t *cu_seqlens_host, int32_t num_seqs,
+                                        int32_t total_tokens, int32_t H, int32_t dk, int32_t dv,
+                                        kda_dtype dt, const float *initial_state,
+                                        float *final_state, void *o, void *workspace,
+                                        size_t workspace_bytes, float *G_out, float *W_out,
+                                        float *U_out, float *delta_out, void *stream)
+{
+    if (dt != KDA_DTYPE_BF16 || dk != 128 || dv != 128) {
+        const kda_status st = check_prefill_sizes(total_tokens, num_seqs, H, dk, dv, dt,
+                                                  KDA_ALGO_TENSOR_CORE);
+        return st != KDA_OK ? st : KDA_ERR_UNSUPPORTED;
+    }
+    for (const float *p : {(const float *)G_out, (const float *)W_out, (const float *)U_out,
+                           (const float *)delta_out})
+        if (p && !aligned(p, 16)) return KDA_ERR_INVALID_ARG;
+    float *const dbg[4] = {G_out, W_out, U_out, delta_out};
+    return prefill_impl(q, k, v, z, A, beta, cu_seqlens_dev, cu_seqlens_host, num_seqs,
+                        total_tokens, H, dk, dv, dt, initial_state, final_state, o, workspace,
+                        workspace_bytes, KDA_ALGO_TENSOR_CORE, stream, nullptr, 0, 0, nullptr,
+                        KDA_GATE_LOWER_BOUNDED, dbg);
+}
+
+extern "C" kda_status kda_decode_check_slots(const int32_t *slots_host, int32_t B, int32_t pool_size)
+{
+    if (B < 0 || pool_size < 0 || (B > 0 && !slots_host)) return KDA_ERR_INVALID_ARG;
+    std::vector<uint8_t> seen((size_t)pool_size, 0);
+    for (int32_t b = 0; b < B; ++b) {
+        const int32_t sl = slots_host[b];
+        if (sl < 0 || sl >= pool_size || seen[(size_t)sl]) return KDA_ERR_INVALID_ARG;
+        seen[(size_t)sl] = 1;
+    }
+    return KDA_OK;
 }
 
 extern "C" kda_status kda_prefill_gated(const void *q, const void *k, const void *v, const void *z,

@@ -25,6 +25,8 @@ struct PrefillArgs {
     float *checkpoints;             // [count, H, dk, dv] or nullptr
     int32_t segments;               // tensor-core path: segments per sequence (1 = no split)
     int32_t gate = 0;               // 0 = K3 lower-bounded gate, 1 = unbounded -softplus
+    // Debug dumps of the tensor-core path's stages (fp32 [T, H, 128]; nullptr = none).
+    float *dbg_G = nullptr, *dbg_W = nullptr, *dbg_U = nullptr, *dbg_delta = nullptr;
     void *const *events;            // optional cudaEvent_t per kernel boundary
     int32_t num_events;
     // Records boundary i (0 = before the first kernel) when the caller asked for it.

@@ -688,7 +688,8 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
              const uint8_t *__restrict__ blocks, int64_t max_chunks,
              const float *S0user, float *Sfuser, __nv_bfloat16 *__restrict__ o, int32_t *status,
              int ckpt_every, const int32_t *__restrict__ ckpt_off, float *__restrict__ ckpts,
-             int G, float *__restrict__ Sx, float *__restrict__ Mx, uint8_t *__restrict__ Eimg)
+             int G, float *__restrict__ Sx, float *__restrict__ Mx, uint8_t *__restrict__ Eimg,
+             float *__restrict__ dbg_delta)
 {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
@@ -903,6 +904,17 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
                     }
                 }
                 tmem_st16(tmem_addr(tb, lq, kTDl + 16 * hh), dl);
+                if (dbg_delta) {
+                    // Debug dump: delta as the products consume it (bf16), per token.
+                    const int t0c = tbeg + c * kChunk, lenc = min(kChunk, tend - t0c);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int r = 32 * hh + i;
+                        const uint32_t pr = dl[i >> 1];
+                        const float dv = __uint_as_float((i & 1) ? (pr & 0xFFFF0000u) : (pr << 16));
+                        if (r < lenc) dbg_delta[((size_t)(t0c + r) * H + h) * kDV + j] = dv;
+                    }
+                }
                 tmem_st_wait();
             }
             tc_fence_before_sync();
@@ -1179,6 +1191,50 @@ correct_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk
     if (warp == 0) tmem_dealloc(tb, 128);
 }
 
+// ------------------------------------------------------------------ debug --
+
+// Stage a1 on its own: G[t,h,c] = the inclusive cumulative gate of its 64-token
+// chunk (chunks aligned to each sequence start), with the intra kernel's gate
+// arithmetic.  One CTA of 128 threads (channels) per (chunk, head).
+__global__ void __launch_bounds__(128)
+debug_gate_kernel(const __nv_bfloat16 *__restrict__ z, const float *__restrict__ A,
+                  const int2 *__restrict__ chunk_loc, const int32_t *__restrict__ chunk_off, int N,
+                  int H, float *__restrict__ Gout)
+{
+    const int h = blockIdx.x % H, g = blockIdx.x / H;
+    if (g >= chunk_off[N]) return;
+    const int2 loc = chunk_loc[g];
+    const int c = threadIdx.x;
+    const float eA = __expf(A[(size_t)h * kDK + c]);
+    float acc = 0.f;
+    for (int r = 0; r < loc.y; ++r) {
+        const size_t idx = ((size_t)(loc.x + r) * H + h) * kDK + c;
+        acc += gate_log_decay_fast(eA, __bfloat162float(z[idx]));
+        Gout[idx] = acc;
+    }
+}
+
+// Stage a2's outputs read back from the per-(chunk, head) blocks: W (rows 0..63 of
+// the [W; Qt] image) and U, as fp32 [T, H, 128].
+__global__ void __launch_bounds__(256)
+debug_unpack_kernel(const uint8_t *__restrict__ blocks, int64_t max_chunks,
+                    const int2 *__restrict__ chunk_loc, const int32_t *__restrict__ chunk_off, int N,
+                    int H, float *__restrict__ Wout, float *__restrict__ Uout)
+{
+    const int h = blockIdx.x % H, g = blockIdx.x / H;
+    if (g >= chunk_off[N]) return;
+    const int2 loc = chunk_loc[g];
+    const uint8_t *blk = blocks + ((size_t)h * max_chunks + g) * kBlockBytes;
+    for (int e = threadIdx.x; e < loc.y * kDK; e += 256) {
+        const int r = e / kDK, c = e % kDK;
+        const size_t idx = ((size_t)(loc.x + r) * H + h) * kDK + c;
+        if (Wout)
+            Wout[idx] = __bfloat162float(*(const __nv_bfloat16 *)(blk + kOffWQ + sw128_offset(r, c, 128)));
+        if (Uout)
+            Uout[idx] = __bfloat162float(((const __nv_bfloat16 *)(blk + kOffU))[r * kDV + c]);
+    }
+}
+
 // cuTensorMapEncodeTiled, fetched from the driver through the runtime (no
 // link-time dependency on libcuda).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
@@ -1338,10 +1394,21 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
                    stream>>>(
         a.cu_seqlens, chunk_off, order, a.num_seqs, a.H, blocks, max_chunks, a.initial_state,
         a.final_state, (__nv_bfloat16 *)a.o, a.status, a.ckpt_every, ckpt_off, a.checkpoints,
-        G, Sx, Mx, Eimg);
+        G, Sx, Mx, Eimg, a.dbg_delta);
     a.mark(3, stream);
     err = cudaGetLastError();
-    if (err != cudaSuccess || G == 1) return err;
+    if (err != cudaSuccess) return err;
+    if (max_chunks > 0 && a.dbg_G) {
+        debug_gate_kernel<<<(unsigned)(max_chunks * a.H), 128, 0, stream>>>(
+            (const __nv_bfloat16 *)a.z, a.A, chunk_loc, chunk_off, a.num_seqs, a.H, a.dbg_G);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    if (max_chunks > 0 && (a.dbg_W || a.dbg_U)) {
+        debug_unpack_kernel<<<(unsigned)(max_chunks * a.H), 256, 0, stream>>>(
+            blocks, max_chunks, chunk_loc, chunk_off, a.num_seqs, a.H, a.dbg_W, a.dbg_U);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    if (G == 1) return cudaSuccess;
 
     compose_kernel<<<(unsigned)((int64_t)a.num_seqs * a.H * (kDV / kComposeCols)), kComposeThreads,
                      kComposeSmem, stream>>>(chunk_off, a.H, G, Sx, Mx, Simg, a.final_state);

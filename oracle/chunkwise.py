@@ -117,3 +117,46 @@ def prefill(q, k, v, z, A, beta, cu_seqlens, initial_state=None, chunk: int = 16
                 o[c0:c1, h] = O
             sf[i, h] = S
     return o, sf
+
+
+def chunk_intermediates(q, k, v, g, beta, S0):
+    """The stage values of ``chunk_step`` for one chunk of one head: G [C,dk], the
+    strictly lower A [C,C], W = T Diag(beta) Kt [C,dk], U = T Diag(beta) V [C,dv],
+    D = U - W S0 [C,dv] (the state-independent part of the update), O, S_out."""
+    C = q.shape[0]
+    G = np.cumsum(g, axis=0)
+    Kt, Kh, Qt = k * np.exp(G), k * np.exp(-G), q * np.exp(G)
+    A = np.tril(beta[:, None] * (Kt @ Kh.T), -1)
+    Tinv = np.linalg.inv(np.eye(C) + A)
+    W = Tinv @ (beta[:, None] * Kt)
+    U = Tinv @ (beta[:, None] * v)
+    D = U - W @ S0
+    O = Qt @ S0 + np.tril(Qt @ Kh.T) @ D
+    S_out = np.exp(G[-1])[:, None] * S0 + (k * np.exp(G[-1] - G)).T @ D
+    return dict(G=G, A=A, W=W, U=U, D=D, O=O, S_out=S_out)
+
+
+def prefill_intermediates(q, k, v, z, A, beta, cu_seqlens, initial_state=None, chunk: int = 64):
+    """Per-token stage values over packed sequences, chunks aligned to each
+    sequence start: G, W [T,H,dk]; U, D [T,H,dv]; plus o and the final states."""
+    q, k, v, z, A, beta = (np.asarray(t, dtype=np.float64) for t in (q, k, v, z, A, beta))
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    n = cu.shape[0] - 1
+    out = dict(G=np.zeros((T, H, dk)), W=np.zeros((T, H, dk)), U=np.zeros((T, H, dv)),
+               D=np.zeros((T, H, dv)), o=np.zeros((T, H, dv)), final_state=np.zeros((n, H, dk, dv)))
+    for i in range(n):
+        for h in range(H):
+            S = (np.zeros((dk, dv)) if initial_state is None
+                 else np.asarray(initial_state[i, h], dtype=np.float64).copy())
+            for c0 in range(int(cu[i]), int(cu[i + 1]), chunk):
+                c1 = min(c0 + chunk, int(cu[i + 1]))
+                r = chunk_intermediates(q[c0:c1, h], k[c0:c1, h], v[c0:c1, h], _gate(z[c0:c1, h], A[h]),
+                                        beta[c0:c1, h], S)
+                for key in ("G", "W", "U", "D"):
+                    out[key][c0:c1, h] = r[key]
+                out["o"][c0:c1, h] = r["O"]
+                S = r["S_out"]
+            out["final_state"][i, h] = S
+    return out

@@ -262,3 +262,25 @@ def test_gated_entry_points_validate_the_gate():
     dec = B._lib.kda_decode_step_gated(_fake(), _fake(), _fake(), _fake(), _fake(), _fake(), 2, 2,
                                        128, 128, BF16, _fake(), 2, None, _fake(), 3, None)
     assert dec == INVALID
+
+
+def test_decode_slot_check_and_debug_validation():
+    ok = (ctypes.c_int32 * 4)(3, 0, 2, 1)
+    dup = (ctypes.c_int32 * 3)(0, 2, 2)
+    oor = (ctypes.c_int32 * 2)(0, 4)
+    chk = B._lib.kda_decode_check_slots
+    assert chk(ctypes.cast(ok, ctypes.c_void_p), 4, 4) == OK
+    assert chk(ctypes.cast(dup, ctypes.c_void_p), 3, 4) == INVALID
+    assert chk(ctypes.cast(oor, ctypes.c_void_p), 2, 4) == INVALID
+    assert chk(None, 2, 4) == INVALID
+    assert chk(None, 0, 4) == OK
+    assert B.kda_decode_check_slots([1, 0], 2) and not B.kda_decode_check_slots([1, 1], 2)
+
+    def dbg(dt=BF16, dk=128, G=None):
+        return B._lib.kda_prefill_debug(_fake(), _fake(), _fake(), _fake(), _fake(), _fake(), _fake(),
+                                        None, 2, 10, 4, dk, 128, dt, None, None, _fake(), None, 0,
+                                        G, None, None, None, None)
+    assert dbg(dt=F32) == UNSUPPORTED
+    assert dbg(dk=64) == UNSUPPORTED
+    assert dbg(dk=96) == UNSUPPORTED
+    assert dbg(G=_fake(0x10004)) == INVALID

@@ -458,3 +458,24 @@ def test_softplus_decode_continues_prefill():
                                 x["beta"][8:9], s8, gate="softplus")
     np.testing.assert_allclose(od[0], o[8], rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(sd, sf, rtol=1e-12, atol=1e-14)
+
+
+# ------------------------------------------- stage intermediates (debug dumps) ----
+
+def test_chunk_intermediates_satisfy_their_definitions():
+    """W and U solve (I + A) W = Diag(beta) Kt and (I + A) U = Diag(beta) V (checked
+    by multiplication, not by another inverse); D = U - W S0; and the stages put
+    together give the recurrence's outputs and final state."""
+    x = _inputs([70, 64, 9], H=2, dk=6, dv=5, seed=16)
+    ref_o, ref_s = oracle.prefill(**x)
+    got = chunkwise.prefill_intermediates(**x, chunk=64)
+    assert _relerr(got["o"], ref_o) < 1e-11 and _relerr(got["final_state"], ref_s) < 1e-11
+    q, k, v, b = x["q"][:64, 0], x["k"][:64, 0], x["v"][:64, 0], x["beta"][:64, 0]
+    g = oracle.gate(x["z"][:64], x["A"])[:, 0]
+    r = chunkwise.chunk_intermediates(q, k, v, g, b, x["initial_state"][0, 0])
+    G = np.cumsum(g, axis=0)
+    np.testing.assert_allclose(r["G"], G, rtol=1e-13)
+    M = np.eye(64) + r["A"]
+    np.testing.assert_allclose(M @ r["W"], b[:, None] * k * np.exp(G), rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(M @ r["U"], b[:, None] * v, rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(r["D"], r["U"] - r["W"] @ x["initial_state"][0, 0], rtol=1e-12, atol=1e-14)

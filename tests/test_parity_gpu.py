@@ -243,6 +243,31 @@ def test_auto_with_checkpoints_keeps_sequences_whole():
     assert relerr(to_np(got[1]), ref_S) <= TOL_BF16
 
 
+# ------------------------------------------------ stage intermediates ----
+
+def test_stage_intermediates_match_the_chunkwise_form():
+    """The debug entry point's dumps of the fused stages, each against the fp64
+    chunkwise form at the tensor-core path's 64-token chunks: a1 G (fp32), a2 W
+    and U, a3 delta = U - W S_in (bf16 values) -- and the dumps change nothing."""
+    from oracle import chunkwise
+    lengths = [1, 63, 64, 65, 130, 200]
+    x = _cuda(prefill_inputs(lengths, 2, 128, 128, "bf16", seed=90, s0_std=0.05))
+    d = K.kda_prefill_debug(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"], x["cu_seqlens"],
+                            x["cu_seqlens_host"], initial_state=x["initial_state"])
+    o_plain, S_plain = _run(x, "tensor_core")
+    torch.cuda.synchronize()
+    assert torch.equal(d["o"], o_plain) and torch.equal(d["final_state"], S_plain)
+    ref = chunkwise.prefill_intermediates(*(to_np(x[key]) for key in ("q", "k", "v", "z", "A", "beta")),
+                                          x["cu_seqlens_host"].numpy(), to_np(x["initial_state"]), chunk=64)
+    for key, dkey, tol in (("G", "G", 1e-5), ("W", "W", TOL_BF16), ("U", "U", TOL_BF16),
+                           ("delta", "D", TOL_BF16)):
+        got = to_np(d[key])
+        assert np.isfinite(got).all(), key
+        assert relerr(got, ref[dkey]) <= tol, (key, relerr(got, ref[dkey]))
+    assert relerr(to_np(d["o"]), ref["o"]) <= TOL_BF16
+    assert relerr(to_np(d["final_state"]), ref["final_state"]) <= TOL_BF16
+
+
 # ------------------------------------------------------- plan edge cases ----
 
 @pytest.mark.parametrize("algo", ["tensor_core", "tensor_core_split"])
