@@ -682,6 +682,9 @@ constexpr uint32_t kEImg = kChunk * kDK * 2;    // E image of one (chunk, head):
 constexpr uint32_t kSinImg = kDV * kDK * 2;     // S_in image of one (segment, head): 32 KiB
 constexpr size_t kStateF32 = (size_t)kDK * kDV;  // one fp32 state, in floats
 
+// DUMP: the debug variant that also writes delta (dbg_delta); the production
+// instantiation has no trace of it.
+template <bool DUMP>
 __global__ void __launch_bounds__(kStateThreads, 1)
 state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_off,
              const int32_t *__restrict__ order, int N, int H,
@@ -904,7 +907,7 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
                     }
                 }
                 tmem_st16(tmem_addr(tb, lq, kTDl + 16 * hh), dl);
-                if (dbg_delta) {
+                if (DUMP) {
                     // Debug dump: delta as the products consume it (bf16), per token.
                     const int t0c = tbeg + c * kChunk, lenc = min(kChunk, tend - t0c);
 #pragma unroll
@@ -1354,8 +1357,8 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
     err = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                (int)cudaSharedmemCarveoutMaxShared);
     if (err != cudaSuccess) return err;
-    err = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)kStateSmem);
+    auto state_fn = a.dbg_delta ? state_kernel<true> : state_kernel<false>;
+    err = cudaFuncSetAttribute(state_fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem);
     if (err != cudaSuccess) return err;
     if (G > 1) {
         err = cudaFuncSetAttribute(compose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1390,8 +1393,8 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
         if (err != cudaSuccess) return err;
     }
     a.mark(2, stream);
-    state_kernel<<<(unsigned)((int64_t)a.num_seqs * a.H * (2 * G - 1)), kStateThreads, kStateSmem,
-                   stream>>>(
+    state_fn<<<(unsigned)((int64_t)a.num_seqs * a.H * (2 * G - 1)), kStateThreads, kStateSmem,
+               stream>>>(
         a.cu_seqlens, chunk_off, order, a.num_seqs, a.H, blocks, max_chunks, a.initial_state,
         a.final_state, (__nv_bfloat16 *)a.o, a.status, a.ckpt_every, ckpt_off, a.checkpoints,
         G, Sx, Mx, Eimg, a.dbg_delta);
