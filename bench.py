@@ -122,9 +122,16 @@ class ClockSampler:
 
 
 def _source_sha(name: str) -> str:
+    """sha256 prefix of a kernel source with its comments and blank lines removed,
+    so that an edit of comments alone keeps a traffic record valid."""
+    import re
     path = os.path.join(ROOT, "linear_attention_serving_prefill_b200", "csrc", name)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    with open(path) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def _traffic(kernel_file: str, kernel: str, units: int):

@@ -7,10 +7,12 @@
 // log-decay in (-80, 0), so the reciprocal factors stay below e^80 and the
 // diagonal tiles use the same dense matrix multiply as the off-diagonal ones).
 //
-// Three launches per call:
-//   1. plan:   per-sequence chunk offsets and a longest-first order.
-//   2. intra:  persistent, one CTA per SM over the (64-token chunk, head) items.  Gate and cumulative
-//              log-decay G in fp32, then on the tensor cores
+// Three launches per call (five when sequences are split into segments):
+//   1. plan:   per-sequence chunk offsets, a per-chunk (first token, length)
+//              table and a longest-first order.
+//   2. intra:  persistent, two CTAs of 256 threads per SM over the (64-token
+//              chunk, head) items.  Gate and cumulative log-decay G in fp32, then
+//              on the tensor cores
 //                A = strictly_lower(Diag(beta) Kt Kh^T), P = lower(Qt Kh^T)
 //              (16-token sub-tiles, each with its own reference point), the
 //              unit-lower inverse T = (I + A)^-1 on CUDA cores in fp32, and
@@ -26,6 +28,9 @@
 //                O^T  = D[:, 64:] + Dl^T P^T       -> o
 //              Bulk copies stream the per-chunk blocks through a two-stage
 //              shared-memory ring.
+//   4. compose and 5. correct (sequence split only): the affine scan over a
+//              sequence's segments and the output correction o += E S_in.
+//   (kda_prefill_debug adds a stand-alone gate kernel and a block unpacker.)
 //
 // Within a chunk (tokens r, s; G inclusive from the chunk start):
 //   Dl = (I + A)^-1 Diag(beta) (V - Kt S_in) = U - W S_in,
