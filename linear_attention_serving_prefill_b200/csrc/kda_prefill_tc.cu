@@ -309,6 +309,7 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 sAbort = 1;
             }
             compute_sync();  // beta and A (landed by warp 0's cp.async) are visible
+            tc_fence_after_sync();  // the previous item's TMEM reads precede this item's writes
             const IntraItem inf = info;
             const int len = inf.len, h = inf.h;
             uint8_t *blk = blocks + ((size_t)h * max_chunks + inf.g) * kBlockBytes;
@@ -321,9 +322,13 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             }
 
             // Pass 1: gate of channels c0, c0 + 1 summed over the sub-tile's 16 rows.
-            // (Pass 2 forms the running sums L_r = G_r - m_I again from z, in the
-            // same order, instead of holding them in registers.)
+            // Each row's running sum L_r = G_r - m_I is parked in TMEM for pass 2
+            // (lane 32 (warp % 4) + lane, 32 columns from 128 + 32 (warp / 4)); those
+            // columns are free from the previous item's W/U readback until this
+            // item's W/U product, and registers are not.
+            const uint32_t lcol = tmem_addr(tb, 32 * (warp & 3), 128 + 32 * (warp >> 2));
             float2 acc = make_float2(0.f, 0.f);
+            float lst[8];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int r = 16 * I + i;
@@ -332,7 +337,11 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                     acc.x += gate_log_decay_fast(eA.x, zz.x);
                     acc.y += gate_log_decay_fast(eA.y, zz.y);
                 }
+                lst[2 * (i & 3)] = acc.x;
+                lst[2 * (i & 3) + 1] = acc.y;
+                if ((i & 3) == 3) tmem_st8(lcol + 8 * (i >> 2), lst);
             }
+            tmem_st_wait();
             sTot[I][c0] = acc.x;
             sTot[I][c0 + 1] = acc.y;
             compute_sync();
@@ -355,23 +364,24 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 fac[Ip] = Ip > I ? make_float2(__expf(mref[Ip].x - mI.x), __expf(mref[Ip].y - mI.y))
                                  : make_float2(1.f, 1.f);
 
-            // Pass 2: scaled operands of channels c0, c0 + 1 for the 16 rows.
+            // Pass 2: scaled operands of channels c0, c0 + 1 for the 16 rows, with L
+            // read back from TMEM four rows at a time.
             // Kt = k e^{L} and Qt = q e^{L} replace k and q in place (same thread,
             // same address); the rest goes to R, to the block, or into registers.
             // beta K e^G, beta V and K e^{G_C - G} wait in registers until the tiles
             // that receive them are no longer read.
             uint32_t pk0[8], pk1[8], pv0[8], pv1[8], kd0[8], kd1[8];
-            float2 Lr = make_float2(0.f, 0.f);  // L of the current row
+            float lrd[8];  // L of four rows, from pass 1
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int r = 16 * I + i;
                 const bool valid = r < len;
                 const uint32_t off = sw128_offset(r, c0, 64);
-                if (valid) {
-                    const float2 zz = ld_bf16x2_smem(sm, kRawZ + off);
-                    Lr.x += gate_log_decay_fast(eA.x, zz.x);
-                    Lr.y += gate_log_decay_fast(eA.y, zz.y);
+                if ((i & 3) == 0) {
+                    tmem_ld8(lcol + 8 * (i >> 2), lrd);
+                    tmem_ld_wait();
                 }
+                const float2 Lr = make_float2(lrd[2 * (i & 3)], lrd[2 * (i & 3) + 1]);
                 const float2 kv = valid ? ld_bf16x2_smem(sm, kRawK + off) : make_float2(0.f, 0.f);
                 const float2 qv = valid ? ld_bf16x2_smem(sm, kRawQ + off) : make_float2(0.f, 0.f);
                 const float2 vv = valid ? ld_bf16x2_smem(sm, kRawV + off) : make_float2(0.f, 0.f);
@@ -452,23 +462,19 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 // M = 64 layout: TMEM lane 32 q + i holds row 16 q + i (i < 16).  Warp w:
                 // lane quarter q = w % 4, sub-tiles 2 (w / 4) and 2 (w / 4) + 1.
                 const int q = warp & 3, hb = warp >> 2;
+                // Half-warp u = lane / 16 takes sub-tile 2 hb + u.
+                const int Ia = 2 * hb + (lane >> 4);
+                uint32_t rr[32];
+                tmem_ld16x2_32(tmem_addr(tb, 32 * q, 64 * hb), rr);
+                tmem_ld_wait();
+                const int sidx = 16 * q + (lane & 15);
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int Ia = 2 * hb + u;
-                    uint32_t rr[32];
-                    tmem_ld32(tmem_addr(tb, 32 * q, 32 * Ia), rr);
-                    tmem_ld_wait();
-                    if (lane < 16) {
-                        const int sidx = 16 * q + lane;
-#pragma unroll
-                        for (int jr = 0; jr < 16; ++jr) {
-                            const int r = 16 * Ia + jr;
-                            Af[r * kLd + sidx] = sidx < r ? sBeta[r] * __uint_as_float(rr[jr]) : 0.f;
-                            const float pvv = sidx <= r ? __uint_as_float(rr[16 + jr]) : 0.f;
-                            *(__nv_bfloat16 *)(sm + kRawK + 8192 + sw128_offset(r, sidx, 64)) =
-                                __float2bfloat16_rn(pvv);
-                        }
-                    }
+                for (int jr = 0; jr < 16; ++jr) {
+                    const int r = 16 * Ia + jr;
+                    Af[r * kLd + sidx] = sidx < r ? sBeta[r] * __uint_as_float(rr[jr]) : 0.f;
+                    const float pvv = sidx <= r ? __uint_as_float(rr[16 + jr]) : 0.f;
+                    *(__nv_bfloat16 *)(sm + kRawK + 8192 + sw128_offset(r, sidx, 64)) =
+                        __float2bfloat16_rn(pvv);
                 }
             }
             // (K e^{G_C - G})^T staged in the q tile (Qt is no longer read) as the
@@ -610,26 +616,24 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 // Rows r = 16 q + i (i < 16) of lane quarter q = w % 4; warps 0-3 read W
                 // (columns 0..127) into rows 0..63 of the block's [W; Qt] image, warps
                 // 4-7 read U (columns 128..255) into its row-major block region.
-                const int q = warp & 3, hb = warp >> 2, r = 16 * q + lane;
+                const int q = warp & 3, hb = warp >> 2, r = 16 * q + (lane & 15);
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
+                for (int j = 0; j < 2; ++j) {
                     uint32_t rr[32];
-                    tmem_ld32(tmem_addr(tb, 32 * q, 128 * hb + 32 * q4), rr);
+                    tmem_ld16x2_32(tmem_addr(tb, 32 * q, 128 * hb + 64 * j), rr);
                     tmem_ld_wait();
-                    if (lane < 16) {
 #pragma unroll
-                        for (int cc = 0; cc < 32; cc += 8) {
-                            const uint4 w4 = make_uint4(
-                                pack_bf16(__uint_as_float(rr[cc]), __uint_as_float(rr[cc + 1])),
-                                pack_bf16(__uint_as_float(rr[cc + 2]), __uint_as_float(rr[cc + 3])),
-                                pack_bf16(__uint_as_float(rr[cc + 4]), __uint_as_float(rr[cc + 5])),
-                                pack_bf16(__uint_as_float(rr[cc + 6]), __uint_as_float(rr[cc + 7])));
-                            const int col = 32 * q4 + cc;
-                            if (hb == 0)
-                                *(uint4 *)(blk + kOffWQ + sw128_offset(r, col, 128)) = w4;
-                            else
-                                *(uint4 *)(blk + kOffU + (r * 128 + col) * 2) = w4;
-                        }
+                    for (int cc = 0; cc < 32; cc += 8) {
+                        const uint4 w4 = make_uint4(
+                            pack_bf16(__uint_as_float(rr[cc]), __uint_as_float(rr[cc + 1])),
+                            pack_bf16(__uint_as_float(rr[cc + 2]), __uint_as_float(rr[cc + 3])),
+                            pack_bf16(__uint_as_float(rr[cc + 4]), __uint_as_float(rr[cc + 5])),
+                            pack_bf16(__uint_as_float(rr[cc + 6]), __uint_as_float(rr[cc + 7])));
+                        const int col = 64 * j + 32 * (lane >> 4) + cc;
+                        if (hb == 0)
+                            *(uint4 *)(blk + kOffWQ + sw128_offset(r, col, 128)) = w4;
+                        else
+                            *(uint4 *)(blk + kOffU + (r * 128 + col) * 2) = w4;
                     }
                 }
             }
