@@ -615,7 +615,8 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             {
                 // Rows r = 16 q + i (i < 16) of lane quarter q = w % 4; warps 0-3 read W
                 // (columns 0..127) into rows 0..63 of the block's [W; Qt] image, warps
-                // 4-7 read U (columns 128..255) into its row-major block region.
+                // 4-7 read U (columns 128..255) into its row-major block region.  Each
+                // load covers 64 columns: 32 for each half-warp.
                 const int q = warp & 3, hb = warp >> 2, r = 16 * q + (lane & 15);
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
