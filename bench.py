@@ -121,17 +121,21 @@ class ClockSampler:
                 "samples": len(mine)}
 
 
-def _source_sha(name: str) -> str:
-    """sha256 prefix of a kernel source with its comments and blank lines removed,
-    so that an edit of comments alone keeps a traffic record valid."""
+def _code_sha(text: str) -> str:
+    """sha256 prefix of C/CUDA source text with its comments, trailing blanks and
+    blank lines removed, so that an edit of comments alone keeps the same key."""
     import re
-    path = os.path.join(ROOT, "linear_attention_serving_prefill_b200", "csrc", name)
-    with open(path) as f:
-        text = f.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     text = re.sub(r"//[^\n]*", "", text)
     code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
     return hashlib.sha256(code.encode()).hexdigest()[:16]
+
+
+def _source_sha(name: str) -> str:
+    """The `_code_sha` key of one kernel source file of the package."""
+    path = os.path.join(ROOT, "linear_attention_serving_prefill_b200", "csrc", name)
+    with open(path) as f:
+        return _code_sha(f.read())
 
 
 def _traffic(kernel_file: str, kernel: str, units: int):
