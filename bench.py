@@ -332,6 +332,74 @@ def gate_leg(K, rank_seed, rank, world, dev, stream, args, max_over_ranks, barri
     return out
 
 
+def decode_leg(K, rank, world, dev, stream, args, hbm_peak, barrier, batch=None):
+    """Decode step on B cached states (default the 256 x 96 workload), H=96,
+    updated in place: GB/s of state traffic over args.decode_steps steps, then
+    speculative verify / replay of 4 drafts on the same batch."""
+    from linear_attention_serving_prefill_b200.workloads import CONFIGS, decode_inputs
+    from dataclasses import replace
+    dcfg = CONFIGS["decode_256"]
+    if batch:
+        dcfg = replace(dcfg, B=batch, name=dcfg.name.replace("B=256", f"B={batch}"))
+    d = decode_inputs(dcfg.B, dcfg.H, dcfg.dk, dcfg.dv, dcfg.dtype, seed=rank_seed(dcfg.seed, rank),
+                      nsets=dcfg.nsets, device=dev)
+    od = torch.empty(dcfg.B, dcfg.H, dcfg.dv, dtype=torch.bfloat16, device=dev)
+
+    def dstep(i):
+        j = i % dcfg.nsets
+        K.kda_decode_step(d["q"][j], d["k"][j], d["v"][j], d["z"][j], d["A"], d["beta"][j],
+                          d["state"], None, o=od, stream=stream)
+
+    for i in range(args.warmup):
+        dstep(i)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.decode_steps):
+        dstep(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.decode_steps
+    state_bytes = 2 * dcfg.B * dcfg.H * dcfg.dk * dcfg.dv * 4
+    dgbs = state_bytes / (dms / 1e3) / 1e9
+    decode = {"config": dcfg.name, "ms_per_step": dms, "state_gbs": dgbs,
+              "frac_of_hbm": dgbs / hbm_peak, "steps": args.decode_steps,
+              "state_bytes_per_step": state_bytes, "gpu_launches": args.decode_steps}
+
+    # Speculative decoding on the same batch: verify 4 drafts per sequence (state
+    # read once, not written), then replay the accepted ones (here all 4).
+    Tq = 4
+    sq, sk, sv, sz = (d[key][:Tq].permute(1, 0, 2, 3).contiguous() for key in ("q", "k", "v", "z"))
+    sbeta = d["beta"][:Tq].permute(1, 0, 2).contiguous()
+    so = torch.empty(dcfg.B, Tq, dcfg.H, dcfg.dv, dtype=torch.bfloat16, device=dev)
+    for _ in range(args.warmup):
+        K.kda_decode_multi(sq, sk, sv, sz, d["A"], sbeta, d["state"], o=so, stream=stream)
+    torch.cuda.synchronize()
+    barrier()
+    reps = 50
+    e0.record(stream)
+    for _ in range(reps):
+        K.kda_decode_multi(sq, sk, sv, sz, d["A"], sbeta, d["state"], o=so, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    vms = max_over_ranks(e0.elapsed_time(e1), world, dev) / reps
+    e0.record(stream)
+    for _ in range(reps):
+        K.kda_decode_multi(sq, sk, sv, sz, d["A"], sbeta, d["state"], update_state=True,
+                           want_outputs=False, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    rms = max_over_ranks(e0.elapsed_time(e1), world, dev) / reps
+    decode["spec_verify"] = {"drafts": Tq, "ms": vms,
+                             "state_read_gbs": state_bytes / 2 / (vms / 1e3) / 1e9,
+                             "tokens_per_s": dcfg.B * Tq / (vms / 1e3)}
+    decode["spec_replay"] = {"accepted": Tq, "ms": rms,
+                             "state_gbs": state_bytes / (rms / 1e3) / 1e9}
+    del d, od, so
+    return decode
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -348,6 +416,10 @@ def main():
                     help="prefill_4k is the small case used for profiler captures")
     ap.add_argument("--prefill-only", action="store_true",
                     help="skip the decode, end-to-end and CPU legs (profiler captures)")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run the decode and speculative legs alone (profiler captures)")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="sequences of the decode legs (default: the 256-sequence workload)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
@@ -372,6 +444,16 @@ def main():
     def barrier():
         if world > 1:
             dist.barrier()
+
+    if args.decode_only:
+        hbm_peak = _peaks()[0]
+        decode = decode_leg(K, rank, world, dev, torch.cuda.current_stream(), args, hbm_peak,
+                            barrier, batch=args.decode_batch or None)
+        if rank == 0:
+            print(json.dumps({"decode": decode, "gpu": torch.cuda.get_device_name(dev)}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
 
     cfg = CONFIGS[args.workload]
     from dataclasses import replace
@@ -425,14 +507,22 @@ def main():
     hbm_peak, tc_peak, peak_src = _peaks()
     dom = max(range(nk), key=lambda j: per_kernel_ms[j])
     launch_ms = per_kernel_ms[dom]
-    alg_bytes = th * kernel_bytes_per_th[dom]
+    # The method's algorithmic bytes (1,284 per token-head: q, k, v, z, beta in,
+    # o out) over the dominant kernel's launch time.  The bytes that kernel
+    # moves by this design (its own reads plus the intermediate block it
+    # writes) are reported beside it under "own_bytes_*", not in "frac".
+    alg_bytes = th * BYTES_PER_TOKEN_HEAD
     achieved = alg_bytes / (launch_ms / 1e3) / 1e9
+    own_bytes = th * kernel_bytes_per_th[dom]
+    own_gbs = own_bytes / (launch_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak,
                 "traffic": _traffic(kernel_file, kernel_names[dom], th),
                 "kernel": kernel_names[dom], "peak_source": peak_src,
                 "algorithmic_bytes_per_launch": alg_bytes,
-                "algorithmic_bytes_per_token_head": kernel_bytes_per_th[dom],
+                "algorithmic_bytes_per_token_head": BYTES_PER_TOKEN_HEAD,
+                "own_bytes_per_token_head": kernel_bytes_per_th[dom],
+                "own_bytes_gbs": own_gbs, "own_bytes_frac": own_gbs / hbm_peak,
                 "kernels_ms": dict(zip(kernel_names, per_kernel_ms))}
     path_gbs = th * BYTES_PER_TOKEN_HEAD / (ms_per_step / 1e3) / 1e9
     path = {"bytes_per_token_head": BYTES_PER_TOKEN_HEAD, "achieved_gbs": path_gbs,
@@ -474,64 +564,7 @@ def main():
                 "extra_bytes_per_step": n_ck * H * dk * dv * 4}
         del ckbuf
 
-        # Decode step: B=256 cached states, H=96, updated in place; GB/s of state traffic.
-        dcfg = CONFIGS["decode_256"]
-        d = decode_inputs(dcfg.B, dcfg.H, dcfg.dk, dcfg.dv, dcfg.dtype, seed=rank_seed(dcfg.seed, rank),
-                          nsets=dcfg.nsets, device=dev)
-        od = torch.empty(dcfg.B, dcfg.H, dcfg.dv, dtype=torch.bfloat16, device=dev)
-
-        def dstep(i):
-            j = i % dcfg.nsets
-            K.kda_decode_step(d["q"][j], d["k"][j], d["v"][j], d["z"][j], d["A"], d["beta"][j],
-                              d["state"], None, o=od, stream=stream)
-
-        for i in range(args.warmup):
-            dstep(i)
-        torch.cuda.synchronize()
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(args.decode_steps):
-            dstep(i)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        dms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.decode_steps
-        state_bytes = 2 * dcfg.B * dcfg.H * dcfg.dk * dcfg.dv * 4
-        dgbs = state_bytes / (dms / 1e3) / 1e9
-        decode = {"config": dcfg.name, "ms_per_step": dms, "state_gbs": dgbs,
-                  "frac_of_hbm": dgbs / hbm_peak, "steps": args.decode_steps,
-                  "state_bytes_per_step": state_bytes, "gpu_launches": args.decode_steps}
-
-        # Speculative decoding on the same batch: verify 4 drafts per sequence (state
-        # read once, not written), then replay the accepted ones (here all 4).
-        Tq = 4
-        sq, sk, sv, sz = (d[key][:Tq].permute(1, 0, 2, 3).contiguous() for key in ("q", "k", "v", "z"))
-        sbeta = d["beta"][:Tq].permute(1, 0, 2).contiguous()
-        so = torch.empty(dcfg.B, Tq, dcfg.H, dcfg.dv, dtype=torch.bfloat16, device=dev)
-        for _ in range(args.warmup):
-            K.kda_decode_multi(sq, sk, sv, sz, d["A"], sbeta, d["state"], o=so, stream=stream)
-        torch.cuda.synchronize()
-        barrier()
-        reps = 50
-        e0.record(stream)
-        for _ in range(reps):
-            K.kda_decode_multi(sq, sk, sv, sz, d["A"], sbeta, d["state"], o=so, stream=stream)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        vms = max_over_ranks(e0.elapsed_time(e1), world, dev) / reps
-        e0.record(stream)
-        for _ in range(reps):
-            K.kda_decode_multi(sq, sk, sv, sz, d["A"], sbeta, d["state"], update_state=True,
-                               want_outputs=False, stream=stream)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        rms = max_over_ranks(e0.elapsed_time(e1), world, dev) / reps
-        decode["spec_verify"] = {"drafts": Tq, "ms": vms,
-                                 "state_read_gbs": state_bytes / 2 / (vms / 1e3) / 1e9,
-                                 "tokens_per_s": dcfg.B * Tq / (vms / 1e3)}
-        decode["spec_replay"] = {"accepted": Tq, "ms": rms,
-                                 "state_gbs": state_bytes / (rms / 1e3) / 1e9}
-        del d, od, so
+        decode = decode_leg(K, rank, world, dev, stream, args, hbm_peak, barrier)
 
         # End to end through the C ABI: pinned host inputs -> device, prefill, result ->
         # host, every byte of every step inside the timed region.  Steps are
