@@ -50,7 +50,7 @@
 extern "C" {
 #endif
 
-#define KDA_ABI_VERSION 2
+#define KDA_ABI_VERSION 3
 
 typedef enum {
     KDA_OK = 0,
@@ -180,13 +180,19 @@ kda_status kda_prefill_checkpointed(const void *q, const void *k, const void *v,
  * tile is unbounded, so the reciprocal factors of the dense tile form overflow and
  * every diagonal tile needs the position-pair path: the fp32 CUDA-core path
  * computes each intra-chunk decay e^{G_r - G_s} as one exponent per pair and key
- * channel.  With KDA_GATE_SOFTPLUS, algo AUTO or CUDA_CORE runs that path;
- * TENSOR_CORE(_SPLIT), whose dense diagonal tiles rest on the bound, returns
- * KDA_ERR_UNSUPPORTED.  The per-token log-decay is clamped at -110 (e^{-110} is
- * 0 in fp32), which changes no result and keeps a chunk's cumulative decay
- * small enough for fp32 differences.  That path needs no workspace (workspace may
- * be NULL with workspace_bytes = 0).  A gate value outside the enum is
- * KDA_ERR_INVALID_ARG.
+ * channel.  With KDA_GATE_SOFTPLUS:
+ *   - CUDA_CORE runs the fp32 CUDA-core path with that pair form for every
+ *     16-token chunk (no workspace: it may be NULL with workspace_bytes = 0);
+ *   - TENSOR_CORE(_SPLIT), and AUTO for bf16 with dk = dv = 128, run the
+ *     tensor-core path as it stood before the bound: off-diagonal 16-token
+ *     sub-tile pairs on tcgen05 with a reference between them (every factor
+ *     <= 1, formed as one exponent), and the four diagonal 16 x 16 tiles of each
+ *     64-token chunk computed pair by pair on CUDA cores by a separate kernel.
+ *     Its workspace is kda_prefill_gated_workspace_size(..., gate), 8 KiB per
+ *     (chunk, head) more than the bounded gate's.
+ * The per-token log-decay is clamped at -110 (e^{-110} is 0 in fp32), which
+ * changes no result and keeps a chunk's cumulative decay small enough for fp32
+ * differences.  A gate value outside the enum is KDA_ERR_INVALID_ARG.
  */
 kda_status kda_prefill_gated(const void *q, const void *k, const void *v, const void *z,
                              const float *A, const float *beta,
@@ -195,6 +201,15 @@ kda_status kda_prefill_gated(const void *q, const void *k, const void *v, const 
                              int32_t dv, kda_dtype dt, const float *initial_state,
                              float *final_state, void *o, void *workspace,
                              size_t workspace_bytes, kda_algo algo, kda_gate gate, void *stream);
+
+/*
+ * Workspace bytes of kda_prefill_gated with the given gate (for
+ * KDA_GATE_LOWER_BOUNDED equal to kda_prefill_workspace_size); 0 for the
+ * CUDA-core path or invalid arguments (an invalid gate included).
+ */
+size_t kda_prefill_gated_workspace_size(int32_t total_tokens, int32_t num_seqs, int32_t H,
+                                        int32_t dk, int32_t dv, kda_dtype dt, kda_algo algo,
+                                        kda_gate gate);
 
 /*
  * Debug run of the tensor-core prefill (bf16, dk = dv = 128; otherwise
@@ -285,12 +300,20 @@ int32_t kda_prefill_segments(int32_t total_tokens, int32_t num_seqs, int32_t H, 
  * at 96 heads) returns KDA_ERR_WORKSPACE and launches nothing.  It calls no
  * cudaMalloc, cudaFree or other allocating routine.
  *
- * The first call on each device looks up the array's device address; make
- * that first call before any stream capture.  Every call on a device shares the
- * one array and leaves its contents behind; the kernels overwrite every scratch
- * byte they later read, so nothing needs clearing.  Calls whose work overlaps
- * on the GPU (different streams, or several host threads) race on the array:
- * the caller must serialise them, e.g. by issuing them all on one stream.
+ * The first call on each device looks up the array's device address, and it
+ * is also the call that places the array in that device's memory: the CUDA
+ * runtime loads a library's device code lazily by default, so the 64 MiB are
+ * taken at this first call, not when the library is loaded.  A caller that
+ * later gives away all free device memory (for example to a cache pool) makes
+ * one call first -- any small valid input -- before reserving that memory,
+ * and before any stream capture.  The address is cached per device and
+ * context; after a device reset (which destroys the context and the array's
+ * contents) the next call looks it up again and places a fresh array.
+ * Every call on a device shares the one array and leaves its contents behind;
+ * the kernels overwrite every scratch byte they later read, so nothing needs
+ * clearing.  Calls whose work overlaps on the GPU (different streams, or
+ * several host threads) race on the array: the caller must serialise them,
+ * e.g. by issuing them all on one stream.
  */
 kda_status kda_prefill_noalloc(const void *q, const void *k, const void *v, const void *z,
                                const float *A, const float *beta,

@@ -29,6 +29,7 @@ SIGNATURES = {
     "kda_abi_version": ([], _I32),
     "kda_status_string": ([_I32], ctypes.c_char_p),
     "kda_prefill_workspace_size": ([_I32, _I32, _I32, _I32, _I32, _I32, _I32], _SZ),
+    "kda_prefill_gated_workspace_size": ([_I32] * 8, _SZ),
     "kda_prefill": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _P], _I32),
     "kda_prefill_ex": ([_P] * 8 + [_I32] * 6 + [_P] * 4 + [_SZ, _I32, _P, _P, _I32], _I32),
     "kda_prefill_kernel_count": ([_I32] * 7, _I32),
@@ -105,6 +106,14 @@ def kda_prefill_workspace_size(total_tokens: int, num_seqs: int, H: int, dk: int
                                                KDA_DTYPE[dtype], KDA_ALGO[algo]))
 
 
+def kda_prefill_gated_workspace_size(total_tokens: int, num_seqs: int, H: int, dk: int, dv: int,
+                                     dtype=torch.bfloat16, algo: str = "auto",
+                                     gate: str = "bounded") -> int:
+    return int(_lib.kda_prefill_gated_workspace_size(total_tokens, num_seqs, H, dk, dv,
+                                                     KDA_DTYPE[dtype], KDA_ALGO[algo],
+                                                     KDA_GATE[gate]))
+
+
 def kda_prefill(q, k, v, z, A, beta, cu_seqlens, cu_seqlens_host=None, initial_state=None,
                 output_final_state: bool = True, final_state=None, o=None, workspace=None,
                 algo: str = "auto", stream=None, stage_events=None, gate: str = "bounded"):
@@ -128,7 +137,7 @@ def kda_prefill(q, k, v, z, A, beta, cu_seqlens, cu_seqlens_host=None, initial_s
         o = torch.empty(T, H, dv, dtype=dt, device=q.device)
     if final_state is None and output_final_state:
         final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
-    need = kda_prefill_workspace_size(T, N, H, dk, dv, dt, algo)
+    need = kda_prefill_gated_workspace_size(T, N, H, dk, dv, dt, algo, gate)
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     host = None

@@ -1,6 +1,7 @@
 // C-ABI layer of libkda_b200: argument validation, workspace sizing and
 // dispatch to the kernels.  Nothing here allocates device memory; every call is
 // asynchronous on the caller's stream.
+#include <cuda.h>
 #include <mutex>
 #include <vector>
 #include <stdint.h>
@@ -14,11 +15,43 @@
 // instead of hanging.  One instance per device that loads the library.
 __device__ int32_t g_kda_device_status = 0;
 
+namespace kda {
+
+// cuCtxGetCurrent / cuCtxGetId, fetched from the driver through the runtime (no
+// link-time dependency on libcuda).
+bool current_context_id(unsigned long long *id)
+{
+    using GetCurrent = CUresult (*)(CUcontext *);
+    using GetId = CUresult (*)(CUcontext, unsigned long long *);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = (GetCurrent)p;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = (GetId)p;
+    });
+    CUcontext ctx = nullptr;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+}  // namespace kda
+
 namespace {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_status_mu;
+// Per device: the status word's device address and the context it belongs to.
+// A device reset destroys the context (and unloads the module); the next call
+// sees a new context id and looks the address up again.
 int32_t *g_status_ptr[kMaxDevices] = {nullptr};
+unsigned long long g_status_ctx[kMaxDevices] = {0};
 
 bool head_dim_ok(int32_t d) { return d == 32 || d == 64 || d == 128; }
 bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
@@ -28,10 +61,14 @@ kda_status status_word(int32_t **out)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_status_mu);
-    if (!g_status_ptr[dev]) {
+    unsigned long long ctx = 0;
+    const bool have_ctx = kda::current_context_id(&ctx);
+    if (!g_status_ptr[dev] || !have_ctx || ctx != g_status_ctx[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_kda_device_status) != cudaSuccess) return KDA_ERR_CUDA;
         g_status_ptr[dev] = (int32_t *)p;
+        // The lookup made the device's primary context current if it was not.
+        g_status_ctx[dev] = kda::current_context_id(&ctx) ? ctx : 0;
     }
     *out = g_status_ptr[dev];
     return KDA_OK;
@@ -90,14 +127,24 @@ extern "C" const char *kda_status_string(kda_status s)
     return "KDA_ERR_UNKNOWN";
 }
 
+extern "C" size_t kda_prefill_gated_workspace_size(int32_t total_tokens, int32_t num_seqs,
+                                                   int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+                                                   kda_algo algo, kda_gate gate)
+{
+    if (check_prefill_sizes(total_tokens, num_seqs, H, dk, dv, dt, algo) != KDA_OK) return 0;
+    if (gate != KDA_GATE_LOWER_BOUNDED && gate != KDA_GATE_SOFTPLUS) return 0;
+    if (use_tensor_core(dk, dv, dt, algo))
+        return kda::tc_workspace_bytes(total_tokens, num_seqs, H,
+                                       segments_for(total_tokens, num_seqs, H, dk, dv, dt, algo),
+                                       gate == KDA_GATE_SOFTPLUS ? 1 : 0);
+    return 0;  // the CUDA-core path keeps everything on chip
+}
+
 extern "C" size_t kda_prefill_workspace_size(int32_t total_tokens, int32_t num_seqs, int32_t H,
                                              int32_t dk, int32_t dv, kda_dtype dt, kda_algo algo)
 {
-    if (check_prefill_sizes(total_tokens, num_seqs, H, dk, dv, dt, algo) != KDA_OK) return 0;
-    if (use_tensor_core(dk, dv, dt, algo))
-        return kda::tc_workspace_bytes(total_tokens, num_seqs, H,
-                                       segments_for(total_tokens, num_seqs, H, dk, dv, dt, algo));
-    return 0;  // the CUDA-core path keeps everything on chip
+    return kda_prefill_gated_workspace_size(total_tokens, num_seqs, H, dk, dv, dt, algo,
+                                            KDA_GATE_LOWER_BOUNDED);
 }
 
 extern "C" int32_t kda_prefill_segments(int32_t total_tokens, int32_t num_seqs, int32_t H,
@@ -137,12 +184,6 @@ kda_status prefill_impl(const void *q, const void *k, const void *v, const void 
     kda_status st = check_prefill_sizes(total_tokens, num_seqs, H, dk, dv, dt, algo);
     if (st != KDA_OK) return st;
     if (gate != KDA_GATE_LOWER_BOUNDED && gate != KDA_GATE_SOFTPLUS) return KDA_ERR_INVALID_ARG;
-    if (gate == KDA_GATE_SOFTPLUS) {
-        // The tensor-core path relies on the lower bound; the unbounded gate runs
-        // on the CUDA-core path with its position-pair diagonal tiles.
-        if (algo == KDA_ALGO_TENSOR_CORE || algo == KDA_ALGO_TENSOR_CORE_SPLIT) return KDA_ERR_UNSUPPORTED;
-        algo = KDA_ALGO_CUDA_CORE;
-    }
     if (checkpoint_every < 0 || checkpoint_every % 64 != 0) return KDA_ERR_INVALID_ARG;
     if (checkpoint_every > 0 && (!checkpoints || !aligned(checkpoints, 16))) return KDA_ERR_INVALID_ARG;
     if (checkpoint_every > 0 && algo == KDA_ALGO_TENSOR_CORE_SPLIT) return KDA_ERR_UNSUPPORTED;
@@ -161,7 +202,8 @@ kda_status prefill_impl(const void *q, const void *k, const void *v, const void 
             if (cu_seqlens_host[i + 1] < cu_seqlens_host[i]) return KDA_ERR_INVALID_ARG;
     }
     if (num_seqs == 0) return KDA_OK;
-    const size_t need = kda_prefill_workspace_size(total_tokens, num_seqs, H, dk, dv, dt, algo);
+    const size_t need = kda_prefill_gated_workspace_size(total_tokens, num_seqs, H, dk, dv, dt,
+                                                         algo, gate);
     if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
 
     int32_t *status = nullptr;

@@ -8,6 +8,11 @@
 
 namespace kda {
 
+// Identifier of the calling thread's current CUDA context (cuCtxGetId: unique
+// for the process lifetime, so a context destroyed and created again, as by
+// cudaDeviceReset, gets a new one).  False when no context is current.
+bool current_context_id(unsigned long long *id);
+
 struct PrefillArgs {
     const void *q, *k, *v, *z;
     const float *A, *beta;

@@ -12,6 +12,7 @@
 #include <stdint.h>
 
 #include "kda.h"
+#include "kda_internal.h"
 
 namespace {
 
@@ -31,18 +32,25 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void *g_scratch_ptr[kMaxDevices] = {nullptr};
+unsigned long long g_scratch_ctx[kMaxDevices] = {0};
 
 // Device address of the scratch array on the current device, looked up once
-// per device (the first call on each device does this set-up).
+// per device and context (the first call on each device does this set-up; it
+// is also where the runtime, which loads device code lazily, first places the
+// array in that device's memory).  A device reset destroys the context, and
+// the module with it; the next call sees a new context id and looks again.
 kda_status scratch_on_current_device(void **out)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_scratch_ptr[dev]) {
+    unsigned long long ctx = 0;
+    const bool have_ctx = kda::current_context_id(&ctx);
+    if (!g_scratch_ptr[dev] || !have_ctx || ctx != g_scratch_ctx[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_kda_noalloc_scratch) != cudaSuccess || !p) return KDA_ERR_CUDA;
         g_scratch_ptr[dev] = p;
+        g_scratch_ctx[dev] = kda::current_context_id(&ctx) ? ctx : 0;
     }
     *out = g_scratch_ptr[dev];
     return KDA_OK;

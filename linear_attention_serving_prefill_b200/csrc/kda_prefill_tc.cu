@@ -40,6 +40,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
+#include <cstring>
 #include <mutex>
 
 #include "kda_common.cuh"
@@ -156,9 +157,13 @@ plan_kernel(const int32_t *__restrict__ cu, int N, int every, int32_t *__restric
 // Persistent, two CTAs of 256 threads per SM, each walking (chunk, head) items
 // b, b + gridDim.x, ...; item w is chunk w / H of head w % H.  A CTA holds one
 // item at a time; the SM's other CTA overlaps its waits (loads, products,
-// barriers).  Thread (cp, I) owns channels 2 cp, 2 cp + 1 of the 16 rows of
-// sub-tile I = warp / 2, so the sub-tile index is uniform across a warp.
+// barriers).  Thread (cp, p) owns channels 2 cp, 2 cp + 1 of the 8-row
+// half-blocks p and 7 - p (p = warp / 2), so the rows' sub-tiles are uniform
+// across a warp and every thread has the same share of R copies.
 constexpr int kIntraThreads = 256;
+// Waits of the intra kernel (inputs, products) let the waiting warps sleep up to
+// this long per try, so that they leave the issue slots to the SM's other CTA.
+constexpr uint32_t kIntraSuspendNs = 20000;
 constexpr uint32_t kRawTile = kChunk * kDK * 2;    // one [64][128] bf16 tile, 16 KiB
 // Shared memory (offsets from a 1024-aligned base).  The raw k, q, v, z tiles
 // arrive by two 128-byte-swizzled TMA boxes each, as K-major operand images
@@ -221,24 +226,74 @@ __device__ __forceinline__ float2 ld_bf16x2_smem(const uint8_t *base, uint32_t o
     return __bfloat1622float2(*(const __nv_bfloat162 *)(base + off));
 }
 
-__device__ __forceinline__ uint32_t bf16_bits(float x) {
-    return __bfloat16_as_ushort(__float2bfloat16_rn(x));
-}
 
 // The gate with the fast exponential and division (a few ulp; the bf16 path's
 // tolerance is far looser).  Limits as in gate_log_decay: exp(A) z -> +inf gives
 // g_min, -> -inf gives 0 (1 / +inf through the fast division is 0).
-__device__ __forceinline__ float gate_log_decay_fast(float expA, float z) {
-    return __fdividef(kGMin, 1.0f + __expf(-expA * z));
+// Packed fp32 pair arithmetic (one f32x2 instruction for both lanes of a
+// channel pair; each lane is an IEEE round-to-nearest operation) and the
+// approximate base-2 exponential and reciprocal of the special-function unit.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float2 exp2_2(float2 x) { return make_float2(ex2_approx(x.x), ex2_approx(x.y)); }
+constexpr float kLog2e = 1.4426950408889634f;
+__device__ __forceinline__ float2 log2e2() { return make_float2(kLog2e, kLog2e); }
+__device__ __forceinline__ uint32_t pack2(float2 v) { return pack_bf16(v.x, v.y); }
+
+// The gate with the approximate exponential and reciprocal (a few ulp; the
+// bf16 path's tolerance is far looser), given eAn = -exp(A) log2(e):
+// g = g_min / (1 + 2^{eAn z}).  Limits as in gate_log_decay: exp(A) z -> +inf
+// gives 2^{-inf} = 0 and g = g_min; -> -inf gives 1 / inf = 0, i.e. g = -0.
+__device__ __forceinline__ float gate_fast(float eAn, float z) {
+    return kGMin * rcp_approx(1.0f + ex2_approx(eAn * z));
+}
+__device__ __forceinline__ float2 gate2(float2 eAn, float2 z) {
+    const float2 d = add2(exp2_2(mul2(eAn, z)), make_float2(1.f, 1.f));
+    return mul2(make_float2(rcp_approx(d.x), rcp_approx(d.y)), make_float2(kGMin, kGMin));
 }
 
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+constexpr float kLn2 = 0.6931471805599453f;
+
+// The unbounded gate g = -softplus(exp(A) z) = -(max(x, 0) + ln(1 + e^{-|x|})),
+// x = exp(A) z, with the approximate exponential and logarithm (absolute error
+// of a few 1e-7), clamped at kGClampSoftplus like the exact form.
+__device__ __forceinline__ float gate_softplus_fast(float eA, float z) {
+    const float x = eA * z;
+    const float l1p = kLn2 * lg2_approx(1.0f + ex2_approx(-fabsf(x) * kLog2e));
+    return fmaxf(-(fmaxf(x, 0.0f) + l1p), kGClampSoftplus);
+}
+
+// GATE = kGateBounded: the K3 gate, dense diagonal tiles (the bound keeps every
+// factor below e^80).  GATE = kGateSoftplus: the unbounded gate; the diagonal
+// 16 x 16 tiles of A and P come from diag_pair_kernel (`pairs`), their R rows
+// are zero, and every other factor is formed as one exponent <= 0.
+template <int GATE>
 __global__ void __launch_bounds__(kIntraThreads, 2)
 intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_z,
              const float *__restrict__ A, const float *__restrict__ beta,
              const int2 *__restrict__ chunk_loc, const int32_t *__restrict__ chunk_off, int N, int H,
-             uint8_t *__restrict__ blocks, int64_t max_chunks, int32_t *status)
+             uint8_t *__restrict__ blocks, int64_t max_chunks, int32_t *status,
+             const float *__restrict__ pairs)
 {
+    constexpr bool kSoftplus = GATE == kGateSoftplus;
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
     __shared__ uint64_t full, mma_bar, ap_bar;
@@ -247,7 +302,7 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     __shared__ int2 next_loc;
     __shared__ float sBeta[kChunk];
     __shared__ float sA[kDK];
-    __shared__ float sTot[4][kDK];
+    __shared__ float sHalf[8][kDK];   // gate sums of the eight 8-row half-blocks
     __shared__ volatile int sAbort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -297,14 +352,14 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     int issued = 1;  // items requested so far (meaningful in warp 0)
 
     {
-        const int cp = ((warp & 1) << 5) | lane, c0 = 2 * cp, I = warp >> 1;
+        const int cp = ((warp & 1) << 5) | lane, c0 = 2 * cp, p = warp >> 1;
         float *Af = (float *)(sm + kIAf), *Tf = (float *)(sm + kITf), *Xf = (float *)(sm + kIXf);
         uint32_t mma_count = 0;
         int mma_failed = -1, ap_failed = -1;  // parity of a product wait that gave up
         int it = 0;
         for (int w = blockIdx.x; w < total_items && !sAbort; w += gridDim.x, ++it) {
             if (warp == 0) cp_async_wait_all();  // this item's beta and A values
-            if (!mbar_wait(&full, it & 1, globaltimer_ns() + kWaitNs)) {
+            if (!mbar_wait<kIntraSuspendNs>(&full, it & 1, globaltimer_ns() + kWaitNs)) {
                 if (tid == 0) record_timeout(status);
                 sAbort = 1;
             }
@@ -313,7 +368,10 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             const IntraItem inf = info;
             const int len = inf.len, h = inf.h;
             uint8_t *blk = blocks + ((size_t)h * max_chunks + inf.g) * kBlockBytes;
-            const float2 eA = make_float2(__expf(sA[c0]), __expf(sA[c0 + 1]));
+            // exp(A) of channels c0, c0 + 1; for the bounded gate pre-multiplied by
+            // -log2(e), the form gate2 takes.
+            const float2 eA2 = exp2_2(mul2(*(const float2 *)&sA[c0], log2e2()));
+            const float2 eAn = kSoftplus ? eA2 : mul2(eA2, make_float2(-kLog2e, -kLog2e));
             const bool has_next = w + (int)gridDim.x < total_items;
             // The next item's chunk-table entry, fetched asynchronously for issue().
             if (tid == 0 && has_next) {
@@ -321,98 +379,157 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 cp_async_commit();
             }
 
-            // Pass 1: gate of channels c0, c0 + 1 summed over the sub-tile's 16 rows.
-            // Each row's running sum L_r = G_r - m_I is parked in TMEM for pass 2
-            // (lane 32 (warp % 4) + lane, 32 columns from 128 + 32 (warp / 4)); those
-            // columns are free from the previous item's W/U readback until this
-            // item's W/U product, and registers are not.
+            // Pass 1: gate of channels c0, c0 + 1 over two 8-row half-blocks, b = p and
+            // b = 7 - p (p = warp / 2).  Half-block b lies in sub-tile b / 2, whose rows
+            // are copied into 4 - b / 2 of the R images in pass 2, so this pairing gives
+            // every thread the same number of copies.  Each row's running sum from its
+            // half-block start is parked in TMEM for pass 2 (lane 32 (warp % 4) + lane,
+            // 16 columns per half-block from 128 + 32 (warp / 4)); those columns are free
+            // from the previous item's W/U readback until this item's W/U product.
+            // beta V of the same rows is formed here too, so that the v tile is dead
+            // after this pass.
             const uint32_t lcol = tmem_addr(tb, 32 * (warp & 3), 128 + 32 * (warp >> 2));
-            float2 acc = make_float2(0.f, 0.f);
-            float lst[8];
+            uint32_t pv0[8], pv1[8];   // beta V, rows (2 m, 2 m + 1) of channel c0 / c0 + 1
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = 16 * I + i;
-                if (r < len) {
-                    const float2 zz = ld_bf16x2_smem(sm, kRawZ + sw128_offset(r, c0, 64));
-                    acc.x += gate_log_decay_fast(eA.x, zz.x);
-                    acc.y += gate_log_decay_fast(eA.y, zz.y);
+            for (int q = 0; q < 2; ++q) {
+                const int b = q == 0 ? p : 7 - p;
+                float2 acc = make_float2(0.f, 0.f);
+                float lst[8];
+                float2 hv[2];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = 8 * b + i;
+                    const uint32_t so = sw128_offset(r, c0, 64);
+                    float2 vv = make_float2(0.f, 0.f);
+                    if (r < len) {
+                        const float2 zz = ld_bf16x2_smem(sm, kRawZ + so);
+                        acc = add2(acc, kSoftplus ? make_float2(gate_softplus_fast(eAn.x, zz.x),
+                                                                gate_softplus_fast(eAn.y, zz.y))
+                                                  : gate2(eAn, zz));
+                        vv = ld_bf16x2_smem(sm, kRawV + so);
+                    }
+                    hv[i & 1] = mul2(vv, make_float2(sBeta[r], sBeta[r]));
+                    if (i & 1) {
+                        pv0[4 * q + (i >> 1)] = pack_bf16(hv[0].x, hv[1].x);
+                        pv1[4 * q + (i >> 1)] = pack_bf16(hv[0].y, hv[1].y);
+                    }
+                    lst[2 * (i & 3)] = acc.x;
+                    lst[2 * (i & 3) + 1] = acc.y;
+                    if ((i & 3) == 3) tmem_st8(lcol + 16 * q + 8 * (i >> 2), lst);
                 }
-                lst[2 * (i & 3)] = acc.x;
-                lst[2 * (i & 3) + 1] = acc.y;
-                if ((i & 3) == 3) tmem_st8(lcol + 8 * (i >> 2), lst);
+                *(float2 *)&sHalf[b][c0] = acc;
             }
             tmem_st_wait();
-            sTot[I][c0] = acc.x;
-            sTot[I][c0 + 1] = acc.y;
             compute_sync();
             if (sAbort) break;
-            // Sub-tile references m_J = G at the end of sub-tile J - 1 (m_0 = 0), G_C.
-            float2 mref[5];
-            mref[0] = make_float2(0.f, 0.f);
+            // (beta V)^T (rows = channels, K = tokens) into the z tile, dead since pass
+            // 1: rows 128..255 of the B operand of the W/U product.
 #pragma unroll
-            for (int J = 0; J < 4; ++J)
-                mref[J + 1] = make_float2(mref[J].x + sTot[J][c0], mref[J].y + sTot[J][c0 + 1]);
-            const float2 mI = I == 0 ? mref[0] : I == 1 ? mref[1] : I == 2 ? mref[2] : mref[3];
-            const float2 GC = mref[4];
-            const float2 emI = make_float2(__expf(mI.x), __expf(mI.y));
-            const float2 egc = make_float2(__expf(GC.x - mI.x), __expf(GC.y - mI.y));
-            // fac[Ip] = e^{m_Ip - m_I} carries a column operand from sub-tile I's
-            // reference to a later sub-tile's (1 for Ip = I).
-            float2 fac[4];
-#pragma unroll
-            for (int Ip = 0; Ip < 4; ++Ip)
-                fac[Ip] = Ip > I ? make_float2(__expf(mref[Ip].x - mI.x), __expf(mref[Ip].y - mI.y))
-                                 : make_float2(1.f, 1.f);
-
-            // Pass 2: scaled operands of channels c0, c0 + 1 for the 16 rows, with L
-            // read back from TMEM four rows at a time.
-            // Kt = k e^{L} and Qt = q e^{L} replace k and q in place (same thread,
-            // same address); the rest goes to R, to the block, or into registers.
-            // beta K e^G, beta V and K e^{G_C - G} wait in registers until the tiles
-            // that receive them are no longer read.
-            uint32_t pk0[8], pk1[8], pv0[8], pv1[8], kd0[8], kd1[8];
-            float lrd[8];  // L of four rows, from pass 1
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = 16 * I + i;
-                const bool valid = r < len;
-                const uint32_t off = sw128_offset(r, c0, 64);
-                if ((i & 3) == 0) {
-                    tmem_ld8(lcol + 8 * (i >> 2), lrd);
-                    tmem_ld_wait();
-                }
-                const float2 Lr = make_float2(lrd[2 * (i & 3)], lrd[2 * (i & 3) + 1]);
-                const float2 kv = valid ? ld_bf16x2_smem(sm, kRawK + off) : make_float2(0.f, 0.f);
-                const float2 qv = valid ? ld_bf16x2_smem(sm, kRawQ + off) : make_float2(0.f, 0.f);
-                const float2 vv = valid ? ld_bf16x2_smem(sm, kRawV + off) : make_float2(0.f, 0.f);
-                const float2 e1 = make_float2(__expf(Lr.x), __expf(Lr.y));    // in [e^-80, 1]
-                const float2 e2 = make_float2(__expf(-Lr.x), __expf(-Lr.y));  // in [1, e^80]
-                const float br = sBeta[r];
-                *(uint32_t *)(sm + kRawK + off) = pack_bf16(kv.x * e1.x, kv.y * e1.y);
-                *(uint32_t *)(sm + kRawQ + off) = pack_bf16(qv.x * e1.x, qv.y * e1.y);
-                const float2 kb = make_float2(kv.x * e2.x, kv.y * e2.y);
-#pragma unroll
-                for (int Ip = 0; Ip < 4; ++Ip)
-                    if (Ip >= I)
-                        *(uint32_t *)(sm + r_region(Ip, c0 >> 6) + sw128_offset(r, c0 & 63, 64)) =
-                            pack_bf16(kb.x * fac[Ip].x, kb.y * fac[Ip].y);
-                *(uint32_t *)(blk + kOffWQ + sw128_offset(64 + r, c0, 128)) =
-                    pack_bf16(qv.x * e1.x * emI.x, qv.y * e1.y * emI.y);
-                const uint32_t hk0 = bf16_bits(br * kv.x * e1.x * emI.x), hk1 = bf16_bits(br * kv.y * e1.y * emI.y);
-                const uint32_t hv0 = bf16_bits(br * vv.x), hv1 = bf16_bits(br * vv.y);
-                const uint32_t hd0 = bf16_bits(kb.x * egc.x), hd1 = bf16_bits(kb.y * egc.y);
-                if ((i & 1) == 0) {
-                    pk0[i >> 1] = hk0; pk1[i >> 1] = hk1; pv0[i >> 1] = hv0; pv1[i >> 1] = hv1;
-                    kd0[i >> 1] = hd0; kd1[i >> 1] = hd1;
-                } else {
-                    pk0[i >> 1] |= hk0 << 16; pk1[i >> 1] |= hk1 << 16;
-                    pv0[i >> 1] |= hv0 << 16; pv1[i >> 1] |= hv1 << 16;
-                    kd0[i >> 1] |= hd0 << 16; kd1[i >> 1] |= hd1 << 16;
-                }
+            for (int q = 0; q < 2; ++q) {
+                const int kk = 8 * (q == 0 ? p : 7 - p);
+                *(uint4 *)(sm + kRawZ + sw128_offset(c0, kk, 128)) =
+                    make_uint4(pv0[4 * q], pv0[4 * q + 1], pv0[4 * q + 2], pv0[4 * q + 3]);
+                *(uint4 *)(sm + kRawZ + sw128_offset(c0 + 1, kk, 128)) =
+                    make_uint4(pv1[4 * q], pv1[4 * q + 1], pv1[4 * q + 2], pv1[4 * q + 3]);
             }
-            if (I == 0) {
-                ((float *)(blk + kOffDecay))[c0] = __expf(GC.x);
-                ((float *)(blk + kOffDecay))[c0 + 1] = __expf(GC.y);
+            // G_C = the sum of the eight half-blocks; e^{G_C} goes to the block
+            // (warps 0 and 1 hold channels 0..127 between them).
+            float2 GC = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int b = 0; b < 8; ++b) GC = add2(GC, *(const float2 *)&sHalf[b][c0]);
+            if (warp < 2) *(float2 *)(blk + kOffDecay + 4 * c0) = exp2_2(mul2(GC, log2e2()));
+
+            // Pass 2, per half-block: scaled operands of channels c0, c0 + 1 for its 8
+            // rows, with L = G - m_I read back from TMEM four rows at a time.
+            // Kt = k e^{L} and Qt = q e^{L} replace k and q in place (same thread, same
+            // address); the R copies, Q e^{G} and K e^{G_C - G} (to the block) and
+            // (beta K e^{G})^T (into the v tile, dead since pass 1) are written as soon
+            // as they are formed.
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int b = q == 0 ? p : 7 - p, I = b >> 1;
+                // Sub-tile references m_J = G at the end of sub-tile J - 1 (m_0 = 0):
+                // m_I, and fac[Ip] = e^{m_Ip - m_I} for the later sub-tiles Ip > I, which
+                // carries a column operand from sub-tile I's reference to Ip's.
+                float2 mI = make_float2(0.f, 0.f), fac[4];
+                {
+                    float2 m = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int J = 0; J < 4; ++J) {
+                        if (J == I) mI = m;
+                        fac[J] = m;
+                        m = add2(m, add2(*(const float2 *)&sHalf[2 * J][c0], *(const float2 *)&sHalf[2 * J + 1][c0]));
+                    }
+                }
+                // Bounded gate: fac[J] = e^{m_J - m_I}.  Unbounded gate: fac[J] = m_J - m_I
+                // (<= 0), added to -L inside one exponent per copy instead.
+#pragma unroll
+                for (int J = 1; J < 4; ++J)
+                    fac[J] = kSoftplus ? sub2(fac[J], mI) : exp2_2(mul2(sub2(fac[J], mI), log2e2()));
+                const float2 off = (b & 1) ? *(const float2 *)&sHalf[b - 1][c0] : make_float2(0.f, 0.f);
+                const float2 emI = exp2_2(mul2(mI, log2e2()));
+                const float2 gcm = sub2(GC, mI);
+                const float2 egc = kSoftplus ? gcm : exp2_2(mul2(gcm, log2e2()));
+                uint32_t pk0[4], pk1[4], kd0[4], kd1[4];
+                float lrd[8];  // partial sums of four rows, from pass 1
+#pragma unroll
+                for (int i2 = 0; i2 < 8; i2 += 2) {
+                    float2 hk[2], hd[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int i = i2 + u, r = 8 * b + i;
+                        const bool valid = r < len;
+                        const uint32_t so = sw128_offset(r, c0, 64);
+                        if ((i & 3) == 0) {
+                            tmem_ld8(lcol + 16 * q + 8 * (i >> 2), lrd);
+                            tmem_ld_wait();
+                        }
+                        const float2 L = add2(make_float2(lrd[2 * (i & 3)], lrd[2 * (i & 3) + 1]), off);
+                        const float2 kv = valid ? ld_bf16x2_smem(sm, kRawK + so) : make_float2(0.f, 0.f);
+                        const float2 qv = valid ? ld_bf16x2_smem(sm, kRawQ + so) : make_float2(0.f, 0.f);
+                        const float2 lg = mul2(L, log2e2());
+                        const float2 e1 = exp2_2(lg);                          // in [e^-80, 1]
+                        const float br = sBeta[r];
+                        const float2 kt = mul2(kv, e1), qt = mul2(qv, e1);
+                        *(uint32_t *)(sm + kRawK + so) = pack2(kt);
+                        *(uint32_t *)(sm + kRawQ + so) = pack2(qt);
+                        const uint32_t ro = sw128_offset(r, c0 & 63, 64);
+                        if constexpr (kSoftplus) {
+                            // Diagonal tile rows are zero (the pair kernel supplies that
+                            // tile); later sub-tiles get k e^{m_Ip - G} as one exponent.
+                            *(uint32_t *)(sm + r_region(I, c0 >> 6) + ro) = 0u;
+#pragma unroll
+                            for (int Ip = 1; Ip < 4; ++Ip)
+                                if (Ip > I)
+                                    *(uint32_t *)(sm + r_region(Ip, c0 >> 6) + ro) =
+                                        pack2(mul2(kv, exp2_2(mul2(sub2(fac[Ip], L), log2e2()))));
+                            hd[u] = mul2(kv, exp2_2(mul2(sub2(egc, L), log2e2())));
+                        } else {
+                            const float2 kb = mul2(kv, exp2_2(make_float2(-lg.x, -lg.y)));  // [1, e^80]
+                            *(uint32_t *)(sm + r_region(I, c0 >> 6) + ro) = pack2(kb);
+#pragma unroll
+                            for (int Ip = 1; Ip < 4; ++Ip)
+                                if (Ip > I)
+                                    *(uint32_t *)(sm + r_region(Ip, c0 >> 6) + ro) = pack2(mul2(kb, fac[Ip]));
+                            hd[u] = mul2(kb, egc);
+                        }
+                        *(uint32_t *)(blk + kOffWQ + sw128_offset(64 + r, c0, 128)) = pack2(mul2(qt, emI));
+                        hk[u] = mul2(mul2(kt, emI), make_float2(br, br));
+                    }
+                    // Rows i2, i2 + 1 of each channel as one bf16 pair (low half = row i2).
+                    pk0[i2 >> 1] = pack_bf16(hk[0].x, hk[1].x);
+                    pk1[i2 >> 1] = pack_bf16(hk[0].y, hk[1].y);
+                    kd0[i2 >> 1] = pack_bf16(hd[0].x, hd[1].x);
+                    kd1[i2 >> 1] = pack_bf16(hd[0].y, hd[1].y);
+                }
+                // (beta K e^G)^T into the v tile: rows 0..127 of the W/U product's B
+                // operand; (K e^{G_C - G})^T straight to its block region (rows =
+                // channels, K = tokens 8 b .. 8 b + 7, the state kernel's B operand).
+                const int kk = 8 * b;
+                *(uint4 *)(sm + kRawV + sw128_offset(c0, kk, 128)) = make_uint4(pk0[0], pk0[1], pk0[2], pk0[3]);
+                *(uint4 *)(sm + kRawV + sw128_offset(c0 + 1, kk, 128)) = make_uint4(pk1[0], pk1[1], pk1[2], pk1[3]);
+                *(uint4 *)(blk + kOffKd + sw128_offset(c0, kk, 128)) = make_uint4(kd0[0], kd0[1], kd0[2], kd0[3]);
+                *(uint4 *)(blk + kOffKd + sw128_offset(c0 + 1, kk, 128)) = make_uint4(kd1[0], kd1[1], kd1[2], kd1[3]);
             }
 
             // A/P products, per sub-tile I (M = 64 rows s of R^(I), N = 16 + 16):
@@ -438,21 +555,7 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                     }
                 mma_commit(&ap_bar);
             }
-            // Meanwhile: [beta K e^G ; beta V]^T (rows = channels, K = tokens), the
-            // B operand of the W/U product, into the v and z tiles (no longer read).
-#pragma unroll
-            for (int hlf = 0; hlf < 2; ++hlf) {
-                const int kk = 16 * I + 8 * hlf;
-                *(uint4 *)(sm + kRawV + sw128_offset(c0, kk, 128)) =
-                    make_uint4(pk0[4 * hlf], pk0[4 * hlf + 1], pk0[4 * hlf + 2], pk0[4 * hlf + 3]);
-                *(uint4 *)(sm + kRawV + sw128_offset(c0 + 1, kk, 128)) =
-                    make_uint4(pk1[4 * hlf], pk1[4 * hlf + 1], pk1[4 * hlf + 2], pk1[4 * hlf + 3]);
-                *(uint4 *)(sm + kRawZ + sw128_offset(c0, kk, 128)) =
-                    make_uint4(pv0[4 * hlf], pv0[4 * hlf + 1], pv0[4 * hlf + 2], pv0[4 * hlf + 3]);
-                *(uint4 *)(sm + kRawZ + sw128_offset(c0 + 1, kk, 128)) =
-                    make_uint4(pv1[4 * hlf], pv1[4 * hlf + 1], pv1[4 * hlf + 2], pv1[4 * hlf + 3]);
-            }
-            if (!mbar_wait(&ap_bar, it & 1, globaltimer_ns() + kWaitNs)) {
+            if (!mbar_wait<kIntraSuspendNs>(&ap_bar, it & 1, globaltimer_ns() + kWaitNs)) {
                 if (tid == 0) record_timeout(status);
                 sAbort = 1;
                 ap_failed = it & 1;
@@ -468,6 +571,19 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 tmem_ld16x2_32(tmem_addr(tb, 32 * q, 64 * hb), rr);
                 tmem_ld_wait();
                 const int sidx = 16 * q + (lane & 15);
+                if (kSoftplus && q == Ia) {
+                    // The diagonal tile, from the pair kernel: [A | P][I][s][r] per item.
+                    const float4 *pa = (const float4 *)(pairs + ((size_t)h * max_chunks + inf.g) * 2048 +
+                                                        Ia * 256 + (lane & 15) * 16);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        const float4 av = pa[v4], pv = pa[256 + v4];
+                        rr[4 * v4] = __float_as_uint(av.x); rr[4 * v4 + 1] = __float_as_uint(av.y);
+                        rr[4 * v4 + 2] = __float_as_uint(av.z); rr[4 * v4 + 3] = __float_as_uint(av.w);
+                        rr[16 + 4 * v4] = __float_as_uint(pv.x); rr[16 + 4 * v4 + 1] = __float_as_uint(pv.y);
+                        rr[16 + 4 * v4 + 2] = __float_as_uint(pv.z); rr[16 + 4 * v4 + 3] = __float_as_uint(pv.w);
+                    }
+                }
 #pragma unroll
                 for (int jr = 0; jr < 16; ++jr) {
                     const int r = 16 * Ia + jr;
@@ -477,18 +593,11 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                         __float2bfloat16_rn(pvv);
                 }
             }
-            // (K e^{G_C - G})^T staged in the q tile (Qt is no longer read) as the
-            // exact image of its block region, then bulk-stored with P.
-            *(uint4 *)(sm + kRawQ + sw128_offset(c0, 16 * I, 128)) = make_uint4(kd0[0], kd0[1], kd0[2], kd0[3]);
-            *(uint4 *)(sm + kRawQ + sw128_offset(c0, 16 * I + 8, 128)) = make_uint4(kd0[4], kd0[5], kd0[6], kd0[7]);
-            *(uint4 *)(sm + kRawQ + sw128_offset(c0 + 1, 16 * I, 128)) = make_uint4(kd1[0], kd1[1], kd1[2], kd1[3]);
-            *(uint4 *)(sm + kRawQ + sw128_offset(c0 + 1, 16 * I + 8, 128)) = make_uint4(kd1[4], kd1[5], kd1[6], kd1[7]);
             fence_proxy_async_smem();
             tc_fence_before_sync();
             compute_sync();
             if (sAbort) break;
             if (tid == 0) {
-                bulk_s2g(blk + kOffKd, sm + kRawQ, 16384);
                 bulk_s2g(blk + kOffP, sm + kRawK + 8192, 8192);
                 bulk_commit();
             }
@@ -533,25 +642,21 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             compute_sync();
             {
                 // Level 1, blocks (1,0) and (3,2): X = A_ij T_jj, columns 2 sb, 2 sb + 1.
-                const int p = tid >> 7, r = (tid >> 3) & 15, cb = 2 * (tid & 7);
-                const int oi = 32 * p + 16, oj = 32 * p;
+                const int pb = tid >> 7, r = (tid >> 3) & 15, cb = 2 * (tid & 7);
+                const int oi = 32 * pb + 16, oj = 32 * pb;
                 float2 x = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     const float a = Af[(oi + r) * kLd + oj + t];
-                    const float2 tv = *(const float2 *)&Tf[(oj + t) * kLd + oj + cb];
-                    x.x = fmaf(a, tv.x, x.x);
-                    x.y = fmaf(a, tv.y, x.y);
+                    x = fma2(make_float2(a, a), *(const float2 *)&Tf[(oj + t) * kLd + oj + cb], x);
                 }
-                *(float2 *)&Xf[(16 * p + r) * kXLd + cb] = x;
+                *(float2 *)&Xf[(16 * pb + r) * kXLd + cb] = x;
                 compute_sync();
                 float2 y = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     const float tt = Tf[(oi + r) * kLd + oi + t];
-                    const float2 xv = *(const float2 *)&Xf[(16 * p + t) * kXLd + cb];
-                    y.x = fmaf(tt, xv.x, y.x);
-                    y.y = fmaf(tt, xv.y, y.y);
+                    y = fma2(make_float2(tt, tt), *(const float2 *)&Xf[(16 * pb + t) * kXLd + cb], y);
                 }
                 *(float2 *)&Tf[(oi + r) * kLd + oj + cb] = make_float2(-y.x, -y.y);
                 *(uint32_t *)(sT + sw128_offset(oi + r, oj + cb, 64)) = pack_bf16(-y.x, -y.y);
@@ -560,24 +665,25 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             {
                 // Level 2, block rows 32..63 x columns 0..31: columns 4 sb .. 4 sb + 3.
                 const int r = tid >> 3, cb = 4 * (tid & 7);
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                float2 x0 = make_float2(0.f, 0.f), x1 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int t = 0; t < 32; ++t) {
                     const float a = Af[(32 + r) * kLd + t];
                     const float4 tv = *(const float4 *)&Tf[t * kLd + cb];
-                    x.x = fmaf(a, tv.x, x.x); x.y = fmaf(a, tv.y, x.y);
-                    x.z = fmaf(a, tv.z, x.z); x.w = fmaf(a, tv.w, x.w);
+                    x0 = fma2(make_float2(a, a), make_float2(tv.x, tv.y), x0);
+                    x1 = fma2(make_float2(a, a), make_float2(tv.z, tv.w), x1);
                 }
-                *(float4 *)&Xf[r * kXLd + cb] = x;
+                *(float4 *)&Xf[r * kXLd + cb] = make_float4(x0.x, x0.y, x1.x, x1.y);
                 compute_sync();
-                float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+                float2 y0 = make_float2(0.f, 0.f), y1 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int t = 0; t < 32; ++t) {
                     const float tt = Tf[(32 + r) * kLd + 32 + t];
                     const float4 xv = *(const float4 *)&Xf[t * kXLd + cb];
-                    y.x = fmaf(tt, xv.x, y.x); y.y = fmaf(tt, xv.y, y.y);
-                    y.z = fmaf(tt, xv.z, y.z); y.w = fmaf(tt, xv.w, y.w);
+                    y0 = fma2(make_float2(tt, tt), make_float2(xv.x, xv.y), y0);
+                    y1 = fma2(make_float2(tt, tt), make_float2(xv.z, xv.w), y1);
                 }
+                const float4 y = make_float4(y0.x, y0.y, y1.x, y1.y);
                 *(uint2 *)(sT + sw128_offset(32 + r, cb, 64)) =
                     make_uint2(pack_bf16(-y.x, -y.y), pack_bf16(-y.z, -y.w));
             }
@@ -596,7 +702,7 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                            desc_kmajor_sw128(smem_u32(sm + kRawV) + ks * 32), id, ks > 0);
                 mma_commit(&mma_bar);
             }
-            if (!mbar_wait(&mma_bar, mma_count & 1, globaltimer_ns() + kWaitNs)) {
+            if (!mbar_wait<kIntraSuspendNs>(&mma_bar, mma_count & 1, globaltimer_ns() + kWaitNs)) {
                 if (tid == 0) record_timeout(status);
                 sAbort = 1;
                 mma_failed = (int)(mma_count & 1);
@@ -657,22 +763,140 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     if (warp == 0) tmem_dealloc(tb, 256);
 }
 
+// ------------------------------------------------------------------- pair --
+
+// The unbounded gate's diagonal tiles, pair by pair ("Kimi K3: Architecture,
+// Training, and Million-Token Agentic RL", section 3.3: before the bound,
+// diagonal tiles needed a position-pair path).  For the 16-token sub-tile I of
+// a (chunk, head) item and rows s <= r in it:
+//   A[I][s][r] = sum_c k_rc k_sc e^{L_rc - L_sc},   P[I][s][r] = sum_c q_rc k_sc e^{L_rc - L_sc},
+// L the cumulative log-decay from the sub-tile start, one exponent per pair and
+// channel, so no factor overflows however fast the state decays (beta and the
+// causal masks are applied by the intra kernel, which reads these tiles in place
+// of its products' diagonal tiles).  One CTA per item; rows beyond the chunk's
+// length give zeros.  Output per item: 2 x 4 x 16 x 16 fp32.
+constexpr int kPairThreads = 256;
+constexpr int kPairLd = 130;   // fp32 row stride of the staged L, k, q rows
+constexpr uint32_t kPairSmem = 3u * kChunk * kPairLd * 4u;
+
+__global__ void __launch_bounds__(kPairThreads)
+diag_pair_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ q,
+                 const __nv_bfloat16 *__restrict__ z, const float *__restrict__ A,
+                 const int2 *__restrict__ chunk_loc, const int32_t *__restrict__ chunk_off, int N,
+                 int H, int64_t max_chunks, float *__restrict__ pairs)
+{
+    extern __shared__ float psm[];
+    float *Ls = psm, *Ks = psm + kChunk * kPairLd, *Qs = psm + 2 * kChunk * kPairLd;
+    const int h = blockIdx.x % H, g = blockIdx.x / H;
+    if (g >= chunk_off[N]) return;
+    const int2 loc = chunk_loc[g];
+    const int tid = threadIdx.x;
+    {
+        // Thread (rg, cp): channels 2 cp, 2 cp + 1 of sub-tile rg's 16 rows.
+        const int cp = tid & 63, rg = tid >> 6, c0 = 2 * cp;
+        const float eA0 = ex2_approx(A[(size_t)h * kDK + c0] * kLog2e);
+        const float eA1 = ex2_approx(A[(size_t)h * kDK + c0 + 1] * kLog2e);
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+            const int r = 16 * rg + i;
+            float2 kv = make_float2(0.f, 0.f), qv = kv;
+            if (r < loc.y) {
+                const size_t idx = ((size_t)(loc.x + r) * H + h) * kDK + c0;
+                const float2 zz = __bfloat1622float2(*(const __nv_bfloat162 *)(z + idx));
+                kv = __bfloat1622float2(*(const __nv_bfloat162 *)(k + idx));
+                qv = __bfloat1622float2(*(const __nv_bfloat162 *)(q + idx));
+                acc = add2(acc, make_float2(gate_softplus_fast(eA0, zz.x), gate_softplus_fast(eA1, zz.y)));
+            }
+            *(float2 *)&Ls[r * kPairLd + c0] = acc;
+            *(float2 *)&Ks[r * kPairLd + c0] = kv;
+            *(float2 *)&Qs[r * kPairLd + c0] = qv;
+        }
+    }
+    __syncthreads();
+    float *out = pairs + ((size_t)h * max_chunks + g) * 2048;
+    // 4 x 136 (s <= r) pairs; pair index e within a sub-tile: r (r + 1) / 2 + s.
+    for (int pidx = tid; pidx < 4 * 136; pidx += kPairThreads) {
+        const int I = pidx / 136, e = pidx - 136 * I;
+        int r = 0;
+        while ((r + 1) * (r + 2) / 2 <= e) ++r;
+        const int s = e - r * (r + 1) / 2;
+        const float *lr = Ls + (16 * I + r) * kPairLd, *ls = Ls + (16 * I + s) * kPairLd;
+        const float *kr = Ks + (16 * I + r) * kPairLd, *ks = Ks + (16 * I + s) * kPairLd;
+        const float *qr = Qs + (16 * I + r) * kPairLd;
+        float2 a = make_float2(0.f, 0.f), pp = a;
+#pragma unroll 8
+        for (int c = 0; c < kDK; c += 2) {
+            const float2 d = mul2(sub2(*(const float2 *)&lr[c], *(const float2 *)&ls[c]), log2e2());
+            const float2 kse = mul2(*(const float2 *)&ks[c], exp2_2(d));    // e^{L_r - L_s} <= 1
+            a = fma2(*(const float2 *)&kr[c], kse, a);
+            pp = fma2(*(const float2 *)&qr[c], kse, pp);
+        }
+        out[I * 256 + s * 16 + r] = a.x + a.y;
+        out[1024 + I * 256 + s * 16 + r] = pp.x + pp.y;
+    }
+}
+
 // ------------------------------------------------------------------ state --
 
-constexpr int kStateThreads = 320;       // epilogue: warps 0-7, load: 8, mma: 9
+// One CTA of 384 threads per (sequence, head) slot, in three roles:
+//   chain  (warps 0-7): the per-chunk state recurrence.  Thread (j, hh) owns
+//          TMEM lane j = value channel j and half hh of the delta rows, state
+//          columns and the chunk's key channels.  Thread 0 also issues the
+//          block loads and every tensor-core product, between group barriers,
+//          so that no hand-off to another warp sits on the chain.
+//   output (warps 8-11): reads O^T of each finished chunk from TMEM, rounds it
+//          to bf16 in a staging tile and stores whole token rows (one TMA
+//          tensor store per full chunk), off the chain.
+// Per chunk c (buffer b = c & 1 of the [delta | O] accumulator D1):
+//   D1[:, 0:64]   = S^T W^T         (commit -> mma1: the chain may form delta)
+//   D1[:, 64:128] = S^T Qt^T
+//   Dl^T = U^T - D1[:, 0:64]        -> bf16 into TMEM            (chain)
+//   S^T += Dl^T Kd,  D1[:, 64:] += Dl^T P^T   (commit -> mma2[b])
+//   S^T  -> bf16 copy (the next chunk's A operand), then the fp32 master times
+//           the next chunk's e^{G_C}                              (chain)
+//   O^T = D1[:, 64:] -> o                                         (output)
+constexpr int kStateThreads = 384;
+constexpr int kChainThreads = 256, kOutThreads = 128;
 constexpr uint32_t kStageBytes = 75776;  // block rounded up to 1 KiB
 constexpr int kStages = 2;
 constexpr uint32_t kOStage = kStages * kStageBytes;  // 2 x [64][128] bf16 output staging
 constexpr uint32_t kStateSmem = kStages * kStageBytes + 2 * 16384 + 1024;
 // TMEM columns
 constexpr uint32_t kTS = 0, kTSbf = 128, kTDl = 192, kTD1 = 256;  // D1 double buffer: 256, 384
+constexpr int kBarChain = 1, kBarOut = 2;                         // named barrier ids
 
 struct StateBars {
-    uint64_t full[kStages], empty[kStages];
-    uint64_t mma1, dl_ready, sbf_ready, sdec_ready;
-    uint64_t mma2[2], d1_free[2], ostaged[2];
+    uint64_t full[kStages];
+    uint64_t mma1, mma2[2], d1_free[2], drain;
 };
-constexpr uint32_t kEpi = 256;  // epilogue threads: two warpgroups
+
+// Barrier over `nthreads` threads of the CTA (named barrier `id`) that also
+// returns whether any of them passed `pred` = true, so a group leaves a loop
+// together when one of its threads saw a wait give up.
+__device__ __forceinline__ bool group_sync_any(int id, int nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
+        " barrier.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void group_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// One TMA tensor store: the [64 tokens][128 channels] bf16 tile at `smem_src`
+// to rows t0 .. t0 + 63 of head h of o (rows past T are not written).
+__device__ __forceinline__ void tma_store_rows(const CUtensorMap *map, const void *smem_src, int h,
+                                               int t0) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];"
+        ::"l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(h), "r"(t0), "r"(smem_u32(smem_src))
+        : "memory");
+}
 
 // Segments: with G > 1 every sequence of nch chunks is cut into Gn = min(G, nch)
 // runs of chunks, [s nch / Gn, (s + 1) nch / Gn), and each (sequence, head) gets
@@ -696,7 +920,8 @@ constexpr size_t kStateF32 = (size_t)kDK * kDV;  // one fp32 state, in floats
 // instantiation has no trace of it.
 template <bool DUMP>
 __global__ void __launch_bounds__(kStateThreads, 1)
-state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_off,
+state_kernel(const __grid_constant__ CUtensorMap tm_o,
+             const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_off,
              const int32_t *__restrict__ order, int N, int H,
              const uint8_t *__restrict__ blocks, int64_t max_chunks,
              const float *S0user, float *Sfuser, __nv_bfloat16 *__restrict__ o, int32_t *status,
@@ -708,9 +933,8 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
     uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
     __shared__ StateBars bars;
     __shared__ uint32_t tbase;
-    __shared__ volatile int sAbort;
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x, warp = tid >> 5;
     const int slots = 2 * G - 1;
     const int slot = blockIdx.x % slots;
     const int n = order[(blockIdx.x / slots) / H], h = (blockIdx.x / slots) % H;
@@ -736,18 +960,14 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
     const size_t fbase = Gn == 1 ? sbase : 0;  // Sf offset of this (sequence, head)
     uint8_t *eimg = xmode ? Eimg + ((size_t)h * max_chunks + chunk_off[n] + cbeg) * kEImg : nullptr;
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) { mbar_init(&bars.full[s], 1); mbar_init(&bars.empty[s], kEpi + 1); }
+        for (int s = 0; s < kStages; ++s) mbar_init(&bars.full[s], 1);
         mbar_init(&bars.mma1, 1);
-        mbar_init(&bars.dl_ready, kEpi);
-        mbar_init(&bars.sbf_ready, kEpi);
-        mbar_init(&bars.sdec_ready, kEpi);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars.mma2[b], 1);
-            mbar_init(&bars.d1_free[b], kEpi);
-            mbar_init(&bars.ostaged[b], kEpi);
+            mbar_init(&bars.d1_free[b], kOutThreads);
         }
+        mbar_init(&bars.drain, 1);
         fence_mbar_init();
-        sAbort = 0;
     }
     if (warp == 0) { tmem_alloc(&tbase, 512); tmem_relinquish(); }
     tc_fence_before_sync();
@@ -755,84 +975,62 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
     tc_fence_after_sync();
     const uint32_t tb = tbase;
     const uint8_t *blk0 = blocks + ((size_t)h * max_chunks + chunk_off[n] + cbeg) * kBlockBytes;
+    const uint32_t lq = 32 * (warp & 3);
 
-    if (warp == 8) {
-        // ---- loader: one bulk copy per chunk block into the stage ring ----
-        if (lane == 0) {
-            int issued = 0;
-            for (int c = 0; c < nch && !sAbort; ++c) {
-                const int s = c % kStages;
-                if (c >= kStages &&
-                    !mbar_wait(&bars.empty[s], ((c / kStages) - 1) & 1, globaltimer_ns() + kWaitNs)) {
-                    record_timeout(status); sAbort = 1; break;
-                }
-                mbar_arrive_expect_tx(&bars.full[s], kBlockBytes);
-                bulk_g2s(sm + s * kStageBytes, blk0 + (size_t)c * kBlockBytes, kBlockBytes, &bars.full[s]);
-                ++issued;
+    if (warp < 8) {
+        // ------------------------------------------------------- chain --
+        const int j = tid & 127, hh = warp >> 2;
+        uint32_t ra[32], rb[32];
+        bool bad = false;            // this thread saw a bounded wait give up
+        int loads = 0;               // block loads issued (thread 0)
+        bool issued_mma = false;     // thread 0 issued a product
+        auto load = [&](int c) {     // thread 0: block of chunk c into stage c % kStages
+            const int s = c % kStages;
+            mbar_arrive_expect_tx(&bars.full[s], kBlockBytes);
+            bulk_g2s(sm + s * kStageBytes, blk0 + (size_t)c * kBlockBytes, kBlockBytes, &bars.full[s]);
+            ++loads;
+        };
+        auto wait = [&](uint64_t *bar, uint32_t parity) {
+            if (!mbar_wait(bar, parity, globaltimer_ns() + kWaitNs)) {
+                record_timeout(status);
+                bad = true;
+                return false;
             }
-            // Drain: every issued copy has landed before the CTA may exit.
-            for (int c = max(0, issued - kStages); c < issued; ++c)
-                mbar_wait(&bars.full[c % kStages], (c / kStages) & 1, globaltimer_ns() + kWaitNs);
-        }
-    } else if (warp == 9) {
-        // ---- MMA issuer ----
-        if (lane == 0) {
-            const uint32_t id128 = idesc_bf16_f32(128, 128), id64 = idesc_bf16_f32(128, 64);
-            int c = 0;
-            for (; c < nch && !sAbort; ++c) {
-                const int s = c % kStages, b = c & 1;
-                const uint32_t st = smem_u32(sm + s * kStageBytes);
-                const uint32_t d1 = tmem_addr(tb, 0, kTD1 + 128 * b);
-                bool ok = mbar_wait(&bars.full[s], (c / kStages) & 1, globaltimer_ns() + kWaitNs) &&
-                          mbar_wait(&bars.sbf_ready, c & 1, globaltimer_ns() + kWaitNs) &&
-                          (c < 2 || mbar_wait(&bars.d1_free[b], ((c >> 1) - 1) & 1, globaltimer_ns() + kWaitNs));
-                if (!ok) { record_timeout(status); sAbort = 1; break; }
-                tc_fence_after_sync();
-                // D1 = S^T [W; Qt]^T  (M = dv, N = 128 tokens-by-two, K = dk)
+            return true;
+        };
+        // Thread 0: D1 = S^T [W; Qt]^T for chunk c, in two halves so that the
+        // delta half commits first.  Needs the block and a free D1 buffer.
+        auto issue_mma1 = [&](int c) {
+            const int s = c % kStages, b = c & 1;
+            if (!wait(&bars.full[s], (c / kStages) & 1)) return;
+            if (c >= 2 && !wait(&bars.d1_free[b], ((c >> 1) - 1) & 1)) return;
+            tc_fence_after_sync();
+            const uint32_t st = smem_u32(sm + s * kStageBytes);
+            const uint32_t d1 = tmem_addr(tb, 0, kTD1 + 128 * b);
+            const uint32_t id64 = idesc_bf16_f32(128, 64);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_ts(d1, tmem_addr(tb, 0, kTSbf + 8 * ks),
-                           desc_kmajor_sw128(st + kOffWQ + (ks >> 2) * 128 * 128 + (ks & 3) * 32),
-                           id128, ks > 0);
-                mma_commit(&bars.mma1);
-                if (!mbar_wait(&bars.dl_ready, c & 1, globaltimer_ns() + kWaitNs) ||
-                    !mbar_wait(&bars.sdec_ready, c & 1, globaltimer_ns() + kWaitNs)) {
-                    record_timeout(status); sAbort = 1; break;
-                }
-                tc_fence_after_sync();
-                // S^T += Dl^T Kd (N = dk, K = 64 tokens); O^T += Dl^T P^T (N = 64, K = 64)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_ts(tmem_addr(tb, 0, kTS), tmem_addr(tb, 0, kTDl + 8 * ks),
-                           desc_kmajor_sw128(st + kOffKd + ks * 32), id128, true);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_ts(d1 + 64, tmem_addr(tb, 0, kTDl + 8 * ks),
-                           desc_kmajor_sw128(st + kOffP + ks * 32), id64, true);
-                mma_commit(&bars.mma2[b]);
-                mma_commit(&bars.empty[s]);
+                    mma_ts(d1 + 64 * half, tmem_addr(tb, 0, kTSbf + 8 * ks),
+                           desc_kmajor_sw128(st + kOffWQ + (ks >> 2) * 128 * 128 + half * 8192 +
+                                             (ks & 3) * 32),
+                           id64, ks > 0);
+                if (half == 0) mma_commit(&bars.mma1);
             }
-            // Drain: wait for the last committed MMAs before exit.
-            if (c > 0) mbar_wait(&bars.mma2[(c - 1) & 1], ((c - 1) >> 1) & 1, globaltimer_ns() + kWaitNs);
-        }
-    } else {
-        // ---- epilogue, warps 0-7: thread j = TMEM lane = value channel j; half hh
-        // takes delta rows 32 hh .., state columns 64 hh .. and output rows 32 hh .. ----
-        const int j = tid & 127, hh = warp >> 2;
-        const uint32_t lq = 32 * (warp & 3);
-        uint32_t ra[32], rb[32];
+            issued_mma = true;
+        };
+        if (tid == 0)
+            for (int c = 0; c < nch && c < kStages; ++c) load(c);
+
         // Initial state: S^T row j = column j of S0 (this half's 64 key channels):
         // fp32 master pre-multiplied by the first chunk's decay, and the bf16 copy.
         // The transition X starts from the identity: X^T row j = e_j.
-        bool ok = true;
-        const float *dec0 = nullptr;
         const bool nonzero0 = S0 || xmode;
-        if (nonzero0) {
-            ok = mbar_wait(&bars.full[0], 0, globaltimer_ns() + kWaitNs);
-            if (!ok) { record_timeout(status); sAbort = 1; }
-            dec0 = (const float *)(sm + kOffDecay);
-        }
-        for (int q2 = 0; q2 < 2 && ok; ++q2) {
+        const float *dec0 = (const float *)(sm + kOffDecay);
+        if (nonzero0) wait(&bars.full[0], 0);
+        __syncwarp();
+        for (int q2 = 0; q2 < 2; ++q2) {
             const int c0 = 64 * hh + 32 * q2;
             float sv[32];
 #pragma unroll
@@ -848,56 +1046,19 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
         }
         tmem_st_wait();
         tc_fence_before_sync();
-        mbar_arrive(&bars.sbf_ready);
-        mbar_arrive(&bars.sdec_ready);
+        bool failed = group_sync_any(kBarChain, kChainThreads, bad);
+        if (!failed && tid == 0) issue_mma1(0);
 
-        // O^T rows of chunk cc -> o: each thread parks its 32 values in a [64][128]
-        // bf16 staging tile (double-buffered by chunk parity), then the 256
-        // threads write whole 256-byte token rows with 16-byte stores.
-        auto output = [&](int cc) {
-            const int bb = cc & 1;
-            const int t0 = tbeg + cc * kChunk;
-            const int len = min(kChunk, tend - t0);
-            __nv_bfloat16 *ost = (__nv_bfloat16 *)(sm + kOStage + bb * 16384);
-            tmem_ld32(tmem_addr(tb, lq, kTD1 + 128 * bb + 64 + 32 * hh), ra);
-            tmem_ld_wait();
-            tc_fence_before_sync();
-            mbar_arrive(&bars.d1_free[bb]);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ost[(32 * hh + i) * kDV + j] = __float2bfloat16_rn(__uint_as_float(ra[i]));
-            mbar_arrive(&bars.ostaged[bb]);
-            if (!mbar_wait(&bars.ostaged[bb], (cc >> 1) & 1, globaltimer_ns() + kWaitNs)) {
-                record_timeout(status);
-                sAbort = 1;
-                return;
-            }
-            const int r = tid >> 2, part = tid & 3;
-            const uint4 *src = (const uint4 *)(ost + r * kDV + 32 * part);
-            if (eimg) {
-                // E rows as the K-major, 128-byte-swizzled A operand of the
-                // correction product (two 64-wide K halves of 64 rows each).
-                uint8_t *dst = eimg + (size_t)cc * kEImg;
-#pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    *(uint4 *)(dst + ((32 * part + 8 * m) >> 6) * 8192 +
-                               sw128_offset(r, (32 * part + 8 * m) & 63, 64)) = src[m];
-            } else if (r < len) {
-                uint4 *dst = (uint4 *)(o + ((size_t)(t0 + r) * H + h) * kDV + 32 * part);
-#pragma unroll
-                for (int m = 0; m < 4; ++m) dst[m] = src[m];
-            }
-        };
-
-        for (int c = 0; c < nch && !sAbort; ++c) {
+        int c = 0;
+        for (; c < nch && !failed; ++c) {
             const int s = c % kStages, b = c & 1;
             const uint8_t *st = sm + s * kStageBytes;
-            if (!mbar_wait(&bars.full[s], (c / kStages) & 1, globaltimer_ns() + kWaitNs) ||
-                !mbar_wait(&bars.mma1, c & 1, globaltimer_ns() + kWaitNs)) {
-                record_timeout(status); sAbort = 1; break;
-            }
+            wait(&bars.full[s], (c / kStages) & 1);   // U of this block (already landed)
+            wait(&bars.mma1, c & 1);
+            __syncwarp();
             tc_fence_after_sync();
-            // Dl^T[j][r] = U[r][j] - D1[j][r] for this half's 32 rows -> bf16 pairs into TMEM
-            // (U = 0 on the transition).
+            // Dl^T[j][r] = U[r][j] - D1[j][r] for this half's 32 rows -> bf16 pairs into
+            // TMEM (U = 0 on the transition).
             {
                 const __nv_bfloat16 *U = (const __nv_bfloat16 *)(st + kOffU);
                 tmem_ld32(tmem_addr(tb, lq, kTD1 + 128 * b + 32 * hh), ra);
@@ -931,16 +1092,28 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
                 tmem_st_wait();
             }
             tc_fence_before_sync();
-            mbar_arrive(&bars.dl_ready);
-            mbar_arrive(&bars.empty[s]);  // done with U of this stage
-            // The previous chunk's output, off the critical path (its D1 buffer is
-            // only reused by the product two chunks later).
-            if (c > 0) output(c - 1);
-
-            if (!mbar_wait(&bars.mma2[b], (c >> 1) & 1, globaltimer_ns() + kWaitNs)) {
-                record_timeout(status); sAbort = 1; break;
+            if ((failed = group_sync_any(kBarChain, kChainThreads, bad))) break;
+            if (tid == 0) {
+                // S^T += Dl^T Kd (N = dk, K = 64 tokens); O^T += Dl^T P^T (N = 64, K = 64)
+                tc_fence_after_sync();
+                const uint32_t id128 = idesc_bf16_f32(128, 128), id64 = idesc_bf16_f32(128, 64);
+                const uint32_t sa = smem_u32(st);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_ts(tmem_addr(tb, 0, kTS), tmem_addr(tb, 0, kTDl + 8 * ks),
+                           desc_kmajor_sw128(sa + kOffKd + ks * 32), id128, true);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_ts(tmem_addr(tb, 0, kTD1 + 128 * b + 64), tmem_addr(tb, 0, kTDl + 8 * ks),
+                           desc_kmajor_sw128(sa + kOffP + ks * 32), id64, true);
+                mma_commit(&bars.mma2[b]);
+                issued_mma = true;
             }
+            const bool done2 = wait(&bars.mma2[b], (c >> 1) & 1);
+            __syncwarp();
             tc_fence_after_sync();
+            // Stage s is consumed (products done, U read before the barrier): refill it.
+            if (tid == 0 && done2 && c + kStages < nch) load(c + kStages);
             const bool last = (c + 1 == nch);
             // S_out, this half's 64 key channels: two loads, one wait.
             tmem_ld32(tmem_addr(tb, lq, kTS + 64 * hh), ra);
@@ -964,8 +1137,10 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
                         Sf[fbase + (size_t)(64 * hh + 32 + i) * kDV + j] = __uint_as_float(rb[i]);
                     }
                 }
-            } else {
-                // Critical: the bf16 copy that the next chunk's first product reads.
+                break;
+            }
+            // Critical: the bf16 copy that the next chunk's first product reads.
+            {
                 uint32_t sa[16], sbv[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -975,27 +1150,98 @@ state_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk_o
                 tmem_st16(tmem_addr(tb, lq, kTSbf + 32 * hh), sa);
                 tmem_st16(tmem_addr(tb, lq, kTSbf + 32 * hh + 16), sbv);
                 tmem_st_wait();
-                tc_fence_before_sync();
-                mbar_arrive(&bars.sbf_ready);
-                // Off the critical path: the fp32 master times the next chunk's decay.
-                const int s1 = (c + 1) % kStages;
-                if (!mbar_wait(&bars.full[s1], ((c + 1) / kStages) & 1, globaltimer_ns() + kWaitNs)) {
-                    record_timeout(status); sAbort = 1; break;
-                }
-                const float *dec = (const float *)(sm + s1 * kStageBytes + kOffDecay) + 64 * hh;
+            }
+            tc_fence_before_sync();
+            if ((failed = group_sync_any(kBarChain, kChainThreads, bad))) break;
+            if (tid == 0) issue_mma1(c + 1);
+            // Off the critical path: the fp32 master times the next chunk's decay
+            // (done before the next barrier, which precedes the product that adds to it).
+            const int s1 = (c + 1) % kStages;
+            wait(&bars.full[s1], ((c + 1) / kStages) & 1);
+            __syncwarp();
+            const float *dec = (const float *)(sm + s1 * kStageBytes + kOffDecay) + 64 * hh;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    ra[i] = __float_as_uint(__uint_as_float(ra[i]) * dec[i]);
-                    rb[i] = __float_as_uint(__uint_as_float(rb[i]) * dec[32 + i]);
-                }
-                tmem_st32(tmem_addr(tb, lq, kTS + 64 * hh), ra);
-                tmem_st32(tmem_addr(tb, lq, kTS + 64 * hh + 32), rb);
-                tmem_st_wait();
-                tc_fence_before_sync();
-                mbar_arrive(&bars.sdec_ready);
+            for (int i = 0; i < 32; ++i) {
+                ra[i] = __float_as_uint(__uint_as_float(ra[i]) * dec[i]);
+                rb[i] = __float_as_uint(__uint_as_float(rb[i]) * dec[32 + i]);
+            }
+            tmem_st32(tmem_addr(tb, lq, kTS + 64 * hh), ra);
+            tmem_st32(tmem_addr(tb, lq, kTS + 64 * hh + 32), rb);
+            tmem_st_wait();
+            tc_fence_before_sync();
+        }
+        if (tid == 0) {
+            // Drain: every issued copy has landed and every committed product has
+            // finished before the CTA may exit (bounded waits; a timeout is recorded).
+            for (int d = max(0, loads - kStages); d < loads; ++d)
+                mbar_wait(&bars.full[d % kStages], (d / kStages) & 1, globaltimer_ns() + kWaitNs);
+            if (issued_mma) {
+                // One more commit tracks every product this thread issued.
+                mma_commit(&bars.drain);
+                mbar_wait(&bars.drain, 0, globaltimer_ns() + kWaitNs);
             }
         }
-        if (!sAbort) output(nch - 1);  // the last chunk's output
+    } else {
+        // ------------------------------------------------------ output --
+        const int j = tid - kChainThreads;        // TMEM lane = value channel
+        const int Ttot = cu[N];                   // rows past it are clipped by the TMA store
+        bool failed = false;
+        for (int c = 0; c < nch; ++c) {
+            const int b = c & 1;
+            const int t0 = tbeg + c * kChunk, len = min(kChunk, tend - t0);
+            const bool ok = mbar_wait(&bars.mma2[b], (c >> 1) & 1, globaltimer_ns() + kWaitNs);
+            if (!ok) record_timeout(status);
+            __syncwarp();
+            tc_fence_after_sync();
+            uint32_t oa[32], ob[32];
+            tmem_ld32(tmem_addr(tb, lq, kTD1 + 128 * b + 64), oa);
+            tmem_ld32(tmem_addr(tb, lq, kTD1 + 128 * b + 96), ob);
+            tmem_ld_wait();
+            tc_fence_before_sync();
+            mbar_arrive(&bars.d1_free[b]);
+            // Staging buffer c & 1 is free once the stores issued from it (two
+            // chunks ago) have read it; waiting for every earlier store is simpler
+            // and costs nothing here.
+            if (j == 0) bulk_wait_read<0>();
+            __syncwarp();
+            if ((failed = group_sync_any(kBarOut, kOutThreads, !ok))) break;
+            uint8_t *ost = sm + kOStage + (c & 1) * 16384;
+            if (eimg) {
+                // E rows as the K-major, 128-byte-swizzled A operand of the
+                // correction product (two 64-wide K halves of 64 rows each).
+                const uint32_t kh = (uint32_t)(j >> 6) * 8192u;
+#pragma unroll
+                for (int r = 0; r < 32; ++r) {
+                    *(__nv_bfloat16 *)(ost + kh + sw128_offset(r, j & 63, 64)) =
+                        __float2bfloat16_rn(__uint_as_float(oa[r]));
+                    *(__nv_bfloat16 *)(ost + kh + sw128_offset(r + 32, j & 63, 64)) =
+                        __float2bfloat16_rn(__uint_as_float(ob[r]));
+                }
+            } else {
+                __nv_bfloat16 *ot = (__nv_bfloat16 *)ost;
+#pragma unroll
+                for (int r = 0; r < 32; ++r) {
+                    ot[r * kDV + j] = __float2bfloat16_rn(__uint_as_float(oa[r]));
+                    ot[(r + 32) * kDV + j] = __float2bfloat16_rn(__uint_as_float(ob[r]));
+                }
+            }
+            fence_proxy_async_smem();
+            group_sync(kBarOut, kOutThreads);
+            if (eimg) {
+                if (j == 0) { bulk_s2g(eimg + (size_t)c * kEImg, ost, kEImg); bulk_commit(); }
+            } else if (len == kChunk || tend == Ttot) {
+                if (j == 0) { tma_store_rows(&tm_o, ost, h, t0); bulk_commit(); }
+            } else {
+                // A ragged last chunk inside the packed batch: plain stores of its rows.
+                for (int e = j; e < len * 16; e += kOutThreads) {
+                    const int r = e >> 4, part = e & 15;
+                    *(uint4 *)(o + ((size_t)(t0 + r) * H + h) * kDV + 8 * part) =
+                        *(const uint4 *)(ost + (r * kDV + 8 * part) * 2);
+                }
+            }
+        }
+        (void)failed;
+        if (j == 0) bulk_wait<0>();   // every store has completed before the CTA exits
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -1218,11 +1464,11 @@ debug_gate_kernel(const __nv_bfloat16 *__restrict__ z, const float *__restrict__
     if (g >= chunk_off[N]) return;
     const int2 loc = chunk_loc[g];
     const int c = threadIdx.x;
-    const float eA = __expf(A[(size_t)h * kDK + c]);
+    const float eAn = -ex2_approx(A[(size_t)h * kDK + c] * kLog2e) * kLog2e;
     float acc = 0.f;
     for (int r = 0; r < loc.y; ++r) {
         const size_t idx = ((size_t)(loc.x + r) * H + h) * kDK + c;
-        acc += gate_log_decay_fast(eA, __bfloat162float(z[idx]));
+        acc += gate_fast(eAn, __bfloat162float(z[idx]));
         Gout[idx] = acc;
     }
 }
@@ -1280,6 +1526,22 @@ bool encode_rows_map(CUtensorMap *map, const void *base, int32_t T, int32_t H)
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// o [T][H][128] bf16 as a 3-D tensor (channel, head, token) with a {128, 1, 64}
+// box and no swizzle: one chunk's output rows of one head per TMA store, from
+// a dense [64][128] staging tile.
+bool encode_out_map(CUtensorMap *map, void *base, int32_t T, int32_t H)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)kDV, (cuuint64_t)H, (cuuint64_t)(T > 0 ? T : 1)};
+    const cuuint64_t strides[2] = {(cuuint64_t)kDV * 2, (cuuint64_t)H * kDV * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)kDV, 1, (cuuint32_t)kChunk};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 namespace {
@@ -1292,10 +1554,12 @@ constexpr int64_t kMaxSegments = 16;
 // blocks, then (split only)
 // Sx and Mx [N][G][H] fp32 states, S_in images [N][G][H] and E images [H][chunks].
 struct WsLayout {
-    size_t plan, loc, blocks, sx, mx, simg, eimg, total;
+    size_t plan, loc, blocks, sx, mx, simg, eimg, pairs, total;
 };
 
-WsLayout ws_layout(int32_t total_tokens, int32_t num_seqs, int32_t H, int G)
+// With the unbounded gate the layout ends with the pair kernel's diagonal
+// tiles: 8 KiB per (chunk, head).
+WsLayout ws_layout(int32_t total_tokens, int32_t num_seqs, int32_t H, int G, int gate = kGateBounded)
 {
     WsLayout w{};
     if (num_seqs <= 0) return w;
@@ -1312,6 +1576,10 @@ WsLayout ws_layout(int32_t total_tokens, int32_t num_seqs, int32_t H, int G)
         w.simg = w.mx + states * kStateF32 * sizeof(float);
         w.eimg = w.simg + states * kSinImg;
         end = w.eimg + (size_t)H * max_chunks * kEImg;
+    }
+    if (gate == kGateSoftplus) {
+        w.pairs = up(end);
+        end = w.pairs + (size_t)H * max_chunks * 2048 * sizeof(float);
     }
     w.total = end;
     return w;
@@ -1336,9 +1604,9 @@ int tc_split_segments(int32_t total_tokens, int32_t num_seqs, int32_t H, bool fo
     return G < 2 ? 1 : (int)G;
 }
 
-size_t tc_workspace_bytes(int32_t total_tokens, int32_t num_seqs, int32_t H, int segments)
+size_t tc_workspace_bytes(int32_t total_tokens, int32_t num_seqs, int32_t H, int segments, int gate)
 {
-    return ws_layout(total_tokens, num_seqs, H, segments).total;
+    return ws_layout(total_tokens, num_seqs, H, segments, gate).total;
 }
 
 cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream)
@@ -1347,7 +1615,8 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
     const int G = a.segments > 1 ? a.segments : 1;
     if (G > 1 && a.ckpt_every > 0) return cudaErrorInvalidValue;
     const int64_t max_chunks = ((int64_t)a.total_tokens + 63LL * a.num_seqs) / kChunk;
-    const WsLayout w = ws_layout(a.total_tokens, a.num_seqs, a.H, G);
+    const bool softplus = a.gate == kGateSoftplus;
+    const WsLayout w = ws_layout(a.total_tokens, a.num_seqs, a.H, G, a.gate);
     uint8_t *ws = (uint8_t *)a.workspace;
     int32_t *chunk_off = (int32_t *)ws;
     int32_t *ckpt_off = chunk_off + a.num_seqs + 1;
@@ -1360,13 +1629,19 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
     uint8_t *Eimg = G > 1 ? ws + w.eimg : nullptr;
     cudaError_t err;
 
-    err = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto intra_fn = softplus ? intra_kernel<kGateSoftplus> : intra_kernel<kGateBounded>;
+    err = cudaFuncSetAttribute(intra_fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)(kISmem + 1024));
     if (err != cudaSuccess) return err;
     // Two intra CTAs share an SM: ask for the largest shared-memory carveout.
-    err = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+    err = cudaFuncSetAttribute(intra_fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                                (int)cudaSharedmemCarveoutMaxShared);
     if (err != cudaSuccess) return err;
+    if (softplus) {
+        err = cudaFuncSetAttribute(diag_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)kPairSmem);
+        if (err != cudaSuccess) return err;
+    }
     auto state_fn = a.dbg_delta ? state_kernel<true> : state_kernel<false>;
     err = cudaFuncSetAttribute(state_fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem);
     if (err != cudaSuccess) return err;
@@ -1396,16 +1671,27 @@ cudaError_t launch_prefill_tensor_core(const PrefillArgs &a, cudaStream_t stream
         if (!encode_rows_map(&mk, a.k, a.total_tokens, a.H) || !encode_rows_map(&mq, a.q, a.total_tokens, a.H) ||
             !encode_rows_map(&mv, a.v, a.total_tokens, a.H) || !encode_rows_map(&mz, a.z, a.total_tokens, a.H))
             return cudaErrorInvalidValue;
-        intra_kernel<<<grid, kIntraThreads, kISmem + 1024, stream>>>(
+        float *pairs = softplus ? (float *)(ws + w.pairs) : nullptr;
+        if (softplus) {
+            diag_pair_kernel<<<(unsigned)(max_chunks * a.H), kPairThreads, kPairSmem, stream>>>(
+                (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.z,
+                a.A, chunk_loc, chunk_off, a.num_seqs, a.H, max_chunks, pairs);
+            if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        }
+        intra_fn<<<grid, kIntraThreads, kISmem + 1024, stream>>>(
             mk, mq, mv, mz, a.A, a.beta, chunk_loc, chunk_off, a.num_seqs, a.H,
-            blocks, max_chunks, a.status);
+            blocks, max_chunks, a.status, pairs);
         err = cudaGetLastError();
         if (err != cudaSuccess) return err;
     }
     a.mark(2, stream);
+    CUtensorMap mo;
+    memset(&mo, 0, sizeof(mo));  // with no tokens (o may be null) no chunk stores anything
+    if (a.total_tokens > 0 && !encode_out_map(&mo, a.o, a.total_tokens, a.H))
+        return cudaErrorInvalidValue;
     state_fn<<<(unsigned)((int64_t)a.num_seqs * a.H * (2 * G - 1)), kStateThreads, kStateSmem,
                stream>>>(
-        a.cu_seqlens, chunk_off, order, a.num_seqs, a.H, blocks, max_chunks, a.initial_state,
+        mo, a.cu_seqlens, chunk_off, order, a.num_seqs, a.H, blocks, max_chunks, a.initial_state,
         a.final_state, (__nv_bfloat16 *)a.o, a.status, a.ckpt_every, ckpt_off, a.checkpoints,
         G, Sx, Mx, Eimg, a.dbg_delta);
     a.mark(3, stream);

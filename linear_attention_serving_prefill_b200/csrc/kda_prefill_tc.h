@@ -21,7 +21,10 @@ int tc_split_segments(int32_t total_tokens, int32_t num_seqs, int32_t H, bool fo
 // block of MMA-ready tiles per (chunk, head), for the worst case of
 // floor((T + 63 N) / 64) chunks; with segments > 1 also the segment states,
 // transitions, S_in images (N G H of each) and 16 KiB E images per (chunk, head).
-size_t tc_workspace_bytes(int32_t total_tokens, int32_t num_seqs, int32_t H, int segments);
+// With gate == 1 (the unbounded Softplus gate) it also holds the pair kernel's
+// diagonal tiles, 8 KiB per (chunk, head).
+size_t tc_workspace_bytes(int32_t total_tokens, int32_t num_seqs, int32_t H, int segments,
+                          int gate = 0);
 
 // Launches plan, intra-chunk and state kernels on `stream`, then, when
 // a.segments > 1, the segment composition and the output correction.

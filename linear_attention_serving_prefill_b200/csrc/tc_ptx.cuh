@@ -53,13 +53,60 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete.  Gives up (returns
-// false) once the global timer passes `deadline_ns`.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t deadline_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
+// Non-blocking test of the phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits by polling test_wait, for latency-critical hand-offs where the waiting
+// warps have nothing else to do; the deadline is checked every 64 polls.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity, uint64_t deadline_ns) {
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_test_wait(bar, parity)) return true;
         if (globaltimer_ns() > deadline_ns) return false;
+    }
+}
+
+// try_wait with a suspend-time hint: the thread may be suspended for up to
+// `hint_ns` while the phase is incomplete, and resumes when it completes.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete.  Gives up (returns
+// false) once the global timer passes `deadline_ns`.  With SUSPEND_NS > 0 each
+// try_wait may suspend the thread for up to that long (it resumes when the
+// phase completes), so that waiting warps stop taking issue slots from the
+// warps that still work; the deadline is checked between tries.
+template <uint32_t SUSPEND_NS = 0>
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t deadline_ns) {
+    if (SUSPEND_NS == 0) {
+        if (mbar_try_wait(bar, parity)) return true;
+        while (true) {
+            if (mbar_try_wait(bar, parity)) return true;
+            if (globaltimer_ns() > deadline_ns) return false;
+        }
+    } else {
+        while (true) {
+            if (mbar_try_wait_hint(bar, parity, SUSPEND_NS)) return true;
+            if (globaltimer_ns() > deadline_ns) return false;
+        }
     }
 }
 
@@ -73,6 +120,12 @@ __device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gmem_src, u
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
         ::"r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Asks the TMA engine to bring `bytes` of global memory into L2 (no completion
+// to wait for).  Address 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *gmem_src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem_src), "r"(bytes) : "memory");
 }
 
 // One contiguous shared -> global copy on the TMA engine, in the thread's

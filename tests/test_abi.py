@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_abi_version_and_status_strings():
-    assert B._lib.kda_abi_version() == 2
+    assert B._lib.kda_abi_version() == 3
     for code in range(6):
         s = B.kda_status_string(code)
         assert s.startswith(B.STATUS_NAMES[code])
@@ -206,6 +206,18 @@ def test_noalloc_rejects_calls_beyond_its_scratch_limit():
     assert B._lib.kda_prefill_noalloc(*args) == UNSUPPORTED
 
 
+def test_noalloc_limit_edge_is_576_tokens_at_96_heads():
+    """The scratch limit (64 MiB) against the tensor-core workspace: one sequence
+    of 576 tokens at 96 heads (9 chunks) fits, 577 tokens (10 chunks) does not,
+    and neither do two sequences of 288 (their ragged-tail bound is 9 chunks + 1)."""
+    limit = 64 << 20
+    assert B.kda_prefill_workspace_size(576, 1, 96, 128, 128, torch.bfloat16, "tensor_core") <= limit
+    assert B.kda_prefill_workspace_size(577, 1, 96, 128, 128, torch.bfloat16, "tensor_core") > limit
+    assert B.kda_prefill_workspace_size(576, 2, 96, 128, 128, torch.bfloat16, "tensor_core") > limit
+    args = [_fake()] * 6 + [_fake(), None, 1, 577, 96, 128, 128, BF16, None, None, _fake(), None]
+    assert B._lib.kda_prefill_noalloc(*args) == WORKSPACE
+
+
 def test_selftest_rejects_out_of_range_limits():
     assert B._lib.kda_selftest_wait_timeout(0, None) == INVALID
     assert B._lib.kda_selftest_wait_timeout(20_000_000_000, None) == INVALID
@@ -248,14 +260,22 @@ def test_decode_multi_rejects_bad_arguments():
 
 
 def test_gated_entry_points_validate_the_gate():
-    """The unbounded gate runs on the CUDA-core path only; a gate outside the
-    enum is rejected before anything is launched."""
-    def gated(algo, gate, dt=BF16, dk=128, dv=128):
+    """The unbounded gate on the tensor-core path needs its larger workspace
+    (the pair kernel's diagonal tiles); fp32 or d != 128 cannot take that path;
+    a gate outside the enum is rejected before anything is launched."""
+    def gated(algo, gate, dt=BF16, dk=128, dv=128, ws=None, ws_bytes=0):
         return B._lib.kda_prefill_gated(_fake(), _fake(), _fake(), _fake(), _fake(), _fake(),
                                         _fake(), None, 2, 10, 4, dk, dv, dt, None, None, _fake(),
-                                        None, 0, algo, gate, None)
-    assert gated(TC, 1) == UNSUPPORTED
-    assert gated(SPLIT, 1) == UNSUPPORTED
+                                        ws, ws_bytes, algo, gate, None)
+    size = B._lib.kda_prefill_gated_workspace_size
+    bounded, unbounded = size(10, 2, 4, 128, 128, BF16, TC, 0), size(10, 2, 4, 128, 128, BF16, TC, 1)
+    assert bounded == B._lib.kda_prefill_workspace_size(10, 2, 4, 128, 128, BF16, TC)
+    # two (chunk, head) tiles per head here: (10 + 63 * 2) // 64 = 2 chunks x 4 heads x 8 KiB
+    assert unbounded >= bounded + 2 * 4 * 8192
+    assert size(10, 2, 4, 128, 128, BF16, CORE, 1) == 0
+    assert size(10, 2, 4, 128, 128, BF16, TC, 5) == 0
+    assert gated(TC, 1, ws=_fake(), ws_bytes=bounded) == WORKSPACE
+    assert gated(SPLIT, 1, ws=None, ws_bytes=0) == WORKSPACE
     assert gated(AUTO, 7) == INVALID
     assert gated(CORE, -1) == INVALID
     assert gated(TC, 1, dt=F32) == UNSUPPORTED

@@ -308,12 +308,16 @@ def test_split_with_empty_and_single_chunk_sequences_interleaved():
 
 # ------------------------------------------------- unbounded (Softplus) gate ----
 
-@pytest.mark.parametrize("dtype,tol", [("f32", TOL_F32), ("bf16", TOL_BF16)])
+@pytest.mark.parametrize("algo,dtype,tol", [("cuda_core", "f32", TOL_F32), ("cuda_core", "bf16", TOL_BF16),
+                                            ("tensor_core", "bf16", TOL_BF16),
+                                            ("tensor_core_split", "bf16", TOL_BF16)])
 @pytest.mark.parametrize("z_mean", [0.0, 3.0])
-def test_softplus_gate_prefill_matches_oracle(dtype, tol, z_mean):
-    """The unbounded gate on the CUDA-core path (position-pair diagonal tiles).
-    At z_mean = 3 a 16-token cumulative log-decay reaches well below -88, where
-    the dense tile form's e^{-G} would overflow fp32."""
+def test_softplus_gate_prefill_matches_oracle(algo, dtype, tol, z_mean):
+    """The unbounded gate: on the CUDA-core path (every 16-token chunk pair by
+    pair) and on the tensor-core path (off-diagonal sub-tile pairs on tcgen05,
+    the diagonal 16 x 16 tiles pair by pair).  At z_mean = 3 a 16-token
+    cumulative log-decay reaches well below -88, where the dense tile form's
+    e^{-G} would overflow fp32."""
     lengths = [1, 15, 16, 17, 100, 0, 257]
     x = _cuda(prefill_inputs(lengths, 3, 128, 128, dtype, seed=70 + int(z_mean), s0_std=0.02,
                              z_mean=z_mean))
@@ -323,8 +327,10 @@ def test_softplus_gate_prefill_matches_oracle(dtype, tol, z_mean):
         # tokens 165..180: one 16-token chunk of the 257-token sequence (starts at 149)
         assert np.cumsum(g[165:181], axis=0).min() < -88.0
     o, S = K.kda_prefill(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"], x["cu_seqlens"],
-                         x["cu_seqlens_host"], initial_state=x["initial_state"], gate="softplus")
+                         x["cu_seqlens_host"], initial_state=x["initial_state"], gate="softplus",
+                         algo=algo)
     torch.cuda.synchronize()
+    assert K.kda_device_status() == 0
     assert torch.isfinite(o).all() and torch.isfinite(S).all()
     n, H = len(lengths), 3
     ref_o, ref_S, tok = oracle_subset(x, list(range(n)), list(range(H)), gate="softplus")
@@ -332,14 +338,15 @@ def test_softplus_gate_prefill_matches_oracle(dtype, tol, z_mean):
     assert relerr(got_o, ref_o) <= tol and relerr(got_S, ref_S) <= tol
 
 
-def test_softplus_gate_saturated_decay():
+@pytest.mark.parametrize("algo", ["cuda_core", "tensor_core"])
+def test_softplus_gate_saturated_decay(algo):
     """z = 60: per-token log-decay far below the -110 clamp, the state is wiped
     at every step; both sides agree and nothing overflows."""
     x = _cuda(prefill_inputs([70, 33], 2, 128, 128, "bf16", seed=72, s0_std=0.5, z_mean=60.0,
                              z_std=0.0))
     o, S = K.kda_prefill(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"], x["cu_seqlens"],
                          x["cu_seqlens_host"], initial_state=x["initial_state"], gate="softplus",
-                         algo="cuda_core")
+                         algo=algo)
     torch.cuda.synchronize()
     assert torch.isfinite(o).all() and torch.isfinite(S).all()
     ref_o, ref_S, tok = oracle_subset(x, [0, 1], [0, 1], gate="softplus")
@@ -367,6 +374,25 @@ def test_softplus_gate_bounded_inputs_differ_from_bounded_gate():
     assert code == 0
     assert torch.equal(o_g, o_b) and torch.equal(S_g, S_b)
     assert (o_s - o_b).abs().max().item() > 1e-3
+
+
+def test_softplus_gate_tensor_core_long_sequence_sampled_heads():
+    """The unbounded gate's tensor-core path on 4,096 tokens x 8 heads at the
+    workload distributions (every element of o and S), and its agreement with
+    the bounded gate's path when the Softplus decay is mild enough that both
+    read the same inputs differently (the selector is live)."""
+    x = _cuda(prefill_inputs([4096], 8, 128, 128, "bf16", seed=75, s0_std=0.02))
+    o, S = K.kda_prefill(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"], x["cu_seqlens"],
+                         x["cu_seqlens_host"], initial_state=x["initial_state"], gate="softplus",
+                         algo="tensor_core")
+    ob, _ = K.kda_prefill(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"], x["cu_seqlens"],
+                          x["cu_seqlens_host"], initial_state=x["initial_state"], algo="tensor_core")
+    torch.cuda.synchronize()
+    assert K.kda_device_status() == 0
+    ref_o, ref_S, tok = oracle_subset(x, [0], list(range(8)), gate="softplus")
+    got_o, got_S = gpu_subset(o, S, tok, [0], list(range(8)))
+    assert relerr(got_o, ref_o) <= TOL_BF16 and relerr(got_S, ref_S) <= TOL_BF16
+    assert (o.float() - ob.float()).abs().max().item() > 1e-2
 
 
 @pytest.mark.parametrize("dtype,tol", [("f32", TOL_F32), ("bf16", TOL_BF16)])
