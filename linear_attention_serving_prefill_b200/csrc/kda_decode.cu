@@ -10,7 +10,7 @@
 // once.  That is the minimum traffic, 2 * dk * dv * 4 bytes per (sequence,
 // head), so the kernel is bound by HBM bandwidth.  One CTA of 256 threads owns
 // one (sequence, head); thread (rg, cg) holds rows rg, rg + RG, ... of float4
-// column group cg.
+// column group cg, so that every warp reads whole 512-byte rows of the state.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -83,11 +83,24 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     __syncthreads();
 
     if (tid < CG) {
-        float4 tv = sRedV[0][tid], tp = sRedP[0][tid];
-        for (int r = 1; r < RG; ++r) {
-            const float4 a = sRedV[r][tid], c = sRedP[r][tid];
-            tv.x += a.x; tv.y += a.y; tv.z += a.z; tv.w += a.w;
-            tp.x += c.x; tp.y += c.y; tp.z += c.z; tp.w += c.w;
+        // Sum of the RG row-group partials as a pairwise tree, ((0+1)+(2+3))+...,
+        // the order of the multi-token kernel's xor butterfly over its 8 row
+        // groups: at dv = 128 (RG = 8, rows rg + 8 i in both kernels) a one-token
+        // replay there equals this step bit for bit.
+        float4 tv, tp;
+        {
+            float4 v[RG], pp[RG];
+#pragma unroll
+            for (int r = 0; r < RG; ++r) { v[r] = sRedV[r][tid]; pp[r] = sRedP[r][tid]; }
+#pragma unroll
+            for (int w = 1; w < RG; w <<= 1)
+#pragma unroll
+                for (int r = 0; r + w < RG; r += 2 * w) {
+                    v[r].x += v[r + w].x; v[r].y += v[r + w].y; v[r].z += v[r + w].z; v[r].w += v[r + w].w;
+                    pp[r].x += pp[r + w].x; pp[r].y += pp[r + w].y; pp[r].z += pp[r + w].z; pp[r].w += pp[r + w].w;
+                }
+            tv = v[0];
+            tp = pp[0];
         }
         const float bt = beta[tok];
         const size_t vo = tok * DV + (size_t)tid * 4;

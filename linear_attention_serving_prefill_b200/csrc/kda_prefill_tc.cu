@@ -61,7 +61,13 @@ constexpr uint64_t kWaitNs = 2000000000ull;  // per-wait limit: 2 s
 constexpr uint32_t kOffWQ = 0;         // [W; Qt] 128 rows x 128 K, swizzled K-major
 constexpr uint32_t kOffKd = 32768;     // Kd^T 128 rows (key channel) x 64 K (token)
 constexpr uint32_t kOffP = 49152;      // P 64 rows x 64 K
-constexpr uint32_t kOffU = 57344;      // U row-major [64][128] bf16
+constexpr uint32_t kOffU = 57344;      // U [64][128] bf16, 16-byte chunks swizzled per row
+// Byte offset of U[r][j] in its region: row r holds 16 chunks of 8 channels, chunk
+// index XORed with r % 16, so that 16 consecutive rows' stores of one chunk and
+// one row's loads of 32 consecutive channels both spread over the banks.
+__host__ __device__ __forceinline__ uint32_t u_offset(uint32_t r, uint32_t j) {
+    return r * 256u + ((((j >> 3) ^ r) & 15u) << 4) + ((j & 7u) << 1);
+}
 constexpr uint32_t kOffDecay = 73728;  // e^{G_C} [128] fp32
 constexpr uint32_t kBlockBytes = 74240;
 
@@ -166,17 +172,23 @@ constexpr int kIntraThreads = 256;
 constexpr uint32_t kIntraSuspendNs = 20000;
 constexpr uint32_t kRawTile = kChunk * kDK * 2;    // one [64][128] bf16 tile, 16 KiB
 // Shared memory (offsets from a 1024-aligned base).  The raw k, q, v, z tiles
-// arrive by two 128-byte-swizzled TMA boxes each, as K-major operand images
-// [K half][64 rows][128 B]: element (r, c) at sw128_offset(r, c, 64).
-constexpr uint32_t kRawK = 0, kRawQ = kRawTile, kRawV = 2 * kRawTile, kRawZ = 3 * kRawTile;
-// A operands of the A/P products, R^(I) = k e^{m_I - G} scaled to sub-tile I's
-// reference: one 64-row image per (sub-tile I, K half), of which only rows
-// 0 .. 16 I + 15 are valid.  Each region starts where the previous region's
-// valid rows end; a product reads the rows past them (the next regions, or the
-// end of the area) into outputs it discards.  Valid bytes of (I, kb): 2048 (I + 1).
+// arrive by two 128-byte-swizzled TMA boxes each (one per K half of 64
+// channels), as K-major operand images of 64 rows x 128 B.  k and q are
+// interleaved by K half, [k K0 | q K0 | k K1 | q K1], so that after pass 2 each
+// K half holds the 128-row operand [K e^L; Q e^L] of the A/P product:
+// element (r, c) of k at kq_offset(r, c), of q 8 KiB further.  v and z are
+// [K0 | K1]: element (r, c) at sw128_offset(r, c, 64).
+constexpr uint32_t kRawK = 0, kRawQ = 8192, kRawV = 2 * kRawTile, kRawZ = 3 * kRawTile;
+__host__ __device__ __forceinline__ uint32_t kq_offset(uint32_t r, uint32_t c) {
+    return (c >> 6) * 16384u + sw128_offset(r, c & 63, 64);
+}
+// B operand of the A/P product: the images R^(I) = k e^{m_I - G} (rows 0 ..
+// 16 I + 15, scaled to sub-tile I's reference) stacked per K half, 16 + 32 + 48
+// + 64 = 160 rows of 128 B: R^(I) starts at row 8 I (I + 1).
 constexpr uint32_t kIR = 4 * kRawTile;
+constexpr uint32_t kRStack = 160 * 128;             // one K half of the stack: 20 KiB
 __host__ __device__ constexpr uint32_t r_region(int I, int kb) {
-    return kIR + 2048u * (uint32_t)(I * (I + 1) + kb * (I + 1));
+    return kIR + (uint32_t)kb * kRStack + 1024u * (uint32_t)(I * (I + 1));
 }
 constexpr uint32_t kISmem = kIR + 40960;           // 104 KiB
 // Reused inside the R area once the A/P products are read back:
@@ -187,9 +199,9 @@ constexpr uint32_t kITf = kIR + 64 * kLd * 4;      // fp32 T [64][68]
 constexpr uint32_t kIXf = kIR + 128 * kLd * 4;     // fp32 scratch [32][36]
 static_assert(kIXf + 32 * kXLd * 4 <= kIR + 40960, "inverse scratch exceeds the R area");
 // Later uses of the raw tiles within an item:
-//   k tile: K e^{L} (in place) -> T as bf16 operand of the W/U product (first
-//           8 KiB) and the P staging for its bulk store (second 8 KiB);
-//   q tile: Q e^{L} (in place) -> (K e^{G_C - G})^T staging for its bulk store;
+//   k and q: K e^{L}, Q e^{L} (in place), the A operand of the A/P product; then
+//           its first 8 KiB hold T as bf16 operand of the W/U product, the next
+//           8 KiB the P staging for its bulk store;
 //   v, z tiles: [beta K e^G ; beta V]^T, the B operand of the W/U product.
 // Once the W/U product completes no tile is read any more, so the next item's
 // loads are issued then and overlap the W/U readback (which writes W and U to
@@ -311,7 +323,7 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     if (tid == 0) {
         mbar_init(&full, 1);
         mbar_init(&mma_bar, 1);
-        mbar_init(&ap_bar, 4);   // one commit per sub-tile's issuing warp
+        mbar_init(&ap_bar, 1);
         fence_mbar_init();
         sAbort = 0;
     }
@@ -342,8 +354,11 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             const CUtensorMap *maps[4] = {&tm_k, &tm_q, &tm_v, &tm_z};
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
-                tma_rows(sm + m * kRawTile, maps[m], 0, nx.h, nx.t0, &full);
-                tma_rows(sm + m * kRawTile + 8192, maps[m], 64, nx.h, nx.t0, &full);
+                // k, q: K halves 16 KiB apart (interleaved); v, z: 8 KiB apart.
+                const uint32_t base = m < 2 ? 8192u * m : kRawTile * m;
+                const uint32_t kh1 = m < 2 ? 16384u : 8192u;
+                tma_rows(sm + base, maps[m], 0, nx.h, nx.t0, &full);
+                tma_rows(sm + base + kh1, maps[m], 64, nx.h, nx.t0, &full);
             }
         }
         __syncwarp();
@@ -358,12 +373,17 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         int mma_failed = -1, ap_failed = -1;  // parity of a product wait that gave up
         int it = 0;
         for (int w = blockIdx.x; w < total_items && !sAbort; w += gridDim.x, ++it) {
-            if (warp == 0) cp_async_wait_all();  // this item's beta and A values
-            if (!mbar_wait<kIntraSuspendNs>(&full, it & 1, globaltimer_ns() + kWaitNs)) {
-                if (tid == 0) record_timeout(status);
-                sAbort = 1;
+            // Warp 0 alone waits for the item's inputs (its own cp.async of beta and A,
+            // and the TMA boxes); the other warps wait at the barrier, where they take
+            // no issue slots from the SM's other CTA.
+            if (warp == 0) {
+                cp_async_wait_all();
+                if (!mbar_wait<kIntraSuspendNs>(&full, it & 1, globaltimer_ns() + kWaitNs)) {
+                    if (lane == 0) record_timeout(status);
+                    sAbort = 1;
+                }
             }
-            compute_sync();  // beta and A (landed by warp 0's cp.async) are visible
+            compute_sync();  // inputs landed, beta and A visible to every warp
             tc_fence_after_sync();  // the previous item's TMEM reads precede this item's writes
             const IntraItem inf = info;
             const int len = inf.len, h = inf.h;
@@ -420,6 +440,9 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 *(float2 *)&sHalf[b][c0] = acc;
             }
             tmem_st_wait();
+            // The previous item's W/U staging in the R area has been read out before
+            // pass 2 overwrites it.
+            if (tid == 0) bulk_wait_read<0>();
             compute_sync();
             if (sAbort) break;
             // (beta V)^T (rows = channels, K = tokens) into the z tile, dead since pass
@@ -471,7 +494,9 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 const float2 gcm = sub2(GC, mI);
                 const float2 egc = kSoftplus ? gcm : exp2_2(mul2(gcm, log2e2()));
                 uint32_t pk0[4], pk1[4], kd0[4], kd1[4];
-                float lrd[8];  // partial sums of four rows, from pass 1
+                float lrd[16];  // partial sums of the half-block's 8 rows, from pass 1
+                tmem_ld16f(lcol + 16 * q, lrd);
+                tmem_ld_wait();
 #pragma unroll
                 for (int i2 = 0; i2 < 8; i2 += 2) {
                     float2 hk[2], hd[2];
@@ -479,12 +504,8 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                     for (int u = 0; u < 2; ++u) {
                         const int i = i2 + u, r = 8 * b + i;
                         const bool valid = r < len;
-                        const uint32_t so = sw128_offset(r, c0, 64);
-                        if ((i & 3) == 0) {
-                            tmem_ld8(lcol + 16 * q + 8 * (i >> 2), lrd);
-                            tmem_ld_wait();
-                        }
-                        const float2 L = add2(make_float2(lrd[2 * (i & 3)], lrd[2 * (i & 3) + 1]), off);
+                        const uint32_t so = kq_offset(r, c0);
+                        const float2 L = add2(make_float2(lrd[2 * i], lrd[2 * i + 1]), off);
                         const float2 kv = valid ? ld_bf16x2_smem(sm, kRawK + so) : make_float2(0.f, 0.f);
                         const float2 qv = valid ? ld_bf16x2_smem(sm, kRawQ + so) : make_float2(0.f, 0.f);
                         const float2 lg = mul2(L, log2e2());
@@ -532,65 +553,90 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 *(uint4 *)(blk + kOffKd + sw128_offset(c0 + 1, kk, 128)) = make_uint4(kd1[0], kd1[1], kd1[2], kd1[3]);
             }
 
-            // A/P products, per sub-tile I (M = 64 rows s of R^(I), N = 16 + 16):
-            // D[s][32 I + j] = R^(I)_s . Kt_{16 I + j},  D[s][32 I + 16 + j] = R^(I)_s . Qt_{16 I + j}.
+            // A/P product, one M = 128, N = 160 product over both K halves:
+            //   D[r][8 I (I + 1) + s]      = Kt_r . R^(I)_s   (r < 64: A before beta)
+            //   D[64 + r][8 I (I + 1) + s] = Qt_r . R^(I)_s   (P),
+            // of which the readback takes, for row r of sub-tile I, its own image's
+            // columns.  Eight tensor-core instructions for all four sub-tiles.
             fence_proxy_async_smem();
             tc_fence_before_sync();
             compute_sync();
             tc_fence_after_sync();
-            if (warp < 4 && lane == 0) {
-                // Lane 0 of warp Ib issues sub-tile Ib's 16 products (the four warps
-                // sit on different schedulers), then commits them to ap_bar.
-                const int Ib = warp;
-                const uint32_t id = idesc_bf16_f32(64, 16), base = smem_u32(sm);
+            if (warp == 0) {
+                if (elect_one()) {
+                    const uint32_t id = idesc_bf16_f32(128, 160), base = smem_u32(sm);
 #pragma unroll
-                for (int part = 0; part < 2; ++part)
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t a = base + r_region(Ib, ks >> 2) + (ks & 3) * 32;
-                        const uint32_t b = base + (part ? kRawQ : kRawK) + (ks >> 2) * 8192 +
-                                           16 * Ib * 128 + (ks & 3) * 32;
-                        mma_ss(tmem_addr(tb, 0, 32 * Ib + 16 * part), desc_kmajor_sw128(a),
-                               desc_kmajor_sw128(b), id, ks > 0);
-                    }
-                mma_commit(&ap_bar);
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_ss(tmem_addr(tb, 0, 0),
+                               desc_kmajor_sw128(base + (ks >> 2) * 16384 + (ks & 3) * 32),
+                               desc_kmajor_sw128(base + kIR + (ks >> 2) * kRStack + (ks & 3) * 32), id,
+                               ks > 0);
+                    mma_commit(&ap_bar);
+                }
+                __syncwarp();
             }
-            if (!mbar_wait<kIntraSuspendNs>(&ap_bar, it & 1, globaltimer_ns() + kWaitNs)) {
-                if (tid == 0) record_timeout(status);
+            if (warp == 0 && !mbar_wait<kIntraSuspendNs>(&ap_bar, it & 1, globaltimer_ns() + kWaitNs)) {
+                if (lane == 0) record_timeout(status);
                 sAbort = 1;
                 ap_failed = it & 1;
             }
+            compute_sync();  // the A/P products are complete (observed by warp 0)
             tc_fence_after_sync();
             {
-                // M = 64 layout: TMEM lane 32 q + i holds row 16 q + i (i < 16).  Warp w:
-                // lane quarter q = w % 4, sub-tiles 2 (w / 4) and 2 (w / 4) + 1.
-                const int q = warp & 3, hb = warp >> 2;
-                // Half-warp u = lane / 16 takes sub-tile 2 hb + u.
-                const int Ia = 2 * hb + (lane >> 4);
-                uint32_t rr[32];
-                tmem_ld16x2_32(tmem_addr(tb, 32 * q, 64 * hb), rr);
-                tmem_ld_wait();
-                const int sidx = 16 * q + (lane & 15);
-                if (kSoftplus && q == Ia) {
-                    // The diagonal tile, from the pair kernel: [A | P][I][s][r] per item.
-                    const float4 *pa = (const float4 *)(pairs + ((size_t)h * max_chunks + inf.g) * 2048 +
-                                                        Ia * 256 + (lane & 15) * 16);
+                // Warp w: lane quarter qd = w % 4 holds rows r = 32 (qd % 2) + lane of A
+                // (qd < 2) or of P (qd >= 2); half hw = w / 4 takes columns s = 32 hw ..
+                // 32 hw + 31 of those rows, 16 at a time.  The two half-warps' rows lie in
+                // different sub-tiles, whose images start at different D columns, so
+                // each group is loaded at both bases and every lane keeps its own.
+                const int qd = warp & 3, hw = warp >> 2;
+                const int r = 32 * (qd & 1) + lane, Ia = r >> 4;
+                const int I0 = 2 * (qd & 1);
+                const uint32_t nlo = 8u * I0 * (I0 + 1), nhi = 8u * (I0 + 1) * (I0 + 2);
+                const uint32_t lrow = tmem_addr(tb, 32 * qd, 0);
+                const bool isP = qd >= 2;
+                const float br = sBeta[r];
 #pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4) {
-                        const float4 av = pa[v4], pv = pa[256 + v4];
-                        rr[4 * v4] = __float_as_uint(av.x); rr[4 * v4 + 1] = __float_as_uint(av.y);
-                        rr[4 * v4 + 2] = __float_as_uint(av.z); rr[4 * v4 + 3] = __float_as_uint(av.w);
-                        rr[16 + 4 * v4] = __float_as_uint(pv.x); rr[16 + 4 * v4 + 1] = __float_as_uint(pv.y);
-                        rr[16 + 4 * v4 + 2] = __float_as_uint(pv.z); rr[16 + 4 * v4 + 3] = __float_as_uint(pv.w);
+                for (int g = 0; g < 2; ++g) {
+                    const int s0 = 32 * hw + 16 * g;
+                    float va[16], vb[16];
+                    tmem_ld16f(lrow + nlo + s0, va);
+                    tmem_ld16f(lrow + nhi + s0, vb);
+                    tmem_ld_wait();
+                    float v[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] = lane < 16 ? va[e] : vb[e];
+                    if (kSoftplus && 2 * hw + g == Ia) {
+                        // The diagonal tile, from the pair kernel: [A | P][I][r][s] per item.
+                        const float4 *pa = (const float4 *)(pairs + ((size_t)h * max_chunks + inf.g) * 2048 +
+                                                            (isP ? 1024 : 0) + Ia * 256 + (r & 15) * 16);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4) {
+                            const float4 x = pa[v4];
+                            v[4 * v4] = x.x; v[4 * v4 + 1] = x.y; v[4 * v4 + 2] = x.z; v[4 * v4 + 3] = x.w;
+                        }
                     }
-                }
+                    if (!isP) {
+                        // A = strictly_lower(Diag(beta) Kt Kh^T), fp32 rows for the inverse.
 #pragma unroll
-                for (int jr = 0; jr < 16; ++jr) {
-                    const int r = 16 * Ia + jr;
-                    Af[r * kLd + sidx] = sidx < r ? sBeta[r] * __uint_as_float(rr[jr]) : 0.f;
-                    const float pvv = sidx <= r ? __uint_as_float(rr[16 + jr]) : 0.f;
-                    *(__nv_bfloat16 *)(sm + kRawK + 8192 + sw128_offset(r, sidx, 64)) =
-                        __float2bfloat16_rn(pvv);
+                        for (int e = 0; e < 16; e += 4)
+                            *(float4 *)&Af[r * kLd + s0 + e] =
+                                make_float4(s0 + e < r ? br * v[e] : 0.f, s0 + e + 1 < r ? br * v[e + 1] : 0.f,
+                                            s0 + e + 2 < r ? br * v[e + 2] : 0.f,
+                                            s0 + e + 3 < r ? br * v[e + 3] : 0.f);
+                    } else {
+                        // P = lower(Qt Kh^T), bf16 operand image rows (the staging of its store).
+#pragma unroll
+                        for (int e = 0; e < 16; e += 8) {
+                            uint32_t w4[4];
+#pragma unroll
+                            for (int k2 = 0; k2 < 4; ++k2) {
+                                const int sa = s0 + e + 2 * k2;
+                                w4[k2] = pack_bf16(sa <= r ? v[e + 2 * k2] : 0.f, sa + 1 <= r ? v[e + 2 * k2 + 1] : 0.f);
+                            }
+                            *(uint4 *)(sm + kRawK + 8192 + sw128_offset(r, s0 + e, 64)) =
+                                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        }
+                    }
                 }
             }
             fence_proxy_async_smem();
@@ -702,12 +748,13 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                            desc_kmajor_sw128(smem_u32(sm + kRawV) + ks * 32), id, ks > 0);
                 mma_commit(&mma_bar);
             }
-            if (!mbar_wait<kIntraSuspendNs>(&mma_bar, mma_count & 1, globaltimer_ns() + kWaitNs)) {
-                if (tid == 0) record_timeout(status);
+            if (warp == 0 && !mbar_wait<kIntraSuspendNs>(&mma_bar, mma_count & 1, globaltimer_ns() + kWaitNs)) {
+                if (lane == 0) record_timeout(status);
                 sAbort = 1;
                 mma_failed = (int)(mma_count & 1);
             }
             ++mma_count;
+            compute_sync();  // the W/U product is complete (observed by warp 0)
             tc_fence_after_sync();
             // No raw tile is read any more: the next item's loads overlap the readback.
             if (warp == 0 && has_next && !sAbort) {
@@ -720,9 +767,11 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             }
             {
                 // Rows r = 16 q + i (i < 16) of lane quarter q = w % 4; warps 0-3 read W
-                // (columns 0..127) into rows 0..63 of the block's [W; Qt] image, warps
-                // 4-7 read U (columns 128..255) into its row-major block region.  Each
-                // load covers 64 columns: 32 for each half-warp.
+                // (columns 0..127), warps 4-7 read U (columns 128..255).  Each load covers
+                // 64 columns: 32 for each half-warp.  Both are staged in the R area (free
+                // since the inverse) in their block layouts -- W as rows 0..63 of the two
+                // K halves of the [W; Qt] image, U with its row swizzle -- and leave by
+                // three bulk copies.
                 const int q = warp & 3, hb = warp >> 2, r = 16 * q + (lane & 15);
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
@@ -738,14 +787,21 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                             pack_bf16(__uint_as_float(rr[cc + 6]), __uint_as_float(rr[cc + 7])));
                         const int col = 64 * j + 32 * (lane >> 4) + cc;
                         if (hb == 0)
-                            *(uint4 *)(blk + kOffWQ + sw128_offset(r, col, 128)) = w4;
+                            *(uint4 *)(sm + kIR + sw128_offset(r, col, 64)) = w4;
                         else
-                            *(uint4 *)(blk + kOffU + (r * 128 + col) * 2) = w4;
+                            *(uint4 *)(sm + kIR + 16384 + u_offset(r, col)) = w4;
                     }
                 }
             }
+            fence_proxy_async_smem();
             tc_fence_before_sync();
-            compute_sync();  // TMEM is read out before the next item's products
+            compute_sync();  // TMEM is read out before the next item's products; staging written
+            if (tid == 0) {
+                bulk_s2g(blk + kOffWQ, sm + kIR, 8192);
+                bulk_s2g(blk + kOffWQ + 16384, sm + kIR + 8192, 8192);
+                bulk_s2g(blk + kOffU, sm + kIR + 16384, 16384);
+                bulk_commit();
+            }
             if (sAbort) break;
         }
         if (tid == 0) bulk_wait<0>();  // every staged block region has reached memory
@@ -769,12 +825,13 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
 // Training, and Million-Token Agentic RL", section 3.3: before the bound,
 // diagonal tiles needed a position-pair path).  For the 16-token sub-tile I of
 // a (chunk, head) item and rows s <= r in it:
-//   A[I][s][r] = sum_c k_rc k_sc e^{L_rc - L_sc},   P[I][s][r] = sum_c q_rc k_sc e^{L_rc - L_sc},
+//   A[I][r][s] = sum_c k_rc k_sc e^{L_rc - L_sc},   P[I][r][s] = sum_c q_rc k_sc e^{L_rc - L_sc},
 // L the cumulative log-decay from the sub-tile start, one exponent per pair and
 // channel, so no factor overflows however fast the state decays (beta and the
 // causal masks are applied by the intra kernel, which reads these tiles in place
 // of its products' diagonal tiles).  One CTA per item; rows beyond the chunk's
-// length give zeros.  Output per item: 2 x 4 x 16 x 16 fp32.
+// length give zeros.  Output per item: [A | P][I][r][s], 2 x 4 x 16 x 16 fp32
+// (only s <= r is written; the intra kernel masks the rest).
 constexpr int kPairThreads = 256;
 constexpr int kPairLd = 130;   // fp32 row stride of the staged L, k, q rows
 constexpr uint32_t kPairSmem = 3u * kChunk * kPairLd * 4u;
@@ -832,43 +889,55 @@ diag_pair_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__res
             a = fma2(*(const float2 *)&kr[c], kse, a);
             pp = fma2(*(const float2 *)&qr[c], kse, pp);
         }
-        out[I * 256 + s * 16 + r] = a.x + a.y;
-        out[1024 + I * 256 + s * 16 + r] = pp.x + pp.y;
+        out[I * 256 + r * 16 + s] = a.x + a.y;
+        out[1024 + I * 256 + r * 16 + s] = pp.x + pp.y;
     }
 }
 
 // ------------------------------------------------------------------ state --
 
-// One CTA of 384 threads per (sequence, head) slot, in three roles:
-//   chain  (warps 0-7): the per-chunk state recurrence.  Thread (j, hh) owns
-//          TMEM lane j = value channel j and half hh of the delta rows, state
-//          columns and the chunk's key channels.  Thread 0 also issues the
-//          block loads and every tensor-core product, between group barriers,
-//          so that no hand-off to another warp sits on the chain.
+// One CTA of 416 threads per (sequence, head) slot, in three roles:
+//   chain  (warps 0-7): the per-chunk state recurrence on CUDA cores.  Thread
+//          (j, hh) owns TMEM lane j = value channel j and half hh of the delta
+//          rows, state columns and the chunk's key channels.
 //   output (warps 8-11): reads O^T of each finished chunk from TMEM, rounds it
 //          to bf16 in a staging tile and stores whole token rows (one TMA
-//          tensor store per full chunk), off the chain.
-// Per chunk c (buffer b = c & 1 of the [delta | O] accumulator D1):
-//   D1[:, 0:64]   = S^T W^T         (commit -> mma1: the chain may form delta)
-//   D1[:, 64:128] = S^T Qt^T
-//   Dl^T = U^T - D1[:, 0:64]        -> bf16 into TMEM            (chain)
-//   S^T += Dl^T Kd,  D1[:, 64:] += Dl^T P^T   (commit -> mma2[b])
-//   S^T  -> bf16 copy (the next chunk's A operand), then the fp32 master times
-//           the next chunk's e^{G_C}                              (chain)
-//   O^T = D1[:, 64:] -> o                                         (output)
-constexpr int kStateThreads = 384;
+//          tensor store per full chunk).
+//   issue  (warp 12): every tensor-core product and block load, so that no
+//          chain thread spends its time issuing; the hand-offs are mbarriers.
+// Per chunk c, the products the state recurrence waits for are issued first,
+// and those only the outputs need are queued behind them on the tensor pipe,
+// where they run while the chain works on CUDA cores:
+//   DW     = S_in^T W^T             (critical; commit -> mma1)
+//   DO[b]  = S_in^T Qt^T            (outputs; b = c & 1)
+//   Dl^T   = U^T - DW               -> bf16 into TMEM                (chain)
+//   S^T   += Dl^T Kd                (critical; commit -> mma2s)
+//   DO[b] += Dl^T P^T               (outputs; commit -> mma2o[b], empty[stage])
+//   S^T    -> bf16 copy SB[(c + 1) & 1] (the next chunk's A operand),
+//             then the fp32 master times the next chunk's e^{G_C}    (chain)
+//   O^T    = DO[b] -> o                                               (output)
+// The bf16 copy of S is double-buffered so that the output product of chunk c
+// still reads S_in(c) while the chain writes S_in(c + 1).
+constexpr int kStateThreads = 416;
 constexpr int kChainThreads = 256, kOutThreads = 128;
+constexpr int kIssueWarp = 12;
 constexpr uint32_t kStageBytes = 75776;  // block rounded up to 1 KiB
 constexpr int kStages = 2;
 constexpr uint32_t kOStage = kStages * kStageBytes;  // 2 x [64][128] bf16 output staging
 constexpr uint32_t kStateSmem = kStages * kStageBytes + 2 * 16384 + 1024;
-// TMEM columns
-constexpr uint32_t kTS = 0, kTSbf = 128, kTDl = 192, kTD1 = 256;  // D1 double buffer: 256, 384
-constexpr int kBarChain = 1, kBarOut = 2;                         // named barrier ids
+// TMEM columns: fp32 S^T, two bf16 copies of S^T, delta^T (bf16), the W
+// product, two output accumulators.
+constexpr uint32_t kTS = 0, kTSbf = 128, kTDl = 256, kTDW = 288, kTDO = 352;  // SB[b] = 128 + 64 b,
+                                                                               // DO[b] = 352 + 64 b
+constexpr int kBarOut = 2;  // named barrier id of the output warps
+// L2 prefetch distance of the block stream, in chunks: 96 chains x 6 blocks of
+// 72.5 KiB is about 42 MB of the 126 MB L2.
+constexpr int kPrefetchAhead = 6;
 
 struct StateBars {
-    uint64_t full[kStages];
-    uint64_t mma1, mma2[2], d1_free[2], drain;
+    uint64_t full[kStages], empty[kStages];
+    uint64_t mma1, mma2s, mma2o[2], do_free[2];
+    uint64_t sbf_ready, dl_ready, dec_ready, drain;
 };
 
 // Barrier over `nthreads` threads of the CTA (named barrier `id`) that also
@@ -960,12 +1029,16 @@ state_kernel(const __grid_constant__ CUtensorMap tm_o,
     const size_t fbase = Gn == 1 ? sbase : 0;  // Sf offset of this (sequence, head)
     uint8_t *eimg = xmode ? Eimg + ((size_t)h * max_chunks + chunk_off[n] + cbeg) * kEImg : nullptr;
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&bars.full[s], 1);
+        for (int s = 0; s < kStages; ++s) { mbar_init(&bars.full[s], 1); mbar_init(&bars.empty[s], 1); }
         mbar_init(&bars.mma1, 1);
+        mbar_init(&bars.mma2s, 1);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&bars.mma2[b], 1);
-            mbar_init(&bars.d1_free[b], kOutThreads);
+            mbar_init(&bars.mma2o[b], 1);
+            mbar_init(&bars.do_free[b], kOutThreads);
         }
+        mbar_init(&bars.sbf_ready, kChainThreads);
+        mbar_init(&bars.dl_ready, kChainThreads);
+        mbar_init(&bars.dec_ready, kChainThreads);
         mbar_init(&bars.drain, 1);
         fence_mbar_init();
     }
@@ -977,58 +1050,126 @@ state_kernel(const __grid_constant__ CUtensorMap tm_o,
     const uint8_t *blk0 = blocks + ((size_t)h * max_chunks + chunk_off[n] + cbeg) * kBlockBytes;
     const uint32_t lq = 32 * (warp & 3);
 
-    if (warp < 8) {
+    if (warp == kIssueWarp) {
+        // ------------------------------------------------------ issue --
+        // The whole warp runs the loop (waits are warp-uniform); one elected
+        // lane issues each copy, product and commit.
+        const bool leader = elect_one();
+        const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
+        int loads = 0;
+        auto load = [&](int c) {
+            const int s = c % kStages;
+            if (leader) {
+                mbar_arrive_expect_tx(&bars.full[s], kBlockBytes);
+                bulk_g2s(sm + s * kStageBytes, blk0 + (size_t)c * kBlockBytes, kBlockBytes, &bars.full[s]);
+                if (c + kPrefetchAhead < nch)
+                    bulk_prefetch_l2(blk0 + (size_t)(c + kPrefetchAhead) * kBlockBytes, kBlockBytes);
+            }
+            ++loads;
+            __syncwarp();
+        };
+        if (leader)
+            for (int c = kStages; c < nch && c < kPrefetchAhead; ++c)
+                bulk_prefetch_l2(blk0 + (size_t)c * kBlockBytes, kBlockBytes);
+        for (int c = 0; c < nch && c < kStages; ++c) load(c);
+        // The leader waits; the result is broadcast, so the warp stays converged
+        // and leaves the loop as one when a wait gives up.
+        auto wait = [&](uint64_t *bar, uint32_t parity) {
+            int r = 1;
+            if (leader) {
+                r = mbar_wait(bar, parity, globaltimer_ns() + kWaitNs) ? 1 : 0;
+                if (!r) record_timeout(status);
+            }
+            return __shfl_sync(0xffffffffu, r, leader_lane) != 0;
+        };
+        const uint32_t id64 = idesc_bf16_f32(128, 64), id128 = idesc_bf16_f32(128, 128);
+        bool ok = true;
+        for (int c = 0; c < nch && ok; ++c) {
+            const int s = c % kStages, b = c & 1;
+            const uint32_t st = smem_u32(sm + s * kStageBytes);
+            const uint32_t sb = tmem_addr(tb, 0, kTSbf + 64 * b);
+            const uint32_t dO = tmem_addr(tb, 0, kTDO + 64 * b);
+            // Descriptors of this stage's operands (warp-uniform, before any issue).
+            uint64_t dW[8], dQ[8], dK[4], dP[4];
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                dW[ks] = desc_kmajor_sw128(st + kOffWQ + (ks >> 2) * 16384 + (ks & 3) * 32);
+                dQ[ks] = desc_kmajor_sw128(st + kOffWQ + (ks >> 2) * 16384 + 8192 + (ks & 3) * 32);
+            }
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                dK[ks] = desc_kmajor_sw128(st + kOffKd + ks * 32);
+                dP[ks] = desc_kmajor_sw128(st + kOffP + ks * 32);
+            }
+            // DW = S_in^T W^T: needs the block and S_in(c) in bf16.
+            ok = wait(&bars.full[s], (c / kStages) & 1) && wait(&bars.sbf_ready, c & 1);
+            if (!ok) break;
+            tc_fence_after_sync();
+            if (leader) {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_ts(tmem_addr(tb, 0, kTDW), sb + 8 * ks, dW[ks], id64, ks > 0);
+                mma_commit(&bars.mma1);
+            }
+            __syncwarp();
+            // DO[b] = S_in^T Qt^T once output c - 2 has read DO[b].
+            ok = c < 2 || wait(&bars.do_free[b], ((c >> 1) - 1) & 1);
+            if (!ok) break;
+            tc_fence_after_sync();
+            if (leader) {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) mma_ts(dO, sb + 8 * ks, dQ[ks], id64, ks > 0);
+            }
+            __syncwarp();
+            // S^T += Dl^T Kd, then DO[b] += Dl^T P^T: need delta(c) and the decayed master.
+            ok = wait(&bars.dl_ready, c & 1) && wait(&bars.dec_ready, c & 1);
+            if (!ok) break;
+            tc_fence_after_sync();
+            if (leader) {
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_ts(tmem_addr(tb, 0, kTS), tmem_addr(tb, 0, kTDl + 8 * ks), dK[ks], id128, true);
+                mma_commit(&bars.mma2s);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_ts(dO, tmem_addr(tb, 0, kTDl + 8 * ks), dP[ks], id64, true);
+                mma_commit(&bars.mma2o[b]);
+                mma_commit(&bars.empty[s]);
+            }
+            __syncwarp();
+            // Stage s is consumed once these products finish: refill it.
+            if (c + kStages < nch) {
+                ok = wait(&bars.empty[s], (c / kStages) & 1);
+                if (!ok) break;
+                load(c + kStages);
+            }
+        }
+        if (leader) {
+            // Drain: every issued copy has landed and every product has finished
+            // before the CTA may exit (bounded waits).
+            for (int d = max(0, loads - kStages); d < loads; ++d)
+                mbar_wait(&bars.full[d % kStages], (d / kStages) & 1, globaltimer_ns() + kWaitNs);
+            mma_commit(&bars.drain);
+            mbar_wait(&bars.drain, 0, globaltimer_ns() + kWaitNs);
+        }
+        __syncwarp();
+    } else if (warp < 8) {
         // ------------------------------------------------------- chain --
         const int j = tid & 127, hh = warp >> 2;
         uint32_t ra[32], rb[32];
-        bool bad = false;            // this thread saw a bounded wait give up
-        int loads = 0;               // block loads issued (thread 0)
-        bool issued_mma = false;     // thread 0 issued a product
-        auto load = [&](int c) {     // thread 0: block of chunk c into stage c % kStages
-            const int s = c % kStages;
-            mbar_arrive_expect_tx(&bars.full[s], kBlockBytes);
-            bulk_g2s(sm + s * kStageBytes, blk0 + (size_t)c * kBlockBytes, kBlockBytes, &bars.full[s]);
-            ++loads;
-        };
+        // Every lane waits (each reads what the wait guards); the warp decides as
+        // one whether to go on, so the warp-collective TMEM accesses stay converged.
         auto wait = [&](uint64_t *bar, uint32_t parity) {
-            if (!mbar_wait(bar, parity, globaltimer_ns() + kWaitNs)) {
-                record_timeout(status);
-                bad = true;
-                return false;
-            }
-            return true;
+            const bool r = mbar_wait(bar, parity, globaltimer_ns() + kWaitNs);
+            if (!r) record_timeout(status);
+            return __all_sync(0xffffffffu, r);
         };
-        // Thread 0: D1 = S^T [W; Qt]^T for chunk c, in two halves so that the
-        // delta half commits first.  Needs the block and a free D1 buffer.
-        auto issue_mma1 = [&](int c) {
-            const int s = c % kStages, b = c & 1;
-            if (!wait(&bars.full[s], (c / kStages) & 1)) return;
-            if (c >= 2 && !wait(&bars.d1_free[b], ((c >> 1) - 1) & 1)) return;
-            tc_fence_after_sync();
-            const uint32_t st = smem_u32(sm + s * kStageBytes);
-            const uint32_t d1 = tmem_addr(tb, 0, kTD1 + 128 * b);
-            const uint32_t id64 = idesc_bf16_f32(128, 64);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_ts(d1 + 64 * half, tmem_addr(tb, 0, kTSbf + 8 * ks),
-                           desc_kmajor_sw128(st + kOffWQ + (ks >> 2) * 128 * 128 + half * 8192 +
-                                             (ks & 3) * 32),
-                           id64, ks > 0);
-                if (half == 0) mma_commit(&bars.mma1);
-            }
-            issued_mma = true;
-        };
-        if (tid == 0)
-            for (int c = 0; c < nch && c < kStages; ++c) load(c);
-
         // Initial state: S^T row j = column j of S0 (this half's 64 key channels):
-        // fp32 master pre-multiplied by the first chunk's decay, and the bf16 copy.
-        // The transition X starts from the identity: X^T row j = e_j.
+        // fp32 master pre-multiplied by the first chunk's decay, and the bf16 copy
+        // SB[0].  The transition X starts from the identity: X^T row j = e_j.
         const bool nonzero0 = S0 || xmode;
         const float *dec0 = (const float *)(sm + kOffDecay);
-        if (nonzero0) wait(&bars.full[0], 0);
+        bool ok = !nonzero0 || wait(&bars.full[0], 0);
         __syncwarp();
         for (int q2 = 0; q2 < 2; ++q2) {
             const int c0 = 64 * hh + 32 * q2;
@@ -1039,29 +1180,28 @@ state_kernel(const __grid_constant__ CUtensorMap tm_o,
 #pragma unroll
             for (int i = 0; i < 32; ++i) ra[i] = __float_as_uint(nonzero0 ? sv[i] * dec0[c0 + i] : 0.f);
             tmem_st32(tmem_addr(tb, lq, kTS + c0), ra);
-            uint32_t sb[16];
+            uint32_t sbb[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) sb[i] = pack_bf16(sv[2 * i], sv[2 * i + 1]);
-            tmem_st16(tmem_addr(tb, lq, kTSbf + c0 / 2), sb);
+            for (int i = 0; i < 16; ++i) sbb[i] = pack_bf16(sv[2 * i], sv[2 * i + 1]);
+            tmem_st16(tmem_addr(tb, lq, kTSbf + c0 / 2), sbb);
         }
         tmem_st_wait();
         tc_fence_before_sync();
-        bool failed = group_sync_any(kBarChain, kChainThreads, bad);
-        if (!failed && tid == 0) issue_mma1(0);
+        mbar_arrive(&bars.sbf_ready);
+        mbar_arrive(&bars.dec_ready);
 
-        int c = 0;
-        for (; c < nch && !failed; ++c) {
-            const int s = c % kStages, b = c & 1;
+        for (int c = 0; c < nch && ok; ++c) {
+            const int s = c % kStages;
             const uint8_t *st = sm + s * kStageBytes;
-            wait(&bars.full[s], (c / kStages) & 1);   // U of this block (already landed)
-            wait(&bars.mma1, c & 1);
+            ok = wait(&bars.full[s], (c / kStages) & 1) && wait(&bars.mma1, c & 1);
+            if (!ok) break;
             __syncwarp();
             tc_fence_after_sync();
-            // Dl^T[j][r] = U[r][j] - D1[j][r] for this half's 32 rows -> bf16 pairs into
+            // Dl^T[j][r] = U[r][j] - DW[j][r] for this half's 32 rows -> bf16 pairs into
             // TMEM (U = 0 on the transition).
             {
-                const __nv_bfloat16 *U = (const __nv_bfloat16 *)(st + kOffU);
-                tmem_ld32(tmem_addr(tb, lq, kTD1 + 128 * b + 32 * hh), ra);
+                const uint8_t *Ub = st + kOffU;
+                tmem_ld32(tmem_addr(tb, lq, kTDW + 32 * hh), ra);
                 tmem_ld_wait();
                 uint32_t dl[16];
                 if (xmode) {
@@ -1072,8 +1212,10 @@ state_kernel(const __grid_constant__ CUtensorMap tm_o,
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
                         const int r = 32 * hh + i;
-                        const float d0 = __bfloat162float(U[r * kDV + j]) - __uint_as_float(ra[i]);
-                        const float d1v = __bfloat162float(U[(r + 1) * kDV + j]) - __uint_as_float(ra[i + 1]);
+                        const float d0 = __bfloat162float(*(const __nv_bfloat16 *)(Ub + u_offset(r, j))) -
+                                         __uint_as_float(ra[i]);
+                        const float d1v = __bfloat162float(*(const __nv_bfloat16 *)(Ub + u_offset(r + 1, j))) -
+                                          __uint_as_float(ra[i + 1]);
                         dl[i >> 1] = pack_bf16(d0, d1v);
                     }
                 }
@@ -1092,33 +1234,31 @@ state_kernel(const __grid_constant__ CUtensorMap tm_o,
                 tmem_st_wait();
             }
             tc_fence_before_sync();
-            if ((failed = group_sync_any(kBarChain, kChainThreads, bad))) break;
-            if (tid == 0) {
-                // S^T += Dl^T Kd (N = dk, K = 64 tokens); O^T += Dl^T P^T (N = 64, K = 64)
-                tc_fence_after_sync();
-                const uint32_t id128 = idesc_bf16_f32(128, 128), id64 = idesc_bf16_f32(128, 64);
-                const uint32_t sa = smem_u32(st);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_ts(tmem_addr(tb, 0, kTS), tmem_addr(tb, 0, kTDl + 8 * ks),
-                           desc_kmajor_sw128(sa + kOffKd + ks * 32), id128, true);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_ts(tmem_addr(tb, 0, kTD1 + 128 * b + 64), tmem_addr(tb, 0, kTDl + 8 * ks),
-                           desc_kmajor_sw128(sa + kOffP + ks * 32), id64, true);
-                mma_commit(&bars.mma2[b]);
-                issued_mma = true;
-            }
-            const bool done2 = wait(&bars.mma2[b], (c >> 1) & 1);
+            mbar_arrive(&bars.dl_ready);
+            ok = wait(&bars.mma2s, c & 1);
+            if (!ok) break;
             __syncwarp();
             tc_fence_after_sync();
-            // Stage s is consumed (products done, U read before the barrier): refill it.
-            if (tid == 0 && done2 && c + kStages < nch) load(c + kStages);
             const bool last = (c + 1 == nch);
             // S_out, this half's 64 key channels: two loads, one wait.
             tmem_ld32(tmem_addr(tb, lq, kTS + 64 * hh), ra);
             tmem_ld32(tmem_addr(tb, lq, kTS + 64 * hh + 32), rb);
             tmem_ld_wait();
+            if (!last) {
+                // Critical: the bf16 copy that the next chunk's first product reads.
+                uint32_t sa[16], sbv[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    sa[i] = pack_bf16(__uint_as_float(ra[2 * i]), __uint_as_float(ra[2 * i + 1]));
+                    sbv[i] = pack_bf16(__uint_as_float(rb[2 * i]), __uint_as_float(rb[2 * i + 1]));
+                }
+                const uint32_t sbn = kTSbf + 64 * ((c + 1) & 1) + 32 * hh;
+                tmem_st16(tmem_addr(tb, lq, sbn), sa);
+                tmem_st16(tmem_addr(tb, lq, sbn + 16), sbv);
+                tmem_st_wait();
+                tc_fence_before_sync();
+                mbar_arrive(&bars.sbf_ready);
+            }
             // Checkpoint when the state after `pos` tokens falls on a multiple of every.
             const int pos = min((c + 1) * kChunk, tend - tbeg);
             if (ckpt_every > 0 && pos % ckpt_every == 0) {
@@ -1139,25 +1279,11 @@ state_kernel(const __grid_constant__ CUtensorMap tm_o,
                 }
                 break;
             }
-            // Critical: the bf16 copy that the next chunk's first product reads.
-            {
-                uint32_t sa[16], sbv[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    sa[i] = pack_bf16(__uint_as_float(ra[2 * i]), __uint_as_float(ra[2 * i + 1]));
-                    sbv[i] = pack_bf16(__uint_as_float(rb[2 * i]), __uint_as_float(rb[2 * i + 1]));
-                }
-                tmem_st16(tmem_addr(tb, lq, kTSbf + 32 * hh), sa);
-                tmem_st16(tmem_addr(tb, lq, kTSbf + 32 * hh + 16), sbv);
-                tmem_st_wait();
-            }
-            tc_fence_before_sync();
-            if ((failed = group_sync_any(kBarChain, kChainThreads, bad))) break;
-            if (tid == 0) issue_mma1(c + 1);
-            // Off the critical path: the fp32 master times the next chunk's decay
-            // (done before the next barrier, which precedes the product that adds to it).
+            // Off the critical path: the fp32 master times the next chunk's decay,
+            // before the product that adds to it (dec_ready).
             const int s1 = (c + 1) % kStages;
-            wait(&bars.full[s1], ((c + 1) / kStages) & 1);
+            ok = wait(&bars.full[s1], ((c + 1) / kStages) & 1);
+            if (!ok) break;
             __syncwarp();
             const float *dec = (const float *)(sm + s1 * kStageBytes + kOffDecay) + 64 * hh;
 #pragma unroll
@@ -1169,42 +1295,31 @@ state_kernel(const __grid_constant__ CUtensorMap tm_o,
             tmem_st32(tmem_addr(tb, lq, kTS + 64 * hh + 32), rb);
             tmem_st_wait();
             tc_fence_before_sync();
-        }
-        if (tid == 0) {
-            // Drain: every issued copy has landed and every committed product has
-            // finished before the CTA may exit (bounded waits; a timeout is recorded).
-            for (int d = max(0, loads - kStages); d < loads; ++d)
-                mbar_wait(&bars.full[d % kStages], (d / kStages) & 1, globaltimer_ns() + kWaitNs);
-            if (issued_mma) {
-                // One more commit tracks every product this thread issued.
-                mma_commit(&bars.drain);
-                mbar_wait(&bars.drain, 0, globaltimer_ns() + kWaitNs);
-            }
+            mbar_arrive(&bars.dec_ready);
         }
     } else {
         // ------------------------------------------------------ output --
         const int j = tid - kChainThreads;        // TMEM lane = value channel
         const int Ttot = cu[N];                   // rows past it are clipped by the TMA store
-        bool failed = false;
         for (int c = 0; c < nch; ++c) {
             const int b = c & 1;
             const int t0 = tbeg + c * kChunk, len = min(kChunk, tend - t0);
-            const bool ok = mbar_wait(&bars.mma2[b], (c >> 1) & 1, globaltimer_ns() + kWaitNs);
+            const bool ok = mbar_wait(&bars.mma2o[b], (c >> 1) & 1, globaltimer_ns() + kWaitNs);
             if (!ok) record_timeout(status);
             __syncwarp();
             tc_fence_after_sync();
             uint32_t oa[32], ob[32];
-            tmem_ld32(tmem_addr(tb, lq, kTD1 + 128 * b + 64), oa);
-            tmem_ld32(tmem_addr(tb, lq, kTD1 + 128 * b + 96), ob);
+            tmem_ld32(tmem_addr(tb, lq, kTDO + 64 * b), oa);
+            tmem_ld32(tmem_addr(tb, lq, kTDO + 64 * b + 32), ob);
             tmem_ld_wait();
             tc_fence_before_sync();
-            mbar_arrive(&bars.d1_free[b]);
+            mbar_arrive(&bars.do_free[b]);
             // Staging buffer c & 1 is free once the stores issued from it (two
             // chunks ago) have read it; waiting for every earlier store is simpler
             // and costs nothing here.
             if (j == 0) bulk_wait_read<0>();
             __syncwarp();
-            if ((failed = group_sync_any(kBarOut, kOutThreads, !ok))) break;
+            if (group_sync_any(kBarOut, kOutThreads, !ok)) break;
             uint8_t *ost = sm + kOStage + (c & 1) * 16384;
             if (eimg) {
                 // E rows as the K-major, 128-byte-swizzled A operand of the
@@ -1240,7 +1355,6 @@ state_kernel(const __grid_constant__ CUtensorMap tm_o,
                 }
             }
         }
-        (void)failed;
         if (j == 0) bulk_wait<0>();   // every store has completed before the CTA exits
     }
     tc_fence_before_sync();
@@ -1490,7 +1604,7 @@ debug_unpack_kernel(const uint8_t *__restrict__ blocks, int64_t max_chunks,
         if (Wout)
             Wout[idx] = __bfloat162float(*(const __nv_bfloat16 *)(blk + kOffWQ + sw128_offset(r, c, 128)));
         if (Uout)
-            Uout[idx] = __bfloat162float(((const __nv_bfloat16 *)(blk + kOffU))[r * kDV + c]);
+            Uout[idx] = __bfloat162float(*(const __nv_bfloat16 *)(blk + kOffU + u_offset(r, c)));
     }
 }
 

@@ -21,6 +21,14 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// One lane of a converged warp (the same lane on every call).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile("{\n .reg .pred P;\n elect.sync _|P, 0xffffffff;\n selp.u32 %0, 1, 0, P;\n}\n"
+                 : "=r"(pred));
+    return pred != 0;
+}
+
 // ---------------------------------------------------------------- mbarrier --
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
@@ -261,6 +269,18 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&r)[8]) {
                    "=f"(r[6]), "=f"(r[7])
                  : "r"(taddr)
                  : "memory");
+}
+
+// 32 lanes x 32 bits, 16 consecutive columns, fp32 values.
+__device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=f"(r[0]), "=f"(r[1]), "=f"(r[2]), "=f"(r[3]), "=f"(r[4]), "=f"(r[5]), "=f"(r[6]),
+          "=f"(r[7]), "=f"(r[8]), "=f"(r[9]), "=f"(r[10]), "=f"(r[11]), "=f"(r[12]), "=f"(r[13]),
+          "=f"(r[14]), "=f"(r[15])
+        : "r"(taddr)
+        : "memory");
 }
 
 __device__ __forceinline__ void tmem_st_wait() {
