@@ -61,15 +61,17 @@ constexpr uint64_t kWaitNs = 2000000000ull;  // per-wait limit: 2 s
 constexpr uint32_t kOffWQ = 0;         // [W; Qt] 128 rows x 128 K, swizzled K-major
 constexpr uint32_t kOffKd = 32768;     // Kd^T 128 rows (key channel) x 64 K (token)
 constexpr uint32_t kOffP = 49152;      // P 64 rows x 64 K
-constexpr uint32_t kOffU = 57344;      // U [64][128] bf16, 16-byte chunks swizzled per row
-// Byte offset of U[r][j] in its region: row r holds 16 chunks of 8 channels, chunk
-// index XORed with r % 16, so that 16 consecutive rows' stores of one chunk and
-// one row's loads of 32 consecutive channels both spread over the banks.
-__host__ __device__ __forceinline__ uint32_t u_offset(uint32_t r, uint32_t j) {
-    return r * 256u + ((((j >> 3) ^ r) & 15u) << 4) + ((j & 7u) << 1);
-}
+constexpr uint32_t kOffU = 57344;      // U row-major [64][128] bf16
 constexpr uint32_t kOffDecay = 73728;  // e^{G_C} [128] fp32
 constexpr uint32_t kBlockBytes = 74240;
+
+// The dynamic shared memory rounded up to a 1024-byte boundary (the 128-byte
+// swizzle's period).  The offset is added to the __shared__ pointer itself, not
+// through an integer round trip, so the compiler still knows every access made
+// through the result is a shared-memory access (32-bit addressing, LDS/STS).
+__device__ __forceinline__ uint8_t *align_smem_1024(uint8_t *smraw) {
+    return smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
+}
 
 __device__ __forceinline__ void record_timeout(int32_t *status) {
     atomicCAS(status, 0, (int32_t)KDA_TC_TIMEOUT_CODE);
@@ -221,6 +223,13 @@ __device__ __forceinline__ void tma_rows(void *smem_dst, const CUtensorMap *map,
         : "memory");
 }
 
+// Prefetch of the same box into L2 (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_rows(const CUtensorMap *map, int x, int h, int t0) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(h), "r"(t0)
+                 : "memory");
+}
+
 __device__ __forceinline__ void compute_sync() { __syncthreads(); }
 
 __device__ __forceinline__ void cp_async_4(void *smem_dst, const void *gmem_src) {
@@ -307,7 +316,7 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
 {
     constexpr bool kSoftplus = GATE == kGateSoftplus;
     extern __shared__ uint8_t smraw[];
-    uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sm = align_smem_1024(smraw);
     __shared__ uint64_t full, mma_bar, ap_bar;
     __shared__ uint32_t tbase;
     __shared__ IntraItem info;
@@ -440,11 +449,21 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 *(float2 *)&sHalf[b][c0] = acc;
             }
             tmem_st_wait();
-            // The previous item's W/U staging in the R area has been read out before
-            // pass 2 overwrites it.
-            if (tid == 0) bulk_wait_read<0>();
             compute_sync();
             if (sAbort) break;
+            if (tid == 0 && has_next) {
+                // The next item's rows into L2 now, so that its tile loads (issued once
+                // this item's W/U product is done) come from L2.
+                cp_async_wait_all();
+                const int2 loc = next_loc;
+                const int hn = (w + (int)gridDim.x) % H;
+                const CUtensorMap *maps[4] = {&tm_k, &tm_q, &tm_v, &tm_z};
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    tma_prefetch_rows(maps[m], 0, hn, loc.x);
+                    tma_prefetch_rows(maps[m], 64, hn, loc.x);
+                }
+            }
             // (beta V)^T (rows = channels, K = tokens) into the z tile, dead since pass
             // 1: rows 128..255 of the B operand of the W/U product.
 #pragma unroll
@@ -671,18 +690,20 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                     *(__nv_bfloat16 *)(sT + sw128_offset(o + r, o + jc, 64)) = __float2bfloat16_rn(col[r]);
                 }
             } else {
-                const int e = tid - 64;  // the other threads zero the upper blocks
-                for (int f = e; f < 512; f += kIntraThreads - 64) {
-                    const int blkz = f >> 8, r = (f >> 4) & 15, cz = f & 15;
-                    const int ro = 32 * blkz, co = 32 * blkz + 16;
-                    Tf[(ro + r) * kLd + co + cz] = 0.f;   // read by the doubling products
-                }
-                for (int f = e; f < 6 * 256; f += kIntraThreads - 64) {
-                    const int bz = f >> 8, r = (f >> 4) & 15, cz = f & 15;
-                    // upper blocks (0,1) (0,2) (0,3) (1,2) (1,3) (2,3) of the bf16 operand
+                // The other 192 threads zero the upper blocks, one 16-byte store each:
+                // (0,1) (0,2) (0,3) (1,2) (1,3) (2,3) of the bf16 operand, 16 rows x 2
+                // chunks of 8 each, and (0,1), (2,3) of the fp32 T that the doubling
+                // products read, 16 rows x 4 float4 each.
+                const int e = tid - 64;
+                {
+                    const int bz = e >> 5, r = (e >> 1) & 15, hf = e & 1;
                     const int bi = bz < 3 ? 0 : bz < 5 ? 1 : 2;
                     const int bj = bz < 3 ? bz + 1 : bz < 5 ? bz - 1 : 3;
-                    *(__nv_bfloat16 *)(sT + sw128_offset(16 * bi + r, 16 * bj + cz, 64)) = __float2bfloat16_rn(0.f);
+                    *(uint4 *)(sT + sw128_offset(16 * bi + r, 16 * bj + 8 * hf, 64)) = make_uint4(0u, 0u, 0u, 0u);
+                }
+                if (e < 128) {
+                    const int blkz = e >> 6, r = (e >> 2) & 15, c4 = e & 3;
+                    *(float4 *)&Tf[(32 * blkz + r) * kLd + 32 * blkz + 16 + 4 * c4] = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
             compute_sync();
@@ -767,41 +788,34 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             }
             {
                 // Rows r = 16 q + i (i < 16) of lane quarter q = w % 4; warps 0-3 read W
-                // (columns 0..127), warps 4-7 read U (columns 128..255).  Each load covers
-                // 64 columns: 32 for each half-warp.  Both are staged in the R area (free
-                // since the inverse) in their block layouts -- W as rows 0..63 of the two
-                // K halves of the [W; Qt] image, U with its row swizzle -- and leave by
-                // three bulk copies.
+                // (columns 0..127) into rows 0..63 of the block's [W; Qt] image, warps
+                // 4-7 read U (columns 128..255) into its row-major block region.  Each
+                // load gives the two threads of a row 16 consecutive columns, so every
+                // store instruction writes whole 32-byte sectors (16 rows x 32 B).
                 const int q = warp & 3, hb = warp >> 2, r = 16 * q + (lane & 15);
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    uint32_t rr[32];
-                    tmem_ld16x2_32(tmem_addr(tb, 32 * q, 128 * hb + 64 * j), rr);
+                for (int m2 = 0; m2 < 8; m2 += 2) {
+                    uint32_t rr[2][8];
+                    tmem_ld16x2_8(tmem_addr(tb, 32 * q, 128 * hb + 16 * m2), rr[0]);
+                    tmem_ld16x2_8(tmem_addr(tb, 32 * q, 128 * hb + 16 * m2 + 16), rr[1]);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int cc = 0; cc < 32; cc += 8) {
+                    for (int u = 0; u < 2; ++u) {
                         const uint4 w4 = make_uint4(
-                            pack_bf16(__uint_as_float(rr[cc]), __uint_as_float(rr[cc + 1])),
-                            pack_bf16(__uint_as_float(rr[cc + 2]), __uint_as_float(rr[cc + 3])),
-                            pack_bf16(__uint_as_float(rr[cc + 4]), __uint_as_float(rr[cc + 5])),
-                            pack_bf16(__uint_as_float(rr[cc + 6]), __uint_as_float(rr[cc + 7])));
-                        const int col = 64 * j + 32 * (lane >> 4) + cc;
+                            pack_bf16(__uint_as_float(rr[u][0]), __uint_as_float(rr[u][1])),
+                            pack_bf16(__uint_as_float(rr[u][2]), __uint_as_float(rr[u][3])),
+                            pack_bf16(__uint_as_float(rr[u][4]), __uint_as_float(rr[u][5])),
+                            pack_bf16(__uint_as_float(rr[u][6]), __uint_as_float(rr[u][7])));
+                        const int col = 16 * (m2 + u) + 8 * (lane >> 4);
                         if (hb == 0)
-                            *(uint4 *)(sm + kIR + sw128_offset(r, col, 64)) = w4;
+                            *(uint4 *)(blk + kOffWQ + sw128_offset(r, col, 128)) = w4;
                         else
-                            *(uint4 *)(sm + kIR + 16384 + u_offset(r, col)) = w4;
+                            *(uint4 *)(blk + kOffU + (r * 128 + col) * 2) = w4;
                     }
                 }
             }
-            fence_proxy_async_smem();
             tc_fence_before_sync();
-            compute_sync();  // TMEM is read out before the next item's products; staging written
-            if (tid == 0) {
-                bulk_s2g(blk + kOffWQ, sm + kIR, 8192);
-                bulk_s2g(blk + kOffWQ + 16384, sm + kIR + 8192, 8192);
-                bulk_s2g(blk + kOffU, sm + kIR + 16384, 16384);
-                bulk_commit();
-            }
+            compute_sync();  // TMEM is read out before the next item's products
             if (sAbort) break;
         }
         if (tid == 0) bulk_wait<0>();  // every staged block region has reached memory
@@ -999,7 +1013,7 @@ state_kernel(const __grid_constant__ CUtensorMap tm_o,
              float *__restrict__ dbg_delta)
 {
     extern __shared__ uint8_t smraw[];
-    uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sm = align_smem_1024(smraw);
     __shared__ StateBars bars;
     __shared__ uint32_t tbase;
 
@@ -1200,7 +1214,7 @@ state_kernel(const __grid_constant__ CUtensorMap tm_o,
             // Dl^T[j][r] = U[r][j] - DW[j][r] for this half's 32 rows -> bf16 pairs into
             // TMEM (U = 0 on the transition).
             {
-                const uint8_t *Ub = st + kOffU;
+                const __nv_bfloat16 *U = (const __nv_bfloat16 *)(st + kOffU);
                 tmem_ld32(tmem_addr(tb, lq, kTDW + 32 * hh), ra);
                 tmem_ld_wait();
                 uint32_t dl[16];
@@ -1212,10 +1226,8 @@ state_kernel(const __grid_constant__ CUtensorMap tm_o,
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
                         const int r = 32 * hh + i;
-                        const float d0 = __bfloat162float(*(const __nv_bfloat16 *)(Ub + u_offset(r, j))) -
-                                         __uint_as_float(ra[i]);
-                        const float d1v = __bfloat162float(*(const __nv_bfloat16 *)(Ub + u_offset(r + 1, j))) -
-                                          __uint_as_float(ra[i + 1]);
+                        const float d0 = __bfloat162float(U[r * kDV + j]) - __uint_as_float(ra[i]);
+                        const float d1v = __bfloat162float(U[(r + 1) * kDV + j]) - __uint_as_float(ra[i + 1]);
                         dl[i >> 1] = pack_bf16(d0, d1v);
                     }
                 }
@@ -1483,7 +1495,7 @@ correct_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ chunk
     if (s == 0) return;              // segment 0 started from the true state
 
     extern __shared__ uint8_t smraw[];
-    uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sm = align_smem_1024(smraw);
     __shared__ uint64_t bar_ld, bar_mma;
     __shared__ uint32_t tbase;
     __shared__ int sOk;
@@ -1604,7 +1616,7 @@ debug_unpack_kernel(const uint8_t *__restrict__ blocks, int64_t max_chunks,
         if (Wout)
             Wout[idx] = __bfloat162float(*(const __nv_bfloat16 *)(blk + kOffWQ + sw128_offset(r, c, 128)));
         if (Uout)
-            Uout[idx] = __bfloat162float(*(const __nv_bfloat16 *)(blk + kOffU + u_offset(r, c)));
+            Uout[idx] = __bfloat162float(((const __nv_bfloat16 *)(blk + kOffU))[r * kDV + c]);
     }
 }
 

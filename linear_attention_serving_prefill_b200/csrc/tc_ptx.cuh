@@ -227,6 +227,18 @@ __device__ __forceinline__ void tmem_ld16x2_32(uint32_t taddr, uint32_t (&r)[32]
         : "r"(taddr));
 }
 
+// 16 lanes x 32 bits in two halves, 8 columns each: thread t < 16 receives lane t
+// of the warp's quarter, columns col .. col + 7; thread t >= 16 receives lane
+// t - 16, columns col + 8 .. col + 15.  The two threads that share a lane hold 16
+// consecutive columns between them.
+__device__ __forceinline__ void tmem_ld16x2_8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], 8;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7])
+        : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
