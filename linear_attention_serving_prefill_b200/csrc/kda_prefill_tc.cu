@@ -730,29 +730,45 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             }
             compute_sync();
             {
-                // Level 2, block rows 32..63 x columns 0..31: columns 4 sb .. 4 sb + 3.
-                const int r = tid >> 3, cb = 4 * (tid & 7);
-                float2 x0 = make_float2(0.f, 0.f), x1 = make_float2(0.f, 0.f);
+                // Level 2, block rows 32..63 x columns 0..31.  Warps 0-3: each thread
+                // computes rows r and r + 16 x columns cb .. cb + 3 of each product, so
+                // that one float4 of the right factor serves two rows (the products are
+                // bound by shared-memory reads).
+                const int r = (tid >> 3) & 15, cb = 4 * (tid & 7);
+                const bool act = tid < 128;
+                if (act) {
+                    float2 x0 = make_float2(0.f, 0.f), x1 = x0, x2 = x0, x3 = x0;
 #pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    const float a = Af[(32 + r) * kLd + t];
-                    const float4 tv = *(const float4 *)&Tf[t * kLd + cb];
-                    x0 = fma2(make_float2(a, a), make_float2(tv.x, tv.y), x0);
-                    x1 = fma2(make_float2(a, a), make_float2(tv.z, tv.w), x1);
+                    for (int t = 0; t < 32; ++t) {
+                        const float a = Af[(32 + r) * kLd + t], a2 = Af[(48 + r) * kLd + t];
+                        const float4 tv = *(const float4 *)&Tf[t * kLd + cb];
+                        const float2 lo = make_float2(tv.x, tv.y), hi = make_float2(tv.z, tv.w);
+                        x0 = fma2(make_float2(a, a), lo, x0);
+                        x1 = fma2(make_float2(a, a), hi, x1);
+                        x2 = fma2(make_float2(a2, a2), lo, x2);
+                        x3 = fma2(make_float2(a2, a2), hi, x3);
+                    }
+                    *(float4 *)&Xf[r * kXLd + cb] = make_float4(x0.x, x0.y, x1.x, x1.y);
+                    *(float4 *)&Xf[(r + 16) * kXLd + cb] = make_float4(x2.x, x2.y, x3.x, x3.y);
                 }
-                *(float4 *)&Xf[r * kXLd + cb] = make_float4(x0.x, x0.y, x1.x, x1.y);
                 compute_sync();
-                float2 y0 = make_float2(0.f, 0.f), y1 = make_float2(0.f, 0.f);
+                if (act) {
+                    float2 y0 = make_float2(0.f, 0.f), y1 = y0, y2 = y0, y3 = y0;
 #pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    const float tt = Tf[(32 + r) * kLd + 32 + t];
-                    const float4 xv = *(const float4 *)&Xf[t * kXLd + cb];
-                    y0 = fma2(make_float2(tt, tt), make_float2(xv.x, xv.y), y0);
-                    y1 = fma2(make_float2(tt, tt), make_float2(xv.z, xv.w), y1);
+                    for (int t = 0; t < 32; ++t) {
+                        const float tt = Tf[(32 + r) * kLd + 32 + t], tt2 = Tf[(48 + r) * kLd + 32 + t];
+                        const float4 xv = *(const float4 *)&Xf[t * kXLd + cb];
+                        const float2 lo = make_float2(xv.x, xv.y), hi = make_float2(xv.z, xv.w);
+                        y0 = fma2(make_float2(tt, tt), lo, y0);
+                        y1 = fma2(make_float2(tt, tt), hi, y1);
+                        y2 = fma2(make_float2(tt2, tt2), lo, y2);
+                        y3 = fma2(make_float2(tt2, tt2), hi, y3);
+                    }
+                    *(uint2 *)(sT + sw128_offset(32 + r, cb, 64)) =
+                        make_uint2(pack_bf16(-y0.x, -y0.y), pack_bf16(-y1.x, -y1.y));
+                    *(uint2 *)(sT + sw128_offset(48 + r, cb, 64)) =
+                        make_uint2(pack_bf16(-y2.x, -y2.y), pack_bf16(-y3.x, -y3.y));
                 }
-                const float4 y = make_float4(y0.x, y0.y, y1.x, y1.y);
-                *(uint2 *)(sT + sw128_offset(32 + r, cb, 64)) =
-                    make_uint2(pack_bf16(-y.x, -y.y), pack_bf16(-y.z, -y.w));
             }
             // The Kd^T and P staging is read out before the next item's loads land on it.
             if (tid == 0) bulk_wait_read<0>();
