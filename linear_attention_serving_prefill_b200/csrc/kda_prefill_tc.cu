@@ -708,25 +708,39 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             }
             compute_sync();
             {
-                // Level 1, blocks (1,0) and (3,2): X = A_ij T_jj, columns 2 sb, 2 sb + 1.
-                const int pb = tid >> 7, r = (tid >> 3) & 15, cb = 2 * (tid & 7);
+                // Level 1, blocks (1,0) and (3,2): X = A_ij T_jj, then T_ij = -T_ii X.
+                // Warps 0-3: thread (pb, r, cb) computes rows r and r + 8 x columns
+                // cb, cb + 1 of block pair pb (one float2 of the right factor per two rows).
+                const int pb = (tid >> 6) & 1, r = (tid >> 3) & 7, cb = 2 * (tid & 7);
                 const int oi = 32 * pb + 16, oj = 32 * pb;
-                float2 x = make_float2(0.f, 0.f);
+                const bool act = tid < 128;
+                if (act) {
+                    float2 x0 = make_float2(0.f, 0.f), x1 = x0;
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const float a = Af[(oi + r) * kLd + oj + t];
-                    x = fma2(make_float2(a, a), *(const float2 *)&Tf[(oj + t) * kLd + oj + cb], x);
+                    for (int t = 0; t < 16; ++t) {
+                        const float a = Af[(oi + r) * kLd + oj + t], a2 = Af[(oi + r + 8) * kLd + oj + t];
+                        const float2 tv = *(const float2 *)&Tf[(oj + t) * kLd + oj + cb];
+                        x0 = fma2(make_float2(a, a), tv, x0);
+                        x1 = fma2(make_float2(a2, a2), tv, x1);
+                    }
+                    *(float2 *)&Xf[(16 * pb + r) * kXLd + cb] = x0;
+                    *(float2 *)&Xf[(16 * pb + r + 8) * kXLd + cb] = x1;
                 }
-                *(float2 *)&Xf[(16 * pb + r) * kXLd + cb] = x;
                 compute_sync();
-                float2 y = make_float2(0.f, 0.f);
+                if (act) {
+                    float2 y0 = make_float2(0.f, 0.f), y1 = y0;
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const float tt = Tf[(oi + r) * kLd + oi + t];
-                    y = fma2(make_float2(tt, tt), *(const float2 *)&Xf[(16 * pb + t) * kXLd + cb], y);
+                    for (int t = 0; t < 16; ++t) {
+                        const float tt = Tf[(oi + r) * kLd + oi + t], tt2 = Tf[(oi + r + 8) * kLd + oi + t];
+                        const float2 xv = *(const float2 *)&Xf[(16 * pb + t) * kXLd + cb];
+                        y0 = fma2(make_float2(tt, tt), xv, y0);
+                        y1 = fma2(make_float2(tt2, tt2), xv, y1);
+                    }
+                    *(float2 *)&Tf[(oi + r) * kLd + oj + cb] = make_float2(-y0.x, -y0.y);
+                    *(float2 *)&Tf[(oi + r + 8) * kLd + oj + cb] = make_float2(-y1.x, -y1.y);
+                    *(uint32_t *)(sT + sw128_offset(oi + r, oj + cb, 64)) = pack_bf16(-y0.x, -y0.y);
+                    *(uint32_t *)(sT + sw128_offset(oi + r + 8, oj + cb, 64)) = pack_bf16(-y1.x, -y1.y);
                 }
-                *(float2 *)&Tf[(oi + r) * kLd + oj + cb] = make_float2(-y.x, -y.y);
-                *(uint32_t *)(sT + sw128_offset(oi + r, oj + cb, 64)) = pack_bf16(-y.x, -y.y);
             }
             compute_sync();
             {
