@@ -103,7 +103,7 @@ def decode_row(steps=1000):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--quick", action="store_true", help="skip the 248K-token varlen workload")
+    ap.add_argument("--quick", action="store_true", help="skip the 193K-token varlen workload")
     args = ap.parse_args()
     rows = []
     rows += prefill_rows("tiny_f32", config_inputs(CONFIGS["tiny_f32"]))
