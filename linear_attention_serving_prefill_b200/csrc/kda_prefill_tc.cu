@@ -604,9 +604,10 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             {
                 // Warp w: lane quarter qd = w % 4 holds rows r = 32 (qd % 2) + lane of A
                 // (qd < 2) or of P (qd >= 2); half hw = w / 4 takes columns s = 32 hw ..
-                // 32 hw + 31 of those rows, 16 at a time.  The two half-warps' rows lie in
-                // different sub-tiles, whose images start at different D columns, so
-                // each group is loaded at both bases and every lane keeps its own.
+                // 32 hw + 31 of those rows, in two groups of 16 whose four loads share
+                // one wait.  The two half-warps' rows lie in different sub-tiles, whose
+                // images start at different D columns, so each group is loaded at both
+                // bases and every lane keeps its own.
                 const int qd = warp & 3, hw = warp >> 2;
                 const int r = 32 * (qd & 1) + lane, Ia = r >> 4;
                 const int I0 = 2 * (qd & 1);
@@ -614,16 +615,19 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 const uint32_t lrow = tmem_addr(tb, 32 * qd, 0);
                 const bool isP = qd >= 2;
                 const float br = sBeta[r];
+                float va2[2][16], vb2[2][16];
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    tmem_ld16f(lrow + nlo + 32 * hw + 16 * g, va2[g]);
+                    tmem_ld16f(lrow + nhi + 32 * hw + 16 * g, vb2[g]);
+                }
+                tmem_ld_wait();
 #pragma unroll
                 for (int g = 0; g < 2; ++g) {
                     const int s0 = 32 * hw + 16 * g;
-                    float va[16], vb[16];
-                    tmem_ld16f(lrow + nlo + s0, va);
-                    tmem_ld16f(lrow + nhi + s0, vb);
-                    tmem_ld_wait();
                     float v[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] = lane < 16 ? va[e] : vb[e];
+                    for (int e = 0; e < 16; ++e) v[e] = lane < 16 ? va2[g][e] : vb2[g][e];
                     if (kSoftplus && 2 * hw + g == Ia) {
                         // The diagonal tile, from the pair kernel: [A | P][I][r][s] per item.
                         const float4 *pa = (const float4 *)(pairs + ((size_t)h * max_chunks + inf.g) * 2048 +
@@ -974,9 +978,11 @@ constexpr uint32_t kStateSmem = kStages * kStageBytes + 2 * 16384 + 1024;
 constexpr uint32_t kTS = 0, kTSbf = 128, kTDl = 256, kTDW = 288, kTDO = 352;  // SB[b] = 128 + 64 b,
                                                                                // DO[b] = 352 + 64 b
 constexpr int kBarOut = 2;  // named barrier id of the output warps
-// L2 prefetch distance of the block stream, in chunks: 96 chains x 6 blocks of
-// 72.5 KiB is about 42 MB of the 126 MB L2.
-constexpr int kPrefetchAhead = 6;
+// L2 prefetch distance of the block stream, in chunks (one ahead of the
+// two-stage ring).  Measured on the 32K x 96-head workload: 0.86 ms at 2 or 3
+// ahead, 0.94 ms at 6 and 1.13 ms at 8; the 96 chains' prefetched blocks crowd
+// the L2 at the longer distances.
+constexpr int kPrefetchAhead = 3;
 
 struct StateBars {
     uint64_t full[kStages], empty[kStages];
