@@ -398,11 +398,15 @@ extern "C" kda_status kda_decode_multi(const void *q, const void *k, const void 
         (num_tokens && !aligned(num_tokens, 4)))
         return KDA_ERR_INVALID_ARG;
 
+    int32_t *status = nullptr;
+    kda_status st = status_word(&status);
+    if (st != KDA_OK) return st;
+
     kda::DecodeMultiArgs a;
     a.q = q; a.k = k; a.v = v; a.z = z; a.A = A; a.beta = beta;
     a.B = B; a.Tq = Tq; a.H = H; a.dk = dk; a.dv = dv; a.bf16 = (dt == KDA_DTYPE_BF16);
     a.state = state; a.slots = slots; a.num_tokens = num_tokens;
-    a.update_state = update_state != 0; a.o = o;
+    a.update_state = update_state != 0; a.o = o; a.status = status;
     cudaError_t err = kda::launch_decode_multi(a, (cudaStream_t)stream);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

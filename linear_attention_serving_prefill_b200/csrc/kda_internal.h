@@ -61,6 +61,7 @@ struct DecodeMultiArgs {
     const int32_t *num_tokens;      // [B] or nullptr (= Tq)
     bool update_state;
     void *o;                        // [B, Tq, H, dv] or nullptr
+    int32_t *status;                // device status word (a wait that gives up records here)
 };
 
 // Tq tokens per sequence on a register-resident state (verify / replay).
