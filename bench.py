@@ -34,6 +34,7 @@ import torch  # noqa: E402
 
 METRIC = "KDA prefill tokens/s + TFLOP/s (H=96,d=128,T=32K); decode-step GB/s vs HBM peak"
 BYTES_PER_TOKEN_HEAD = 1284        # q,k,v,z bf16 (4*256) + beta fp32 (4) + o bf16 (256)
+L2_BYTES = 126 * 1000 * 1000       # B200 L2 (126 MB)
 FLOPS_PER_TOKEN_HEAD = 108544      # 6*dk*dv + 16*(3*dk + 2*dv) at dk = dv = 128
 FALLBACK_HBM_GBS = 6650.0
 # Kernels per prefill call -> (names, algorithmic bytes per token-head of each,
@@ -637,6 +638,9 @@ def main():
             cpu = {"value": r["tokens_per_s"], "unit": "tokens/s", "cores": r["cores"],
                    "kind": "oracle", "sample": r["sample"], "seconds": r["seconds"]}
 
+    in_bytes = sum(inp[key].numel() * inp[key].element_size() for key in ("q", "k", "v", "z"))
+    l2_note = (f"{'inputs larger than' if in_bytes > L2_BYTES else 'inputs SMALLER than'} L2 "
+               f"(q, k, v, z = {in_bytes / 1e9:.2f} GB per step, L2 {L2_BYTES / 1e6:.0f} MB), no flush")
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -646,7 +650,7 @@ def main():
             "config": {"workload": cfg.name, "global_batch": world, "seq_len": T, "heads": H,
                        "dk": dk, "dv": dv, "parallelism": f"dp{world} (one independent problem per GPU)",
                        "algo": args.algo,
-                       "l2": "inputs larger than L2 (q,k,v,z = 3.2 GB per step), no flush"},
+                       "l2": l2_note},
             "tflops": tflops,
             "roofline": roofline,
             "path_roofline": path,
