@@ -418,7 +418,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="prefill_32k", choices=["prefill_32k", "prefill_4k"],
+    ap.add_argument("--workload", default="prefill_32k", choices=["prefill_32k", "prefill_4k", "varlen_resume"],
                     help="prefill_4k is the small case used for profiler captures")
     ap.add_argument("--prefill-only", action="store_true",
                     help="skip the decode, end-to-end and CPU legs (profiler captures)")
@@ -428,6 +428,8 @@ def main():
                     help="sequences of the decode legs (default: the 256-sequence workload)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.workload == "varlen_resume" and (not args.prefill_only or args.impl == "reference"):
+        ap.error("the varlen_resume workload runs the prefill leg alone (--prefill-only)")
     if args.impl == "reference":
         run_reference(args)
         return
@@ -465,20 +467,22 @@ def main():
     from dataclasses import replace
     inp = config_inputs(replace(cfg, seed=rank_seed(cfg.seed, rank)), device=dev)
     T, H, dk, dv = inp["q"].shape[0], cfg.H, cfg.dk, cfg.dv
+    N = inp["cu_seqlens_host"].numel() - 1
+    S0 = inp.get("initial_state")       # resumed sequences start from a cached state
     stream = torch.cuda.current_stream()
     o = torch.empty(T, H, dv, dtype=torch.bfloat16, device=dev)
-    S = torch.empty(1, H, dk, dv, dtype=torch.float32, device=dev)
-    ws_bytes = K.kda_prefill_workspace_size(T, 1, H, dk, dv, torch.bfloat16, args.algo)
+    S = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    ws_bytes = K.kda_prefill_workspace_size(T, N, H, dk, dv, torch.bfloat16, args.algo)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
 
-    nk = K.kda_prefill_kernel_count(T, 1, H, dk, dv, torch.bfloat16, args.algo)
-    n_seg = K.kda_prefill_segments(T, 1, H, dk, dv, torch.bfloat16, args.algo)
+    nk = K.kda_prefill_kernel_count(T, N, H, dk, dv, torch.bfloat16, args.algo)
+    n_seg = K.kda_prefill_segments(T, N, H, dk, dv, torch.bfloat16, args.algo)
     kernel_names, kernel_bytes_per_th, kernel_file = (KERNELS[nk] if nk != 5 else
                                                       split_kernels(n_seg))
 
     def step(events=None):
         K.kda_prefill(inp["q"], inp["k"], inp["v"], inp["z"], inp["A"], inp["beta"],
-                      inp["cu_seqlens"], inp["cu_seqlens_host"], None, final_state=S, o=o,
+                      inp["cu_seqlens"], inp["cu_seqlens_host"], S0, final_state=S, o=o,
                       workspace=ws, algo=args.algo, stream=stream, stage_events=events)
 
     for _ in range(args.warmup):
@@ -517,7 +521,10 @@ def main():
     # o out) over the dominant kernel's launch time.  The bytes that kernel
     # moves by this design (its own reads plus the intermediate block it
     # writes) are reported beside it under "own_bytes_*", not in "frac".
-    alg_bytes = th * BYTES_PER_TOKEN_HEAD
+    # With initial states the 64 KiB state of every (sequence, head) is read and
+    # the final one written: 2 x 64 KiB more per (sequence, head).
+    state_bytes = 2 * N * H * dk * dv * 4 if S0 is not None else 0
+    alg_bytes = th * BYTES_PER_TOKEN_HEAD + state_bytes
     achieved = alg_bytes / (launch_ms / 1e3) / 1e9
     own_bytes = th * kernel_bytes_per_th[dom]
     own_gbs = own_bytes / (launch_ms / 1e3) / 1e9
@@ -530,11 +537,12 @@ def main():
                 "own_bytes_per_token_head": kernel_bytes_per_th[dom],
                 "own_bytes_gbs": own_gbs, "own_bytes_frac": own_gbs / hbm_peak,
                 "kernels_ms": dict(zip(kernel_names, per_kernel_ms))}
-    path_gbs = th * BYTES_PER_TOKEN_HEAD / (ms_per_step / 1e3) / 1e9
-    path = {"bytes_per_token_head": BYTES_PER_TOKEN_HEAD, "achieved_gbs": path_gbs,
+    path_gbs = alg_bytes / (ms_per_step / 1e3) / 1e9
+    path = {"bytes_per_token_head": BYTES_PER_TOKEN_HEAD, "state_bytes": state_bytes,
+            "achieved_gbs": path_gbs,
             "hbm_frac": path_gbs / hbm_peak, "tensor_tflops": tflops / world,
             "tensor_frac": tflops / world / tc_peak, "tensor_peak": tc_peak,
-            "roofline_ms": th * BYTES_PER_TOKEN_HEAD / hbm_peak / 1e6}
+            "roofline_ms": alg_bytes / hbm_peak / 1e6}
     launches = args.steps * nk
 
     decode = e2e = cpu = ckpt = split = gate_cost = None
@@ -647,7 +655,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": cfg.name, "global_batch": world, "seq_len": T, "heads": H,
+            "config": {"workload": cfg.name, "global_batch": N * world, "seq_len": T, "heads": H,
                        "dk": dk, "dv": dv, "parallelism": f"dp{world} (one independent problem per GPU)",
                        "algo": args.algo,
                        "l2": l2_note},
