@@ -377,7 +377,11 @@ kda_status kda_decode_step_gated(const void *q, const void *k, const void *v, co
  *                each sequence is advanced by its num_tokens[b] tokens in place
  *                (o is written too when non-NULL).
  *   o            [B, Tq, H, dv] dtype dt, or NULL (then update_state must be 1).
- * Tq in [1, 64].  Errors as kda_decode_step.
+ * Tq in [1, 64].  Errors as kda_decode_step.  The kernel copies each state into
+ * on-chip memory with the copy engine and waits for it with a 2 s limit; a wait
+ * that gives up records KDA_ERR_TIMEOUT in the device status word
+ * (kda_device_status) and the launch ends without writing that state.  Two
+ * sequences must not share a slot when update_state is 1.
  */
 kda_status kda_decode_multi(const void *q, const void *k, const void *v, const void *z,
                             const float *A, const float *beta, int32_t B, int32_t Tq, int32_t H,

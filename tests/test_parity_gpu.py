@@ -607,3 +607,42 @@ def test_spec_full_batch_verify_then_replay():
     assert relerr(to_np(st), to_np(st_steps)) <= 1e-6
     for t in range(Tq):
         assert relerr(to_np(ov[:, t]), to_np(outs[t])) <= 1e-2
+
+
+@pytest.mark.parametrize("dk,dv,B", [(128, 128, 100), (64, 32, 1300)])
+def test_spec_persistent_ctas_two_groups(dk, dv, B):
+    """More (sequence, head) items than resident CTAs, so every CTA walks several
+    items (state copy and first-group prefetch of the next item during the
+    current one), with 11 drafts (a second token group fetched from global
+    memory), random slots and accepted counts including 0 and all: verify
+    outputs and replayed states against the oracle."""
+    H, Tq = 4, 11
+    P = B + 7
+    x, s, state, slots = _spec_inputs(B, Tq, H, dk, dv, "bf16", 64 + dk, P)
+    before = state.clone()
+    o = K.kda_decode_multi(s["q"], s["k"], s["v"], s["z"], x["A"].cuda(), s["beta"], state, slots)
+    torch.cuda.synchronize()
+    assert torch.equal(state, before)
+    s0 = before[slots.long()].cpu()
+    ref_o, _ = oracle.prefill(x["q"], x["k"], x["v"], x["z"], x["A"], x["beta"], x["cu_seqlens_host"], s0)
+    assert relerr(to_np(o).reshape(B * Tq, H, dv), ref_o) <= TOL_BF16
+
+    g = torch.Generator().manual_seed(dk + dv)
+    acc = torch.randint(0, Tq + 1, (B,), generator=g).to(torch.int32)
+    acc[0], acc[1], acc[2] = 0, Tq, 8
+    K.kda_decode_multi(s["q"], s["k"], s["v"], s["z"], x["A"].cuda(), s["beta"], state, slots,
+                       num_tokens=acc.cuda(), update_state=True, want_outputs=False)
+    torch.cuda.synchronize()
+    sl = slots.long().cpu()
+    untouched = sorted(set(range(P)) - set(sl.tolist()))
+    assert torch.equal(state[untouched], before[untouched])
+    for b in list(range(6)) + list(range(B - 3, B)):
+        a = int(acc[b])
+        if a == 0:
+            assert torch.equal(state[sl[b]], before[sl[b]])
+            continue
+        tok = slice(b * Tq, b * Tq + a)
+        _, ref_S = oracle.prefill(*(x[key][tok] for key in ("q", "k", "v", "z")), x["A"],
+                                  x["beta"][tok], np.array([0, a], np.int32),
+                                  before[sl[b]].cpu()[None])
+        assert relerr(to_np(state[sl[b]]), ref_S[0]) <= TOL_BF16
