@@ -103,3 +103,14 @@ def test_reference_arm_other_ranks_print_nothing():
                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
     assert out.returncode == 0, out.stderr[-2000:]
     assert not [l for l in out.stdout.splitlines() if l.startswith("{")]
+
+
+@pytest.mark.parametrize("extra", [[], ["--impl", "reference", "--prefill-only"]])
+def test_varlen_workload_is_prefill_only(extra):
+    """The 16-sequence resume workload times the prefill leg alone; asking for the
+    other legs (or the reference arm) is refused on the host before any work."""
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--workload", "varlen_resume",
+                          "--steps", "1"] + extra,
+                         cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 2
+    assert "varlen_resume workload runs the prefill leg alone" in out.stderr
