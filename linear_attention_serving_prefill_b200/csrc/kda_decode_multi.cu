@@ -12,10 +12,12 @@
 //     not written, so a rejected draft leaves no trace;
 //   * replay (update_state = 1): the first num_tokens[b] tokens advance the state,
 //     which is written back in place once.
-// Persistent CTAs of 2 dv threads walk the (sequence, head) items; two fit on an
-// SM.  While a CTA runs an item's tokens from registers, one bulk copy brings
-// the next item's state (dk x dv fp32, contiguous in HBM) into shared memory, so
-// the state stream overlaps the token arithmetic instead of alternating with it.
+// Persistent CTAs of 2 dv threads walk the (sequence, head) items, as many as
+// fit on an SM (two at dk = dv = 128).  While a CTA runs an item's tokens from
+// registers, one bulk copy brings the next item's state (dk x dv fp32,
+// contiguous in HBM) into shared memory and cp.async brings the rows of its
+// first kGroup tokens, so the state stream and the input fetch overlap the token
+// arithmetic instead of alternating with it.
 // Warp w owns the 16 value columns 16 w .. 16 w + 15 (four float4 column groups)
 // for all dk rows: lane (rg, c4) = (lane / 4, lane % 4) holds rows rg, rg + 8,
 // ... of column group 4 w + c4 in registers.  Columns of S never mix, so every
