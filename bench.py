@@ -39,11 +39,13 @@ FLOPS_PER_TOKEN_HEAD = 108544      # 6*dk*dv + 16*(3*dk + 2*dv) at dk = dv = 128
 FALLBACK_HBM_GBS = 6650.0
 # Kernels per prefill call -> (names, algorithmic bytes per token-head of each,
 # source file).  Tensor-core path: the intra kernel reads q, k, v, z (bf16) and
-# beta and writes a 74,240-byte block per (64-token chunk, head), i.e. 1,160 B
+# beta and writes a 74,496-byte block per (64-token chunk, head), i.e. 1,164 B
 # per token-head; the state kernel reads that block and writes o (bf16).
+BLOCK_BYTES_PER_TOKEN_HEAD = 74496 // 64
 KERNELS = {
     1: (["prefill_cuda_core_kernel"], [BYTES_PER_TOKEN_HEAD], "kda_prefill_cuda_core.cu"),
-    3: (["plan_kernel", "intra_kernel", "state_kernel"], [0, 1028 + 1160, 1160 + 256],
+    3: (["plan_kernel", "intra_kernel", "state_kernel"],
+        [0, 1028 + BLOCK_BYTES_PER_TOKEN_HEAD, BLOCK_BYTES_PER_TOKEN_HEAD + 256],
         "kda_prefill_tc.cu"),
 }
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -58,7 +60,8 @@ def split_kernels(G: int):
     The segment composition moves O(N H G) states, nothing per token."""
     f = (G - 1) / G
     return (["plan_kernel", "intra_kernel", "state_kernel", "compose_kernel", "correct_kernel"],
-            [0, 1028 + 1160, 1160 * (1 + f) + 256 + 256 * f, 0, 768 * f], "kda_prefill_tc.cu")
+            [0, 1028 + BLOCK_BYTES_PER_TOKEN_HEAD, BLOCK_BYTES_PER_TOKEN_HEAD * (1 + f) + 256 + 256 * f, 0,
+             768 * f], "kda_prefill_tc.cu")
 
 
 def _peaks():

@@ -61,9 +61,19 @@ constexpr uint64_t kWaitNs = 2000000000ull;  // per-wait limit: 2 s
 constexpr uint32_t kOffWQ = 0;         // [W; Qt] 128 rows x 128 K, swizzled K-major
 constexpr uint32_t kOffKd = 32768;     // Kd^T 128 rows (key channel) x 64 K (token)
 constexpr uint32_t kOffP = 49152;      // P 64 rows x 64 K
-constexpr uint32_t kOffU = 57344;      // U row-major [64][128] bf16
-constexpr uint32_t kOffDecay = 73728;  // e^{G_C} [128] fp32
-constexpr uint32_t kBlockBytes = 74240;
+constexpr uint32_t kOffU = 57344;      // U [64][128] bf16 in 16-channel blocks (u_offset)
+constexpr uint32_t kOffDecay = 73984;  // e^{G_C} [128] fp32
+constexpr uint32_t kBlockBytes = 74496;
+// U element (r, j): blocks of 16 channels, 32 B per row within a block, blocks
+// 2080 B apart.  Each store of the intra kernel's readback (16 rows x 16
+// channels) then fills 512 contiguous bytes instead of 16 separate 32-byte
+// pieces, and the 32-byte skew between blocks (2080 = 16 x 128 + 32) puts the
+// two blocks that a state-kernel warp reads for one row (32 channels) on
+// different shared-memory banks.
+constexpr uint32_t kUBlock = 2080;
+__host__ __device__ __forceinline__ uint32_t u_offset(uint32_t r, uint32_t j) {
+    return (j >> 4) * kUBlock + r * 32u + (j & 15u) * 2u;
+}
 
 // The dynamic shared memory rounded up to a 1024-byte boundary (the 128-byte
 // swizzle's period).  The offset is added to the __shared__ pointer itself, not
@@ -823,9 +833,10 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             {
                 // Rows r = 16 q + i (i < 16) of lane quarter q = w % 4; warps 0-3 read W
                 // (columns 0..127) into rows 0..63 of the block's [W; Qt] image, warps
-                // 4-7 read U (columns 128..255) into its row-major block region.  Each
-                // load gives the two threads of a row 16 consecutive columns, so every
-                // store instruction writes whole 32-byte sectors (16 rows x 32 B).
+                // 4-7 read U (columns 128..255) into its block region.  Each load gives
+                // the two threads of a row 16 consecutive columns, so every store
+                // instruction writes whole 32-byte sectors (16 rows x 32 B); for U those
+                // are 512 contiguous bytes (u_offset).
                 const int q = warp & 3, hb = warp >> 2, r = 16 * q + (lane & 15);
 #pragma unroll
                 for (int m2 = 0; m2 < 8; m2 += 2) {
@@ -844,7 +855,7 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                         if (hb == 0)
                             *(uint4 *)(blk + kOffWQ + sw128_offset(r, col, 128)) = w4;
                         else
-                            *(uint4 *)(blk + kOffU + (r * 128 + col) * 2) = w4;
+                            *(uint4 *)(blk + kOffU + u_offset(r, col)) = w4;
                     }
                 }
             }
@@ -1250,7 +1261,7 @@ state_kernel(const __grid_constant__ CUtensorMap tm_o,
             // Dl^T[j][r] = U[r][j] - DW[j][r] for this half's 32 rows -> bf16 pairs into
             // TMEM (U = 0 on the transition).
             {
-                const __nv_bfloat16 *U = (const __nv_bfloat16 *)(st + kOffU);
+                const uint8_t *Uj = st + kOffU + u_offset(0, j);   // U[r][j] at Uj + 32 r
                 tmem_ld32(tmem_addr(tb, lq, kTDW + 32 * hh), ra);
                 tmem_ld_wait();
                 uint32_t dl[16];
@@ -1262,8 +1273,10 @@ state_kernel(const __grid_constant__ CUtensorMap tm_o,
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
                         const int r = 32 * hh + i;
-                        const float d0 = __bfloat162float(U[r * kDV + j]) - __uint_as_float(ra[i]);
-                        const float d1v = __bfloat162float(U[(r + 1) * kDV + j]) - __uint_as_float(ra[i + 1]);
+                        const float d0 = __bfloat162float(*(const __nv_bfloat16 *)(Uj + 32 * r)) -
+                                         __uint_as_float(ra[i]);
+                        const float d1v = __bfloat162float(*(const __nv_bfloat16 *)(Uj + 32 * (r + 1))) -
+                                          __uint_as_float(ra[i + 1]);
                         dl[i >> 1] = pack_bf16(d0, d1v);
                     }
                 }
@@ -1652,7 +1665,7 @@ debug_unpack_kernel(const uint8_t *__restrict__ blocks, int64_t max_chunks,
         if (Wout)
             Wout[idx] = __bfloat162float(*(const __nv_bfloat16 *)(blk + kOffWQ + sw128_offset(r, c, 128)));
         if (Uout)
-            Uout[idx] = __bfloat162float(((const __nv_bfloat16 *)(blk + kOffU))[r * kDV + c]);
+            Uout[idx] = __bfloat162float(*(const __nv_bfloat16 *)(blk + kOffU + u_offset(r, c)));
     }
 }
 

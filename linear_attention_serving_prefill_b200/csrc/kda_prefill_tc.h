@@ -17,7 +17,7 @@ namespace kda {
 // segment must keep 16 chunks of 64 tokens on average.  `forced` gives G >= 2.
 int tc_split_segments(int32_t total_tokens, int32_t num_seqs, int32_t H, bool forced);
 
-// Workspace bytes of the tensor-core path: the chunk plan plus one 74,240-byte
+// Workspace bytes of the tensor-core path: the chunk plan plus one 74,496-byte
 // block of MMA-ready tiles per (chunk, head), for the worst case of
 // floor((T + 63 N) / 64) chunks; with segments > 1 also the segment states,
 // transitions, S_in images (N G H of each) and 16 KiB E images per (chunk, head).
