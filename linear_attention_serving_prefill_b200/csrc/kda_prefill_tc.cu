@@ -59,7 +59,7 @@ constexpr uint64_t kWaitNs = 2000000000ull;  // per-wait limit: 2 s
 
 // Per (chunk, head) block written by the intra kernel, read by the state kernel.
 constexpr uint32_t kOffWQ = 0;         // [W; Qt] 128 rows x 128 K, swizzled K-major
-constexpr uint32_t kOffKd = 32768;     // Kd^T 128 rows (key channel) x 64 K (token)
+constexpr uint32_t kOffKd = 32768;     // Kd^T 128 rows (key channel) x 64 K (token), no swizzle (kd_offset)
 constexpr uint32_t kOffP = 49152;      // P 64 rows x 64 K
 constexpr uint32_t kOffU = 57344;      // U [64][128] bf16 in 16-channel blocks (u_offset)
 constexpr uint32_t kOffDecay = 73984;  // e^{G_C} [128] fp32
@@ -73,6 +73,14 @@ constexpr uint32_t kBlockBytes = 74496;
 constexpr uint32_t kUBlock = 2080;
 __host__ __device__ __forceinline__ uint32_t u_offset(uint32_t r, uint32_t j) {
     return (j >> 4) * kUBlock + r * 32u + (j & 15u) * 2u;
+}
+// Kd^T element (channel c, token t): K-major without swizzle, 8-channel x
+// 16-byte core matrices (channels 16 B apart, SBO = 128 B), 8-token groups
+// 2048 B apart (LBO).  A warp's store of 32 channels x 8 tokens then covers 8
+// lines instead of 32.
+constexpr uint32_t kKdLbo = 2048, kKdSbo = 128;
+__host__ __device__ __forceinline__ uint32_t kd_offset(uint32_t c, uint32_t t) {
+    return (t >> 3) * kKdLbo + c * 16u + (t & 7u) * 2u;
 }
 
 // The dynamic shared memory rounded up to a 1024-byte boundary (the 128-byte
@@ -578,8 +586,8 @@ intra_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 const int kk = 8 * b;
                 *(uint4 *)(sm + kRawV + sw128_offset(c0, kk, 128)) = make_uint4(pk0[0], pk0[1], pk0[2], pk0[3]);
                 *(uint4 *)(sm + kRawV + sw128_offset(c0 + 1, kk, 128)) = make_uint4(pk1[0], pk1[1], pk1[2], pk1[3]);
-                *(uint4 *)(blk + kOffKd + sw128_offset(c0, kk, 128)) = make_uint4(kd0[0], kd0[1], kd0[2], kd0[3]);
-                *(uint4 *)(blk + kOffKd + sw128_offset(c0 + 1, kk, 128)) = make_uint4(kd1[0], kd1[1], kd1[2], kd1[3]);
+                *(uint4 *)(blk + kOffKd + kd_offset(c0, kk)) = make_uint4(kd0[0], kd0[1], kd0[2], kd0[3]);
+                *(uint4 *)(blk + kOffKd + kd_offset(c0 + 1, kk)) = make_uint4(kd1[0], kd1[1], kd1[2], kd1[3]);
             }
 
             // A/P product, one M = 128, N = 160 product over both K halves:
@@ -1159,7 +1167,7 @@ state_kernel(const __grid_constant__ CUtensorMap tm_o,
             }
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                dK[ks] = desc_kmajor_sw128(st + kOffKd + ks * 32);
+                dK[ks] = desc_kmajor_none(st + kOffKd + kd_offset(0, 16 * ks), kKdLbo, kKdSbo);
                 dP[ks] = desc_kmajor_sw128(st + kOffP + ks * 32);
             }
             // DW = S_in^T W^T: needs the block and S_in(c) in bf16.

@@ -312,6 +312,15 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
            ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
 }
 
+// Shared-memory matrix descriptor for a K-major operand with no swizzle: 8-row x
+// 16-byte core matrices stored contiguously (rows 16 B apart), core matrices
+// `sbo` bytes apart along M/N (the next 8 rows) and `lbo` bytes apart along K
+// (the next 8 elements).  Layout type 0 [61,64); other fields as above.
+__device__ __forceinline__ uint64_t desc_kmajor_none(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1u << 46);
+}
+
 // Instruction descriptor, kind::f16 with bf16 A and B (both K-major) and an
 // fp32 accumulator: D format [4,6) = 1, A format [7,10) = 1, B format
 // [10,13) = 1, N >> 3 at [17,23), M >> 4 at [24,29).
