@@ -55,7 +55,7 @@ extern "C" {
 typedef enum {
     KDA_OK = 0,
     KDA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, bad cu_seqlens */
-    KDA_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement (e.g. dk=96) */
+    KDA_ERR_UNSUPPORTED = 2,   /* valid request the library does not implement (e.g. dk=96) */
     KDA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than kda_prefill_workspace_size */
     KDA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
     KDA_ERR_TIMEOUT = 5        /* a bounded on-device wait gave up (see kda_device_status) */
